@@ -1,0 +1,254 @@
+/*
+ * staple.h -- C ABI of the STAPLE embedding-augmented SwiGLU FFN layer on
+ * NVIDIA B200 (sm_100a).
+ *
+ * The layer (paper: "STAPLE: Static Sparse Upcycling of Pretrained
+ * Checkpoints via Embedding Modules", arXiv 2610.12599; abstract, and the
+ * ai4snews summary's Interpretation section) keeps the pretrained SwiGLU FFN
+ * and adds a token-indexed row of a vocab x d_ff table E to the output of the
+ * up-projection:
+ *
+ *     g = W_gate x,  u = W_up x,  h = u + E[id],  z = SiLU(g) * h,  y = W_down z
+ *
+ * E starts at zero, which gives back the dense FFN exactly.  The tables live
+ * in host DRAM, the ~5% most frequent rows are cached in HBM, only the rows of
+ * the batch's distinct ids reach the GPU, and the table gradient exists for
+ * those rows only (abstract; thelatestinai listing, Figure 4 caption and the
+ * retrieval-path table; AI Radio episode, paper summary).
+ *
+ * Conventions for every call below
+ *  - Every function returns a staple_status; nothing else crosses the ABI.
+ *  - Device work is asynchronous on the caller's stream (a cudaStream_t passed
+ *    as staple_stream; NULL = the legacy default stream).  Errors detected on
+ *    the device (an id >= V, a kernel wait that ran out of time) are recorded
+ *    in the context's device error word; staple_get_error() reads it.
+ *  - The caller owns every tensor.  The library allocates device memory only
+ *    in staple_context_create, staple_table_register (flag DEVICE_COPY) and
+ *    staple_cache_build; the per-step calls allocate nothing and take scratch
+ *    from a caller workspace sized by staple_workspace_bytes().
+ *  - Pointers are device pointers unless the argument says "host".
+ *    Matrices are row-major and dense (leading dimension = row length).
+ *    bf16 tensors are passed as raw 16-bit storage.
+ *  - Data-dependent counts (U distinct ids, the miss count) are written to
+ *    device int32 words, so the host never waits inside a step; outputs whose
+ *    length depends on them are sized for the capacity T.
+ */
+#ifndef STAPLE_H
+#define STAPLE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define STAPLE_ABI_VERSION 1
+
+typedef struct CUstream_st* staple_stream; /* same handle as cudaStream_t */
+
+typedef enum staple_status {
+  STAPLE_OK = 0,
+  STAPLE_EINVAL = -1,       /* bad argument: null pointer, size, alignment, flags */
+  STAPLE_EIDRANGE = -2,     /* (device-detected) a token id was outside [0, V) */
+  STAPLE_ECUDA = -3,        /* a CUDA runtime call failed */
+  STAPLE_ENOMEM = -4,       /* device or pinned-host allocation failed */
+  STAPLE_ETIMEOUT = -5,     /* (device-detected) a bounded kernel wait ran out */
+  STAPLE_EUNSUPPORTED = -6, /* valid request this build does not implement */
+  STAPLE_ENODEV = -7        /* no usable sm_100 device */
+} staple_status;
+
+typedef enum staple_dtype {
+  STAPLE_BF16 = 0, /* bf16 storage, fp32 accumulation, tcgen05 tensor cores */
+  STAPLE_F32 = 1   /* fp32 storage and arithmetic (CUDA cores) */
+} staple_dtype;
+
+typedef struct staple_context staple_context;
+typedef struct staple_table staple_table;
+typedef struct staple_cache staple_cache;
+
+/* ---------------------------------------------------------------- context */
+
+/* ABI version compiled into the library (STAPLE_ABI_VERSION). */
+int staple_abi_version(void);
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char* staple_status_string(staple_status s);
+
+/* Create a context on `device` (makes it current for the calling thread).
+ * Allocates the 4-byte device error word.  EINVAL if out == NULL, ENODEV if
+ * the device is not compute capability 10.x. */
+staple_status staple_context_create(int device, staple_context** out);
+
+/* Free the context.  NULL is accepted. */
+staple_status staple_context_destroy(staple_context* ctx);
+
+/* Synchronize `stream`, copy the device error word to *device_error (a
+ * staple_status value: STAPLE_OK when no kernel reported an error) and clear
+ * it.  The only call that waits for the device. */
+staple_status staple_get_error(staple_context* ctx, staple_stream stream, int32_t* device_error);
+
+/* ------------------------------------------------------------------ tables */
+
+#define STAPLE_TABLE_DEVICE 1u        /* `base` is device memory (the whole table in HBM) */
+#define STAPLE_TABLE_HOST_PINNED 2u   /* `base` is pinned, mapped host memory (cudaHostAlloc) */
+#define STAPLE_TABLE_HOST_REGISTER 4u /* `base` is pageable host memory: page-lock and map it
+                                         (cudaHostRegister) until staple_table_unregister */
+
+/* Describe a table of V rows.  Each row holds `groups` adjacent layers'
+ * d_ff-wide rows back to back (token-major grouping of adjacent tables:
+ * thelatestinai listing, retrieval-path table, Decode row), so the element
+ * (v, layer-in-group l, f) sits at base[(v * groups + l) * F + f].
+ * `bytes` must be >= V * groups * F * sizeof(dtype).  Exactly one location
+ * flag.  The caller keeps ownership of `base`.  EINVAL on a bad argument,
+ * ECUDA if registration fails. */
+staple_status staple_table_register(staple_context* ctx, void* base, size_t bytes, int64_t V,
+                                    int32_t F, int32_t groups, staple_dtype dtype, uint32_t flags,
+                                    staple_table** out);
+
+/* Undo staple_table_register (unregisters host memory it registered). */
+staple_status staple_table_unregister(staple_table* table);
+
+/* ------------------------------------------------------------------- cache */
+
+/* Frequency-aware hot-row cache (abstract: about 5% of the embeddings cached
+ * on the GPU; AI Radio episode: 5-6% of the vocabulary, ~80% hit rate).
+ * Chooses the K = ceil(frac * V) rows with the largest freq[v] (ties: smaller
+ * id first; slot k = rank k), allocates K * groups * F elements of HBM, copies
+ * those rows from the table, and builds an open-addressing id -> slot hash
+ * (capacity: the next power of two >= 2K).  `freq` is a host array of V
+ * counts.  frac in [0, 1]; frac = 0 gives an empty cache (every lookup
+ * misses).  Synchronizes `stream` before returning. */
+staple_status staple_cache_build(staple_context* ctx, const staple_table* table,
+                                 const int64_t* freq, double frac, staple_stream stream,
+                                 staple_cache** out);
+
+/* Number of cached rows and hash capacity. */
+staple_status staple_cache_info(const staple_cache* cache, int32_t* K, int32_t* hash_capacity);
+
+/* Copy the cached ids in slot order into the host array hot_ids[K]. */
+staple_status staple_cache_hot_ids(const staple_cache* cache, int32_t* hot_ids);
+
+/* Device address of the cache rows ([K][groups * F], table dtype). */
+staple_status staple_cache_rows(const staple_cache* cache, const void** rows);
+
+staple_status staple_cache_free(staple_cache* cache);
+
+/* --------------------------------------------------------------- workspace */
+
+/* Bytes of caller-owned device scratch the per-step calls need for T tokens,
+ * d_model D, d_ff F (flags reserved, pass 0).  A workspace of this size (or
+ * larger), 256-byte aligned, may be reused by every call with the same or
+ * smaller sizes, one call at a time per workspace. */
+size_t staple_workspace_bytes(int32_t T, int32_t D, int32_t F, uint32_t flags);
+
+/* ------------------------------------------------------- retrieval (K1..K4) */
+
+/* Deduplicate the batch's token ids once; the inverse map serves every
+ * augmented layer (retrieval-path table, Prefill row).
+ *   ids[T]          token ids, each in [0, V)
+ *   unique[T]       out: the U distinct ids ascending (entries >= U untouched)
+ *   inverse[T]      out: unique[inverse[i]] == ids[i]
+ *   seg_off[T+1]    out: tokens with id unique[j] are
+ *                        sorted_pos[seg_off[j] .. seg_off[j+1]-1]; entries > U untouched
+ *   sorted_pos[T]   out: token positions ordered by (id, position)
+ *   U_dev           out: U (device int32)
+ * T in [0, 32768] and V in [1, 2^31).  An id outside [0, V) sets the error
+ * word to STAPLE_EIDRANGE (outputs are then unspecified).  Radix sort by id
+ * with warp-ballot run detection, one thread block. */
+staple_status staple_dedup(staple_context* ctx, const int32_t* ids, int32_t T, int64_t V,
+                           int32_t* unique, int32_t* inverse, int32_t* seg_off,
+                           int32_t* sorted_pos, int32_t* U_dev, staple_stream stream);
+
+/* Rows of the batch's distinct ids, reusing a dedup: probe the hot-row cache
+ * per distinct id (slot[j] = cache slot or -1), list the misses
+ * (miss_list[0..miss_count) = positions j in unique order), copy hit rows from
+ * the cache on `stream`, and read miss rows straight from the mapped host
+ * table with 16-byte loads on `side` (which then waits for `stream` first and
+ * makes `stream` wait for it at the end; pass side = stream to serialise).
+ * rows[T][groups * F] receives row j of the batch at rows[j]; all of a row's
+ * grouped layers are fetched together.  cache may be NULL (all misses); a
+ * DEVICE table needs no cache (all rows read from HBM). */
+staple_status staple_gather_unique_rows(staple_context* ctx, const staple_cache* cache,
+                                        const staple_table* table, const int32_t* unique,
+                                        const int32_t* U_dev, int32_t T, int32_t* slot,
+                                        int32_t* miss_list, int32_t* miss_count, void* rows,
+                                        staple_stream stream, staple_stream side);
+
+/* staple_dedup followed by staple_gather_unique_rows (ids -> unique/inverse,
+ * hit/miss map, U rows). */
+staple_status staple_gather_rows(staple_context* ctx, const staple_cache* cache,
+                                 const staple_table* table, const int32_t* ids, int32_t T,
+                                 int32_t* unique, int32_t* inverse, int32_t* seg_off,
+                                 int32_t* sorted_pos, int32_t* U_dev, int32_t* slot,
+                                 int32_t* miss_list, int32_t* miss_count, void* rows,
+                                 staple_stream stream, staple_stream side);
+
+/* ------------------------------------------------------------ FFN forward */
+
+typedef enum staple_embed_mode {
+  STAPLE_EMBED_NONE = 0,  /* dense FFN: h = u (the E path disabled) */
+  STAPLE_EMBED_TABLE = 1, /* h = u + base[index[t] * row_pitch + f], index = token ids,
+                             n_rows = V (ids checked against it); a table in HBM */
+  STAPLE_EMBED_ROWS = 2   /* h = u + base[index[t] * row_pitch + f], index = inverse map,
+                             base = gathered rows; n_rows = capacity */
+} staple_embed_mode;
+
+typedef struct staple_embed {
+  int32_t mode;          /* staple_embed_mode */
+  int32_t reserved;
+  const void* base;      /* device; points at this layer's first element (group offset applied) */
+  int64_t row_pitch;     /* elements between consecutive rows (groups * F) */
+  const int32_t* index;  /* device [T] */
+  int64_t n_rows;        /* rows addressable through index */
+} staple_embed;
+
+/* Forward pass of one layer.
+ *   x[T][D], w_gate[F][D], w_up[F][D], w_down[D][F]   inputs (dtype)
+ *   z[T][F]     out: SiLU(g) * h, the down projection's input (kept for dW_down)
+ *   y[T][D]     out: layer output
+ *   g_save, h_save [T][F]  out (training): g and h for the backward pass;
+ *               both NULL for inference
+ * bf16 needs D and F multiples of 64 and 16-byte aligned pointers;
+ * T >= 0.  fp32 accepts any sizes. */
+staple_status staple_ffn_fwd(staple_context* ctx, staple_dtype dtype, int32_t T, int32_t D,
+                             int32_t F, const void* x, const staple_embed* embed,
+                             const void* w_gate, const void* w_up, const void* w_down, void* z,
+                             void* y, void* g_save, void* h_save, void* workspace,
+                             size_t workspace_bytes, staple_stream stream);
+
+/* ----------------------------------------------------------- FFN backward */
+
+/* Table gradient of one layer (spec call: dY -> U gradient rows).
+ * Computes dz = dY W_down, dh = dz * SiLU(g), dg = dz * h * SiLU'(g) into
+ * dgh[T][2F] (dg in columns [0, F), dh in [F, 2F)), then
+ *   dE[j][f] = sum of dh[i][f] over the tokens i of segment j (seg_off /
+ *              sorted_pos from staple_dedup), accumulated in fp32 in
+ *              ascending token position, for j < U (U read from U_dev).
+ * dE is fp32 [T][F] (capacity T rows; rows >= U untouched).  With
+ * dE == NULL only dgh is produced (the dense run). */
+staple_status staple_embed_bwd(staple_context* ctx, staple_dtype dtype, int32_t T, int32_t D,
+                               int32_t F, const void* dy, const void* g_save, const void* h_save,
+                               const void* w_down, const int32_t* sorted_pos,
+                               const int32_t* inverse, const int32_t* seg_off,
+                               const int32_t* U_dev, void* dgh, float* dE, void* workspace,
+                               size_t workspace_bytes, staple_stream stream);
+
+/* Rest of the layer backward, consuming dgh from staple_embed_bwd:
+ *   dx[T][D]       = dg W_gate + dh W_up                      (dtype)
+ *   dw_gate[F][D]  = sum_t dg_t x_t^T       (fp32; NULL: not computed)
+ *   dw_up[F][D]    = sum_t dh_t x_t^T       (fp32; NULL: frozen up-projection,
+ *                    the warmup recipe of the ai4snews summary, Interpretation)
+ *   dw_down[D][F]  = sum_t dY_t z_t^T       (fp32; NULL: not computed)
+ * Gradients are written, not accumulated. */
+staple_status staple_ffn_bwd(staple_context* ctx, staple_dtype dtype, int32_t T, int32_t D,
+                             int32_t F, const void* dy, const void* x, const void* z,
+                             const void* dgh, const void* w_gate, const void* w_up, void* dx,
+                             float* dw_gate, float* dw_up, float* dw_down, void* workspace,
+                             size_t workspace_bytes, staple_stream stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* STAPLE_H */

@@ -1,0 +1,73 @@
+"""The C-ABI library loads and exports every entry point include/staple.h
+declares; host-only calls behave without a GPU."""
+import os
+import re
+import subprocess
+
+import pytest
+
+import token_indexed_sparse_staple_b200 as stp
+from token_indexed_sparse_staple_b200 import _lib
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+ROOT = os.path.dirname(HERE)
+
+
+def header_functions():
+    src = open(os.path.join(ROOT, "include", "staple.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(staple_[a-z_0-9]+)\s*\(", src)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from token_indexed_sparse_staple_b200 import build
+    build.build()
+    return _lib.load()
+
+
+def test_every_declared_function_is_exported(lib):
+    names = header_functions()
+    assert len(names) >= 18
+    out = subprocess.run(["nm", "-D", "--defined-only", _lib.LIB_PATH], capture_output=True,
+                         text=True, check=True).stdout
+    exported = set(re.findall(r"\bT (staple_\w+)", out))
+    missing = [n for n in names if n not in exported]
+    assert not missing, missing
+    for n in names:
+        assert hasattr(lib, n)
+
+
+def test_binding_covers_the_header():
+    assert sorted(_lib.SIGNATURES) == header_functions()
+    for n in header_functions():
+        assert callable(getattr(stp, n)), n
+
+
+def test_host_only_calls(lib):
+    assert stp.staple_abi_version() == 1
+    assert stp.staple_status_string(0) == "STAPLE_OK"
+    assert "EIDRANGE" in stp.staple_status_string(-2)
+    assert stp.staple_status_string(12345) == "STAPLE_UNKNOWN"
+    ws = stp.staple_workspace_bytes(16384, 2048, 8192)
+    assert ws % 256 == 0 and ws >= 256 * 2 * 8192 * 4
+    assert stp.staple_workspace_bytes(-1, 1, 1) == 0
+
+
+def test_no_device_is_reported_not_faked(lib):
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    with pytest.raises(stp.StapleError) as e:
+        stp.staple_context_create(0)
+    assert e.value.status == stp.STAPLE_ENODEV
+
+
+def test_null_arguments_are_rejected_before_any_launch(lib):
+    import ctypes as C
+    h = C.c_void_p()
+    assert lib.staple_context_create(0, None) == stp.STAPLE_EINVAL
+    assert lib.staple_table_register(None, None, 0, 1, 1, 1, 0, 1, C.byref(h)) == stp.STAPLE_EINVAL
+    assert lib.staple_ffn_fwd(None, 0, 1, 64, 64, None, None, None, None, None, None, None,
+                              None, None, None, 0, None) == stp.STAPLE_EINVAL
+    assert lib.staple_dedup(None, None, 0, 10, None, None, None, None, None, None) == stp.STAPLE_EINVAL

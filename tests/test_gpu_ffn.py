@@ -1,0 +1,154 @@
+"""GPU parity of the STAPLE FFN layer (forward and backward) against the
+oracle, at sizes the oracle finishes in seconds that span several tiles and
+ragged tails, plus the exact identities of the method (E = 0 is the dense
+FFN; gathered rows and direct table rows give the same result)."""
+import numpy as np
+import pytest
+
+import oracle
+import synthetic as syn
+from tests.helpers import TOL, assert_close
+from tests.layer_runner import run_layer
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def stp():
+    import token_indexed_sparse_staple_b200 as m
+    return m
+
+
+@pytest.fixture(scope="module")
+def ctx(stp):
+    c = stp.staple_context_create(0)
+    yield c
+    stp.staple_context_destroy(c)
+
+
+def oracle_layer(inp, training=True, zero_table=False):
+    x, wg, wu, wd = (inp.f64(k) for k in ("x", "w_gate", "w_up", "w_down"))
+    E = None if inp.table is None else inp.f64("table")
+    if zero_table and E is not None:
+        E = np.zeros_like(E)
+    fw = oracle.ffn_forward(x, inp.ids, wg, wu, wd, E)
+    if not training:
+        return fw
+    bw = oracle.ffn_backward(inp.f64("dy"), x, inp.ids, wg, wu, wd, fw)
+    return {**fw, **bw}
+
+
+def compare(got, ref, tol, keys):
+    for k in keys:
+        assert_close(got[k], ref[k], tol, k)
+
+
+FWD = ("z", "y")
+SAVED = ("g", "h")
+BWD = ("dg", "dh", "dE", "dx", "dW_gate", "dW_up", "dW_down")
+
+
+# ---------------------------------------------------------------- fp32 path
+
+@pytest.mark.parametrize("embed", ["table", "rows"])
+def test_tiny_f32_layer(stp, ctx, embed):
+    w = syn.WORKLOADS["tiny-f32"]
+    inp = syn.make_layer_inputs(w)
+    got = run_layer(stp, ctx, inp, w.D, w.F, w.V, embed=embed)
+    ref = oracle_layer(inp)
+    np.testing.assert_array_equal(got["unique"], ref["unique"])
+    compare(got, ref, TOL["f32"], FWD + SAVED + BWD)
+
+
+def test_tiny_f32_zero_table_is_dense(stp, ctx):
+    w = syn.WORKLOADS["tiny-f32"]
+    inp = syn.make_layer_inputs(w, zero_table=True)
+    got = run_layer(stp, ctx, inp, w.D, w.F, w.V, embed="table")
+    dense = run_layer(stp, ctx, inp, w.D, w.F, w.V, embed="none")
+    for k in FWD + SAVED + BWD:
+        np.testing.assert_array_equal(got[k] + 0.0, dense[k] + 0.0, err_msg=k)
+    compare(got, oracle_layer(inp), TOL["f32"], FWD + BWD)
+
+
+# ---------------------------------------------------------------- bf16 path
+
+SMALL = [
+    # (T, D, F, V): several M tiles with a ragged tail; F not a multiple of the
+    # 128-feature gate/up tile or the 256-wide tile; D below one tile
+    (300, 128, 320, 1000),
+    (129, 64, 64, 50),
+    (1, 64, 128, 10),
+    (640, 256, 512, 3000),
+]
+
+
+def _bf16_workload(T, D, F, V):
+    return syn.Workload("bf16-small", T=T, D=D, F=F, V=V, layers=1, dtype="bf16", w_std=0.05,
+                        e_std=0.05, x_std=1.0, dy_std=1.0, table="device", cache_frac=0.0,
+                        group=1, training=True)
+
+
+@pytest.mark.parametrize("T,D,F,V", SMALL)
+def test_bf16_layer_matches_oracle(stp, ctx, T, D, F, V):
+    w = _bf16_workload(T, D, F, V)
+    inp = syn.make_layer_inputs(w)
+    got = run_layer(stp, ctx, inp, D, F, V, embed="table")
+    ref = oracle_layer(inp)
+    np.testing.assert_array_equal(got["unique"], ref["unique"])
+    compare(got, ref, TOL["bf16"], FWD + SAVED + BWD)
+
+
+def test_bf16_zero_table_is_bitwise_dense(stp, ctx):
+    w = _bf16_workload(300, 128, 320, 1000)
+    inp = syn.make_layer_inputs(w, zero_table=True)
+    got = run_layer(stp, ctx, inp, w.D, w.F, w.V, embed="table")
+    dense = run_layer(stp, ctx, inp, w.D, w.F, w.V, embed="none")
+    for k in FWD + SAVED + BWD:
+        np.testing.assert_array_equal(got[k] + 0.0, dense[k] + 0.0, err_msg=k)
+
+
+def test_bf16_gathered_rows_equal_table_rows(stp, ctx):
+    w = _bf16_workload(640, 256, 512, 3000)
+    inp = syn.make_layer_inputs(w)
+    direct = run_layer(stp, ctx, inp, w.D, w.F, w.V, embed="table")
+    freq = syn.calibration_freq(w.V, n_tokens=1 << 18)
+    gathered = run_layer(stp, ctx, inp, w.D, w.F, w.V, embed="rows", rows_table=inp.table,
+                         cache_frac=0.05, freq=freq)
+    assert gathered["miss_count"] > 0
+    for k in FWD + SAVED + BWD:
+        np.testing.assert_array_equal(gathered[k], direct[k], err_msg=k)
+
+
+def test_bf16_frozen_up_projection(stp, ctx):
+    w = _bf16_workload(300, 128, 320, 1000)
+    inp = syn.make_layer_inputs(w)
+    got = run_layer(stp, ctx, inp, w.D, w.F, w.V, embed="table", freeze_up=True)
+    ref = oracle_layer(inp)
+    compare(got, ref, TOL["bf16"], ("dW_gate", "dW_down", "dE", "dx"))
+    assert np.all(got["dW_up"] == 7.0)   # untouched
+
+
+def test_bf16_deterministic(stp, ctx):
+    w = _bf16_workload(640, 256, 512, 3000)
+    inp = syn.make_layer_inputs(w)
+    a = run_layer(stp, ctx, inp, w.D, w.F, w.V, embed="table")
+    b = run_layer(stp, ctx, inp, w.D, w.F, w.V, embed="table")
+    for k in FWD + SAVED + BWD:
+        np.testing.assert_array_equal(a[k], b[k], err_msg=k)
+
+
+def test_bf16_out_of_range_id_reported(stp, ctx):
+    w = _bf16_workload(129, 64, 64, 50)
+    inp = syn.make_layer_inputs(w)
+    inp.ids[5] = 50
+    with pytest.raises(AssertionError, match="EIDRANGE"):
+        run_layer(stp, ctx, inp, w.D, w.F, w.V, embed="table", training=False)
+
+
+def test_bf16_rejects_unsupported_shapes(stp, ctx):
+    import torch
+    t = torch.zeros(4096, dtype=torch.bfloat16, device="cuda")
+    e = stp.make_embed(stp.STAPLE_EMBED_NONE)
+    with pytest.raises(stp.StapleError) as ex:
+        stp.staple_ffn_fwd(ctx, stp.STAPLE_BF16, 4, 96, 64, t, e, t, t, t, t, t)
+    assert ex.value.status == stp.STAPLE_EINVAL

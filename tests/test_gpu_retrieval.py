@@ -1,0 +1,162 @@
+"""GPU parity of the retrieval path (dedup, cache build, probe, hit and miss
+gathers) against the oracle: bit-exact for every index and every row byte."""
+import numpy as np
+import pytest
+
+import oracle
+import synthetic as syn
+from tests.helpers import bits, dev, empty, read_device
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def stp():
+    import token_indexed_sparse_staple_b200 as m
+    return m
+
+
+@pytest.fixture(scope="module")
+def ctx(stp):
+    c = stp.staple_context_create(0)
+    yield c
+    stp.staple_context_destroy(c)
+
+
+def run_dedup(stp, ctx, ids, V):
+    import torch
+    T = len(ids)
+    d_ids = torch.from_numpy(np.asarray(ids, dtype=np.int32)).cuda()
+    out = {k: empty(max(T, 1), "i32") for k in ("unique", "inverse", "sorted_pos")}
+    seg = empty(T + 1, "i32")
+    U = empty(1, "i32")
+    stp.staple_dedup(ctx, d_ids, T, V, out["unique"], out["inverse"], seg, out["sorted_pos"], U)
+    assert stp.staple_get_error(ctx) == 0
+    u = int(U.item())
+    return (out["unique"].cpu().numpy()[:u], out["inverse"].cpu().numpy()[:T],
+            seg.cpu().numpy()[:u + 1], out["sorted_pos"].cpu().numpy()[:T])
+
+
+CASES = {
+    "empty": ([], 10),
+    "one": ([7], 10),
+    "all_equal": ([3] * 1000, 10),
+    "all_distinct": (list(range(999, -1, -1)), 1000),
+    "edges": ([0, 99999, 0, 99999, 5], 100000),
+    "V_is_1": ([0, 0, 0], 1),
+}
+
+
+@pytest.mark.parametrize("name", list(CASES))
+def test_dedup_edge_cases(stp, ctx, name):
+    ids, V = CASES[name]
+    got = run_dedup(stp, ctx, ids, V)
+    ref = oracle.dedup(np.array(ids, dtype=np.int32))
+    for g, r, what in zip(got, ref, ("unique", "inverse", "seg_off", "sorted_pos")):
+        np.testing.assert_array_equal(g, r, err_msg=what)
+
+
+@pytest.mark.parametrize("T,V", [(64, 100352), (256, 1000), (1025, 100352), (4097, 50000),
+                                 (16384, 100352), (32768, 100352), (16384, 1 << 20)])
+def test_dedup_zipf(stp, ctx, T, V):
+    ids = syn.zipf_ids(T, V, 1.1, seed=T + V)
+    got = run_dedup(stp, ctx, ids, V)
+    ref = oracle.dedup(ids)
+    for g, r, what in zip(got, ref, ("unique", "inverse", "seg_off", "sorted_pos")):
+        np.testing.assert_array_equal(g, r, err_msg=what)
+
+
+def test_dedup_reports_out_of_range_ids(stp, ctx):
+    import torch
+    ids = torch.tensor([1, 2, 10, 3], dtype=torch.int32, device="cuda")
+    bufs = [empty(4, "i32") for _ in range(3)]
+    seg, U = empty(5, "i32"), empty(1, "i32")
+    stp.staple_dedup(ctx, ids, 4, 10, bufs[0], bufs[1], seg, bufs[2], U)
+    assert stp.staple_get_error(ctx) == stp.STAPLE_EIDRANGE
+    assert stp.staple_get_error(ctx) == 0   # reading clears the word
+
+
+def _table(w, layer=0, groups=1):
+    """[V][groups*F] bf16 table (groups stacked layers, token-major)."""
+    parts = [syn.bf16_normal((w.V, w.F), w.e_std, syn.SEED_E + layer + g)[0] for g in range(groups)]
+    return np.ascontiguousarray(np.stack(parts, axis=1).reshape(w.V, groups * w.F))
+
+
+@pytest.mark.parametrize("where", ["device", "host"])
+@pytest.mark.parametrize("frac", [0.0, 0.05, 1.0])
+@pytest.mark.parametrize("groups", [1, 4])
+def test_cache_and_gather(stp, ctx, where, frac, groups):
+    import torch
+    w = syn.Workload("small", T=3000, D=64, F=128, V=5000, layers=groups, dtype="bf16",
+                     w_std=0.02, e_std=0.01, x_std=1.0, dy_std=1.0, table=where, cache_frac=frac,
+                     group=groups, training=False)
+    E = _table(w, groups=groups)
+    if where == "device":
+        t_store = dev(E, "bf16")
+        flags = stp.STAPLE_TABLE_DEVICE
+    else:
+        t_store = torch.from_numpy(E.view(np.int16)).pin_memory()
+        flags = stp.STAPLE_TABLE_HOST_PINNED
+    table = stp.staple_table_register(ctx, t_store, E.nbytes, w.V, w.F, groups, stp.STAPLE_BF16, flags)
+    freq = syn.calibration_freq(w.V, n_tokens=1 << 18)
+    cache = stp.staple_cache_build(ctx, table, freq, frac)
+    try:
+        hot_ref, slot_of = oracle.hot_set(freq, frac)
+        np.testing.assert_array_equal(stp.staple_cache_hot_ids(cache), hot_ref)
+        K, cap = stp.staple_cache_info(cache)
+        assert K == hot_ref.size and cap >= 2 * K and cap & (cap - 1) == 0
+        if K:
+            raw = read_device(stp.staple_cache_rows(cache), K * groups * w.F * 2)
+            np.testing.assert_array_equal(raw.view(np.uint16).reshape(K, groups * w.F),
+                                          oracle.cache_rows_for(E, hot_ref))
+
+        ids = syn.zipf_ids(w.T, w.V, 1.1, seed=5)
+        T = w.T
+        d_ids = torch.from_numpy(ids).cuda()
+        unique, inverse, sorted_pos, slot, miss = (empty(T, "i32") for _ in range(5))
+        seg, U, mc = empty(T + 1, "i32"), empty(1, "i32"), empty(1, "i32")
+        rows = torch.zeros((T, groups * w.F), dtype=torch.bfloat16, device="cuda")
+        side = torch.cuda.Stream()
+        stp.staple_gather_rows(ctx, cache, table, d_ids, T, unique, inverse, seg, sorted_pos, U,
+                               slot, miss, mc, rows, side=side)
+        assert stp.staple_get_error(ctx) == 0
+        u_ref, inv_ref, _, _ = oracle.dedup(ids)
+        slot_ref, miss_ref = oracle.probe(u_ref, slot_of)
+        Ug = int(U.item())
+        assert Ug == u_ref.size
+        np.testing.assert_array_equal(slot.cpu().numpy()[:Ug], slot_ref)
+        assert int(mc.item()) == miss_ref.size
+        np.testing.assert_array_equal(miss.cpu().numpy()[:miss_ref.size], miss_ref)
+        np.testing.assert_array_equal(bits(rows)[:Ug], oracle.gather_rows(E, u_ref))
+        if frac == 0.05:
+            # Zipf stream: most tokens hit a 5% cache
+            hit_tokens = np.mean(slot_ref[inv_ref] >= 0)
+            assert hit_tokens > 0.6
+    finally:
+        stp.staple_cache_free(cache)
+        stp.staple_table_unregister(table)
+
+
+def test_register_pageable_host_table(stp, ctx):
+    import torch
+    import mmap
+    E = syn.bf16_normal((300, 64), 0.01, 3)[0]
+    mm = mmap.mmap(-1, E.nbytes)   # page-aligned pageable memory
+    host = np.frombuffer(mm, dtype=np.uint16).reshape(E.shape)
+    host[:] = E
+    table = stp.staple_table_register(ctx, host, host.nbytes, 300, 64, 1, stp.STAPLE_BF16,
+                                      stp.STAPLE_TABLE_HOST_REGISTER)
+    try:
+        ids = np.array([5, 299, 5, 0], dtype=np.int32)
+        T = 4
+        d_ids = torch.from_numpy(ids).cuda()
+        bufs = [empty(T, "i32") for _ in range(5)]
+        seg, U, mc = empty(T + 1, "i32"), empty(1, "i32"), empty(1, "i32")
+        rows = torch.zeros((T, 64), dtype=torch.bfloat16, device="cuda")
+        stp.staple_gather_rows(ctx, None, table, d_ids, T, bufs[0], bufs[1], seg, bufs[2], U,
+                               bufs[3], bufs[4], mc, rows)
+        assert stp.staple_get_error(ctx) == 0
+        np.testing.assert_array_equal(bits(rows)[:3], E[[0, 5, 299]])
+        assert int(mc.item()) == 3
+    finally:
+        stp.staple_table_unregister(table)

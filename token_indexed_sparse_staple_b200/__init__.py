@@ -1,0 +1,196 @@
+"""Python binding of libstaple (include/staple.h): the STAPLE embedding-
+augmented SwiGLU FFN layer on B200 (sm_100a).
+
+Each function has the name of the C entry point it calls and only marshals
+arguments: tensors become device (or host) addresses, streams become
+cudaStream_t handles (default: torch's current stream), and a non-zero status
+raises StapleError.  There is no fallback: the library must be built
+(`python -m token_indexed_sparse_staple_b200.build`) and a B200 must be present
+for any compute call.
+"""
+from __future__ import annotations
+
+import ctypes as C
+
+import numpy as np
+
+from . import _lib
+from ._lib import staple_embed
+
+STAPLE_OK = 0
+STAPLE_EINVAL, STAPLE_EIDRANGE, STAPLE_ECUDA, STAPLE_ENOMEM = -1, -2, -3, -4
+STAPLE_ETIMEOUT, STAPLE_EUNSUPPORTED, STAPLE_ENODEV = -5, -6, -7
+STAPLE_BF16, STAPLE_F32 = 0, 1
+STAPLE_EMBED_NONE, STAPLE_EMBED_TABLE, STAPLE_EMBED_ROWS = 0, 1, 2
+STAPLE_TABLE_DEVICE, STAPLE_TABLE_HOST_PINNED, STAPLE_TABLE_HOST_REGISTER = 1, 2, 4
+
+__all__ = [n for n in _lib.SIGNATURES] + [
+    "StapleError", "staple_embed", "make_embed", "lib",
+]
+
+
+class StapleError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        msg = lib().staple_status_string(status).decode()
+        super().__init__(f"{where}: {msg} ({status})")
+
+
+def lib():
+    return _lib.load()
+
+
+def _p(x) -> int | None:
+    """Address of a tensor / array / raw int (None -> NULL)."""
+    if x is None:
+        return None
+    if isinstance(x, int):
+        return x
+    if isinstance(x, np.ndarray):
+        return x.ctypes.data
+    return x.data_ptr()
+
+
+def _stream(s) -> int | None:
+    if s is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(s, int):
+        return s
+    return s.cuda_stream
+
+
+def _ok(status: int, where: str) -> None:
+    if status != STAPLE_OK:
+        raise StapleError(status, where)
+
+
+def make_embed(mode: int, base=None, row_pitch: int = 0, index=None, n_rows: int = 0) -> staple_embed:
+    return staple_embed(mode, 0, _p(base), row_pitch, _p(index), n_rows)
+
+
+# ------------------------------------------------------------------ context
+
+def staple_abi_version() -> int:
+    return lib().staple_abi_version()
+
+
+def staple_status_string(s: int) -> str:
+    return lib().staple_status_string(s).decode()
+
+
+def staple_context_create(device: int = 0) -> int:
+    h = C.c_void_p()
+    _ok(lib().staple_context_create(device, C.byref(h)), "staple_context_create")
+    return h.value
+
+
+def staple_context_destroy(ctx: int) -> None:
+    _ok(lib().staple_context_destroy(ctx), "staple_context_destroy")
+
+
+def staple_get_error(ctx: int, stream=None) -> int:
+    e = C.c_int32()
+    _ok(lib().staple_get_error(ctx, _stream(stream), C.byref(e)), "staple_get_error")
+    return e.value
+
+
+# ------------------------------------------------------------------- tables
+
+def staple_table_register(ctx: int, base, nbytes: int, V: int, F: int, groups: int, dtype: int,
+                          flags: int) -> int:
+    h = C.c_void_p()
+    _ok(lib().staple_table_register(ctx, _p(base), nbytes, V, F, groups, dtype, flags,
+                                    C.byref(h)), "staple_table_register")
+    return h.value
+
+
+def staple_table_unregister(table: int) -> None:
+    _ok(lib().staple_table_unregister(table), "staple_table_unregister")
+
+
+# -------------------------------------------------------------------- cache
+
+def staple_cache_build(ctx: int, table: int, freq: np.ndarray, frac: float, stream=None) -> int:
+    freq = np.ascontiguousarray(freq, dtype=np.int64)
+    h = C.c_void_p()
+    _ok(lib().staple_cache_build(ctx, table, freq.ctypes.data, float(frac), _stream(stream),
+                                 C.byref(h)), "staple_cache_build")
+    return h.value
+
+
+def staple_cache_info(cache: int) -> tuple[int, int]:
+    k, cap = C.c_int32(), C.c_int32()
+    _ok(lib().staple_cache_info(cache, C.byref(k), C.byref(cap)), "staple_cache_info")
+    return k.value, cap.value
+
+
+def staple_cache_hot_ids(cache: int) -> np.ndarray:
+    K, _ = staple_cache_info(cache)
+    out = np.zeros(K, dtype=np.int32)
+    _ok(lib().staple_cache_hot_ids(cache, out.ctypes.data if K else None), "staple_cache_hot_ids")
+    return out
+
+
+def staple_cache_rows(cache: int) -> int:
+    p = C.c_void_p()
+    _ok(lib().staple_cache_rows(cache, C.byref(p)), "staple_cache_rows")
+    return p.value
+
+
+def staple_cache_free(cache: int) -> None:
+    _ok(lib().staple_cache_free(cache), "staple_cache_free")
+
+
+def staple_workspace_bytes(T: int, D: int, F: int, flags: int = 0) -> int:
+    return int(lib().staple_workspace_bytes(T, D, F, flags))
+
+
+# ---------------------------------------------------------------- retrieval
+
+def staple_dedup(ctx, ids, T, V, unique, inverse, seg_off, sorted_pos, U_dev, stream=None):
+    _ok(lib().staple_dedup(ctx, _p(ids), T, V, _p(unique), _p(inverse), _p(seg_off),
+                           _p(sorted_pos), _p(U_dev), _stream(stream)), "staple_dedup")
+
+
+def staple_gather_unique_rows(ctx, cache, table, unique, U_dev, T, slot, miss_list, miss_count,
+                              rows, stream=None, side=None):
+    st = _stream(stream)
+    _ok(lib().staple_gather_unique_rows(ctx, cache, table, _p(unique), _p(U_dev), T, _p(slot),
+                                        _p(miss_list), _p(miss_count), _p(rows), st,
+                                        st if side is None else _stream(side)),
+        "staple_gather_unique_rows")
+
+
+def staple_gather_rows(ctx, cache, table, ids, T, unique, inverse, seg_off, sorted_pos, U_dev,
+                       slot, miss_list, miss_count, rows, stream=None, side=None):
+    st = _stream(stream)
+    _ok(lib().staple_gather_rows(ctx, cache, table, _p(ids), T, _p(unique), _p(inverse),
+                                 _p(seg_off), _p(sorted_pos), _p(U_dev), _p(slot), _p(miss_list),
+                                 _p(miss_count), _p(rows), st,
+                                 st if side is None else _stream(side)), "staple_gather_rows")
+
+
+# ---------------------------------------------------------------------- FFN
+
+def staple_ffn_fwd(ctx, dtype, T, D, F, x, embed, w_gate, w_up, w_down, z, y, g_save=None,
+                   h_save=None, workspace=None, workspace_bytes=0, stream=None):
+    e = C.byref(embed) if embed is not None else None
+    _ok(lib().staple_ffn_fwd(ctx, dtype, T, D, F, _p(x), e, _p(w_gate), _p(w_up), _p(w_down),
+                             _p(z), _p(y), _p(g_save), _p(h_save), _p(workspace),
+                             workspace_bytes, _stream(stream)), "staple_ffn_fwd")
+
+
+def staple_embed_bwd(ctx, dtype, T, D, F, dy, g_save, h_save, w_down, sorted_pos, inverse,
+                     seg_off, U_dev, dgh, dE, workspace=None, workspace_bytes=0, stream=None):
+    _ok(lib().staple_embed_bwd(ctx, dtype, T, D, F, _p(dy), _p(g_save), _p(h_save), _p(w_down),
+                               _p(sorted_pos), _p(inverse), _p(seg_off), _p(U_dev), _p(dgh),
+                               _p(dE), _p(workspace), workspace_bytes, _stream(stream)),
+        "staple_embed_bwd")
+
+
+def staple_ffn_bwd(ctx, dtype, T, D, F, dy, x, z, dgh, w_gate, w_up, dx, dw_gate, dw_up, dw_down,
+                   workspace=None, workspace_bytes=0, stream=None):
+    _ok(lib().staple_ffn_bwd(ctx, dtype, T, D, F, _p(dy), _p(x), _p(z), _p(dgh), _p(w_gate),
+                             _p(w_up), _p(dx), _p(dw_gate), _p(dw_up), _p(dw_down),
+                             _p(workspace), workspace_bytes, _stream(stream)), "staple_ffn_bwd")

@@ -1,0 +1,152 @@
+// K8: the table gradient of the U distinct rows of a batch.
+//
+//   dE[j][f] = sum of dh[i][f] over the tokens i whose id is unique[j]
+//
+// (AI Radio episode, paper summary: during training only the U x d_ff active
+// rows exist on the GPU, as an autograd leaf, so the gradient is one row per
+// distinct id.)  The dedup's sorted_pos lists each segment's tokens in
+// ascending position.  The sorted order is cut into chunks of kSegChunk
+// positions; one block per (chunk, 2048-feature slice) sums each segment
+// piece in order with fp32 accumulators.  A segment that lies inside one
+// chunk is written to dE directly; a piece of a segment that crosses a chunk
+// boundary goes to a partial buffer (at most two pieces per chunk), and a
+// second kernel adds the pieces of each crossing segment in chunk order.  No
+// float atomics: the result is deterministic.
+#include "common.cuh"
+#include "internal.h"
+
+namespace stp {
+
+constexpr int kSegThreads = 256;
+constexpr int kSegVec = 8;                           // features per thread
+constexpr int kSegSlice = kSegThreads * kSegVec;     // features per block
+
+template <bool BF16>
+__device__ __forceinline__ void load8(const void* base, int64_t off, float* v) {
+  if constexpr (BF16) {
+    const uint4 w = __ldg(reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(base) + off));
+    v[0] = bf_lo(w.x); v[1] = bf_hi(w.x); v[2] = bf_lo(w.y); v[3] = bf_hi(w.y);
+    v[4] = bf_lo(w.z); v[5] = bf_hi(w.z); v[6] = bf_lo(w.w); v[7] = bf_hi(w.w);
+  } else {
+    const float4* p = reinterpret_cast<const float4*>(static_cast<const float*>(base) + off);
+    const float4 a = __ldg(p), b = __ldg(p + 1);
+    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+    v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+  }
+}
+
+__device__ __forceinline__ void store8(float* dst, const float* v) {
+  float4* d = reinterpret_cast<float4*>(dst);
+  d[0] = make_float4(v[0], v[1], v[2], v[3]);
+  d[1] = make_float4(v[4], v[5], v[6], v[7]);
+}
+
+// Pieces of chunk c: part[(2c + side) * F + f]; side 0 = the chunk's first
+// segment (it started before the chunk), side 1 = its last segment (it
+// continues after the chunk).
+template <bool BF16>
+__global__ void __launch_bounds__(kSegThreads)
+    seg_reduce_kernel(const void* __restrict__ dh, int64_t ld, const int32_t* __restrict__ sorted_pos,
+                      const int32_t* __restrict__ inverse, const int32_t* __restrict__ seg_off,
+                      int T, int F, float* __restrict__ dE, float* __restrict__ part) {
+  __shared__ int32_t s_pos[kSegChunk];
+  __shared__ int32_t s_seg[kSegChunk];
+  const int c = blockIdx.x;
+  const int p0 = c * kSegChunk;
+  const int p1 = min(T, p0 + kSegChunk);
+  const int n = p1 - p0;
+  if (threadIdx.x < n) {
+    const int pos = sorted_pos[p0 + threadIdx.x];
+    s_pos[threadIdx.x] = pos;
+    s_seg[threadIdx.x] = inverse[pos];
+  }
+  __syncthreads();
+  const int f = (blockIdx.y * kSegThreads + threadIdx.x) * kSegVec;
+  if (f >= F) return;
+  const int first_seg = s_seg[0];
+  float acc[kSegVec];
+#pragma unroll
+  for (int i = 0; i < kSegVec; ++i) acc[i] = 0.0f;
+  int cur = first_seg;
+  auto flush = [&](int j) {
+    const int s0 = seg_off[j], s1 = seg_off[j + 1];
+    if (s0 >= p0 && s1 <= p1) {
+      store8(dE + int64_t(j) * F + f, acc);
+    } else {
+      const int side = (j == first_seg) ? 0 : 1;
+      store8(part + (int64_t(2 * c + side)) * F + f, acc);
+    }
+  };
+  for (int q = 0; q < n; ++q) {
+    const int j = s_seg[q];
+    if (j != cur) {
+      flush(cur);
+      cur = j;
+#pragma unroll
+      for (int i = 0; i < kSegVec; ++i) acc[i] = 0.0f;
+    }
+    float v[kSegVec];
+    load8<BF16>(dh, int64_t(s_pos[q]) * ld + f, v);
+#pragma unroll
+    for (int i = 0; i < kSegVec; ++i) acc[i] += v[i];
+  }
+  if (n > 0) flush(cur);
+}
+
+// One block per (chunk, slice): the segment that starts in chunk c (the last
+// segment of c) and ends after it is completed here from its pieces.
+__global__ void __launch_bounds__(kSegThreads)
+    seg_fixup_kernel(const int32_t* __restrict__ sorted_pos, const int32_t* __restrict__ inverse,
+                     const int32_t* __restrict__ seg_off, int T, int F, float* __restrict__ dE,
+                     const float* __restrict__ part) {
+  const int c = blockIdx.x;
+  const int p0 = c * kSegChunk;
+  const int plast = min(T, p0 + kSegChunk) - 1;
+  const int j = inverse[sorted_pos[plast]];
+  const int s0 = seg_off[j], s1 = seg_off[j + 1];
+  if (!(s0 >= p0 && s1 > p0 + kSegChunk)) return;
+  const int f = (blockIdx.y * kSegThreads + threadIdx.x) * kSegVec;
+  if (f >= F) return;
+  float acc[kSegVec];
+  {
+    const int side = (s0 == p0) ? 0 : 1;
+    const float4* a = reinterpret_cast<const float4*>(part + int64_t(2 * c + side) * F + f);
+    const float4 x = a[0], y = a[1];
+    acc[0] = x.x; acc[1] = x.y; acc[2] = x.z; acc[3] = x.w;
+    acc[4] = y.x; acc[5] = y.y; acc[6] = y.z; acc[7] = y.w;
+  }
+  const int ce = (s1 - 1) / kSegChunk;
+  for (int cc = c + 1; cc <= ce; ++cc) {
+    const float4* a = reinterpret_cast<const float4*>(part + int64_t(2 * cc) * F + f);
+    const float4 x = a[0], y = a[1];
+    acc[0] += x.x; acc[1] += x.y; acc[2] += x.z; acc[3] += x.w;
+    acc[4] += y.x; acc[5] += y.y; acc[6] += y.z; acc[7] += y.w;
+  }
+  store8(dE + int64_t(j) * F + f, acc);
+}
+
+size_t seg_reduce_workspace(int T, int F) {
+  const int64_t chunks = (int64_t(T) + kSegChunk - 1) / kSegChunk;
+  return size_t(chunks) * 2 * size_t(F) * sizeof(float);
+}
+
+staple_status launch_seg_reduce(bool bf16, const void* dh, int64_t ld, const int32_t* sorted_pos,
+                                const int32_t* inverse, const int32_t* seg_off,
+                                const int32_t* U_dev, int T, int F, float* dE, float* part,
+                                cudaStream_t st) {
+  (void)U_dev;
+  if (T == 0) return STAPLE_OK;
+  const int chunks = (T + kSegChunk - 1) / kSegChunk;
+  const dim3 grid(chunks, (F + kSegSlice - 1) / kSegSlice);
+  if (bf16)
+    seg_reduce_kernel<true><<<grid, kSegThreads, 0, st>>>(dh, ld, sorted_pos, inverse, seg_off, T,
+                                                          F, dE, part);
+  else
+    seg_reduce_kernel<false><<<grid, kSegThreads, 0, st>>>(dh, ld, sorted_pos, inverse, seg_off,
+                                                           T, F, dE, part);
+  if (chunks > 1)
+    seg_fixup_kernel<<<grid, kSegThreads, 0, st>>>(sorted_pos, inverse, seg_off, T, F, dE, part);
+  return cudaGetLastError() == cudaSuccess ? STAPLE_OK : STAPLE_ECUDA;
+}
+
+}  // namespace stp

@@ -1,0 +1,223 @@
+// Host side of the bf16 tcgen05 path: TMA tensor maps and the launches of
+// the six contractions of the layer (K5, K6, K7, K9, K10), each with its
+// epilogue fused into the GEMM kernel of gemm_tc.cuh.
+//
+//   K5  [g | u] = x W_gate^T | x W_up^T, epilogue h = u + E[row], z = SiLU(g) h
+//   K6  y       = z W_down^T
+//   K7  dz      = dY W_down,  epilogue dh = dz SiLU(g), dg = dz h SiLU'(g)
+//   K9  dx      = dg W_gate + dh W_up                  (K concatenated)
+//   K10 dW_gate | dW_up = [dg | dh]^T x,  dW_down = dY^T z
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <mutex>
+
+#include "gemm_tc.cuh"
+#include "internal.h"
+
+namespace stp {
+
+namespace {
+
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+std::once_flag g_encode_once;
+
+PFN_cuTensorMapEncodeTiled_v12000 encoder() {
+  std::call_once(g_encode_once, [] {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  });
+  return g_encode;
+}
+
+// 2-D bf16 tensor map over a row-major matrix with `rows` rows of `cols`
+// elements (leading dimension ld), box = box_cols x box_rows, 128-byte swizzle.
+bool make_map(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows, uint64_t ld,
+              uint32_t box_cols, uint32_t box_rows) {
+  auto enc = encoder();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {ld * 2};
+  cuuint32_t box[2] = {box_cols, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// K-major operand [rows][k]: box 64 (k) x 128 (rows).
+bool kmajor(CUtensorMap* m, const void* base, int rows, int k, int64_t ld) {
+  return make_map(m, base, uint64_t(k), uint64_t(rows), uint64_t(ld), tc::BK, 128);
+}
+// MN-major operand stored [k][mn]: box 64 (mn) x 64 (k).
+bool mnmajor(CUtensorMap* m, const void* base, int k, int mn, int64_t ld) {
+  return make_map(m, base, uint64_t(mn), uint64_t(k), uint64_t(ld), 64, tc::BK);
+}
+
+template <bool A_MN, bool B_MN, int BSRC, int EPI>
+staple_status launch(const DeviceInfo& di, const CUtensorMap& a, const CUtensorMap& b0,
+                     const CUtensorMap& b1, tc::Params p, cudaStream_t st) {
+  p.k_blocks = (p.K + tc::BK - 1) / tc::BK;
+  const int ntiles = p.tiles_m * p.tiles_n;
+  if (ntiles == 0) return STAPLE_OK;
+  if (p.group_m <= 0) p.group_m = 16;
+  auto kern = tc::gemm_kernel<A_MN, B_MN, BSRC, EPI>;
+  static bool attr_set = false;  // per instantiation
+  if (!attr_set) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             tc::kSmemBytes) != cudaSuccess)
+      return STAPLE_ECUDA;
+    attr_set = true;
+  }
+  const int grid = std::min(ntiles, di.num_sms);
+  kern<<<grid, tc::kThreads, tc::kSmemBytes, st>>>(a, b0, b1, p);
+  return cudaGetLastError() == cudaSuccess ? STAPLE_OK : STAPLE_ECUDA;
+}
+
+inline int cdiv(int a, int b) { return (a + b - 1) / b; }
+
+}  // namespace
+
+staple_status tc_ffn_fwd(const DeviceInfo& di, int T, int D, int F, const void* x,
+                         const staple_embed* e, const void* wg, const void* wu, const void* wd,
+                         void* z, void* y, void* g_save, void* h_save, int32_t* err,
+                         cudaStream_t st) {
+  if (T == 0) return STAPLE_OK;
+  CUtensorMap mx, mg, mu, mz, md;
+  if (!kmajor(&mx, x, T, D, D) || !kmajor(&mg, wg, F, D, D) || !kmajor(&mu, wu, F, D, D) ||
+      !kmajor(&mz, z, T, F, F) || !kmajor(&md, wd, D, F, F))
+    return STAPLE_ECUDA;
+  {
+    tc::Params p{};
+    p.M = T;
+    p.N = F;
+    p.K = D;
+    p.tiles_m = cdiv(T, tc::BM);
+    p.tiles_n = cdiv(F, tc::BN / 2);
+    p.z = static_cast<uint16_t*>(z);
+    p.g_save = static_cast<uint16_t*>(g_save);
+    p.h_save = static_cast<uint16_t*>(h_save);
+    p.ldf = F;
+    p.e_mode = e ? e->mode : STAPLE_EMBED_NONE;
+    if (e && e->mode != STAPLE_EMBED_NONE) {
+      p.e_base = static_cast<const uint16_t*>(e->base);
+      p.e_pitch = e->row_pitch;
+      p.e_index = e->index;
+      p.e_rows = e->n_rows;
+    }
+    p.err = err;
+    staple_status s = launch<false, false, tc::B_NHALF, tc::EPI_GATEUP>(di, mx, mg, mu, p, st);
+    if (s != STAPLE_OK) return s;
+  }
+  tc::Params q{};
+  q.M = T;
+  q.N = D;
+  q.K = F;
+  q.tiles_m = cdiv(T, tc::BM);
+  q.tiles_n = cdiv(D, tc::BN);
+  q.out = y;
+  q.ldo = D;
+  q.m_split = T;
+  q.err = err;
+  return launch<false, false, tc::B_ONE, tc::EPI_BF16>(di, mz, md, md, q, st);
+}
+
+staple_status tc_dz(const DeviceInfo& di, int T, int D, int F, const void* dy, const void* g_save,
+                    const void* h_save, const void* wd, void* dgh, int32_t* err, cudaStream_t st) {
+  if (T == 0) return STAPLE_OK;
+  CUtensorMap mdy, mwd;
+  // A = dY [T][D] (K-major over d); B(n = f, k = d) = W_down[d][f]: MN-major
+  if (!kmajor(&mdy, dy, T, D, D) || !mnmajor(&mwd, wd, D, F, F)) return STAPLE_ECUDA;
+  tc::Params p{};
+  p.M = T;
+  p.N = F;
+  p.K = D;
+  p.tiles_m = cdiv(T, tc::BM);
+  p.tiles_n = cdiv(F, tc::BN);
+  p.ldf = F;
+  p.g_in = static_cast<const uint16_t*>(g_save);
+  p.h_in = static_cast<const uint16_t*>(h_save);
+  p.dgh = static_cast<uint16_t*>(dgh);
+  p.err = err;
+  return launch<false, true, tc::B_ONE, tc::EPI_DZ>(di, mdy, mwd, mwd, p, st);
+}
+
+staple_status tc_ffn_bwd(const DeviceInfo& di, int T, int D, int F, const void* dy,
+                         const void* x, const void* z, const void* dgh, const void* wg,
+                         const void* wu, void* dx, float* dwg, float* dwu, float* dwd,
+                         int32_t* err, cudaStream_t st) {
+  staple_status s;
+  const uint16_t* dgh16 = static_cast<const uint16_t*>(dgh);
+  if (T == 0) {
+    if (dwg && cudaMemsetAsync(dwg, 0, size_t(F) * D * 4, st) != cudaSuccess) return STAPLE_ECUDA;
+    if (dwu && cudaMemsetAsync(dwu, 0, size_t(F) * D * 4, st) != cudaSuccess) return STAPLE_ECUDA;
+    if (dwd && cudaMemsetAsync(dwd, 0, size_t(F) * D * 4, st) != cudaSuccess) return STAPLE_ECUDA;
+    return STAPLE_OK;
+  }
+  if (dx) {
+    // K9: A = dgh [T][2F] K-major; B(n = d, k = f') = W_gate[f'][d] | W_up[f' - F][d]: MN-major
+    CUtensorMap ma, mb0, mb1;
+    if (!kmajor(&ma, dgh, T, 2 * F, 2 * F) || !mnmajor(&mb0, wg, F, D, D) ||
+        !mnmajor(&mb1, wu, F, D, D))
+      return STAPLE_ECUDA;
+    tc::Params p{};
+    p.M = T;
+    p.N = D;
+    p.K = 2 * F;
+    p.ksplit = F;
+    p.tiles_m = cdiv(T, tc::BM);
+    p.tiles_n = cdiv(D, tc::BN);
+    p.out = dx;
+    p.ldo = D;
+    p.m_split = T;
+    p.err = err;
+    if ((s = launch<false, true, tc::B_KSPLIT, tc::EPI_BF16>(di, ma, mb0, mb1, p, st)) !=
+        STAPLE_OK)
+      return s;
+  }
+  if (dwg || dwu) {
+    // K10a: C[m = f'][n = d] = sum_t dgh[t][f'] x[t][d]; A and B MN-major
+    const bool both = dwg && dwu;
+    const int M = both ? 2 * F : F;
+    CUtensorMap ma, mb;
+    if (!mnmajor(&ma, dwg ? dgh16 : dgh16 + F, T, M, 2 * F) || !mnmajor(&mb, x, T, D, D))
+      return STAPLE_ECUDA;
+    tc::Params p{};
+    p.M = M;
+    p.N = D;
+    p.K = T;
+    p.tiles_m = cdiv(M, tc::BM);
+    p.tiles_n = cdiv(D, tc::BN);
+    p.out = dwg ? dwg : dwu;
+    p.out2 = dwu;
+    p.ldo = D;
+    p.m_split = both ? F : M;
+    p.err = err;
+    if ((s = launch<true, true, tc::B_ONE, tc::EPI_F32>(di, ma, mb, mb, p, st)) != STAPLE_OK)
+      return s;
+  }
+  if (dwd) {
+    // K10b: C[m = d][n = f] = sum_t dY[t][d] z[t][f]; A and B MN-major
+    CUtensorMap ma, mb;
+    if (!mnmajor(&ma, dy, T, D, D) || !mnmajor(&mb, z, T, F, F)) return STAPLE_ECUDA;
+    tc::Params p{};
+    p.M = D;
+    p.N = F;
+    p.K = T;
+    p.tiles_m = cdiv(D, tc::BM);
+    p.tiles_n = cdiv(F, tc::BN);
+    p.out = dwd;
+    p.ldo = F;
+    p.m_split = D;
+    p.err = err;
+    if ((s = launch<true, true, tc::B_ONE, tc::EPI_F32>(di, ma, mb, mb, p, st)) != STAPLE_OK)
+      return s;
+  }
+  return STAPLE_OK;
+}
+
+}  // namespace stp

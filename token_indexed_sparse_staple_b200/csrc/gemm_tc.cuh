@@ -1,0 +1,391 @@
+// Persistent, warp-specialised tcgen05 GEMM for sm_100a with the STAPLE
+// epilogues fused in.
+//
+//   C[M][N] = sum_k A(m, k) * B(n, k)        bf16 operands, fp32 accumulators
+//
+// A and B are read by TMA into 128-byte-swizzled shared-memory stages.  Each
+// operand may be K-major (k contiguous in global memory) or MN-major (m or n
+// contiguous), which covers every contraction of the layer's forward and
+// backward pass without transposing anything in memory.  The B operand may
+// come from two tensors: stacked along N (the gate and up projections share
+// one 256-wide tile: columns [0,128) are W_gate rows, [128,256) the matching
+// W_up rows) or concatenated along K (dx = dg W_gate + dh W_up).
+//
+// Block = 6 warps: warp 0 issues TMA, warp 1 allocates tensor memory and
+// issues the MMAs (one thread), warps 2..5 drain the accumulators (each warp
+// may only touch its 32-lane quarter of tensor memory) and run the epilogue.
+// Two 128x256 fp32 accumulators in tensor memory (all 512 columns) let the
+// epilogue of one tile overlap the main loop of the next.  Every wait is
+// bounded (see mbar_wait): on a timeout the block records STAPLE_ETIMEOUT,
+// drains its outstanding copies and releases tensor memory before exiting.
+#pragma once
+
+#include "common.cuh"
+
+namespace stp {
+namespace tc {
+
+constexpr int BM = 128;
+constexpr int BN = 256;
+constexpr int BK = 64;
+constexpr int STAGES = 4;
+constexpr int kThreads = 192;
+constexpr int A_STAGE = BM * BK * 2;  // 16 KiB
+constexpr int B_STAGE = BN * BK * 2;  // 32 KiB
+constexpr int STAGE_BYTES = A_STAGE + B_STAGE;
+constexpr int kTmemCols = 512;
+constexpr int kSmemBytes = STAGES * STAGE_BYTES + 1024 /*align*/ + 256 /*barriers*/;
+
+enum BSrc { B_ONE = 0, B_NHALF = 1, B_KSPLIT = 2 };
+enum Epi { EPI_BF16 = 0, EPI_F32 = 1, EPI_GATEUP = 2, EPI_DZ = 3 };
+
+struct Params {
+  int32_t M, N, K;            // output rows, output columns (features for GATEUP / DZ), K
+  int32_t tiles_m, tiles_n, k_blocks;
+  int32_t ksplit;             // B_KSPLIT: first k served by the second B tensor
+  int32_t group_m;            // tile raster: group_m M-blocks per sweep over N
+  // EPI_BF16 / EPI_F32: out[m * ldo + n]; rows m >= m_split go to out2[(m - m_split) * ldo + n]
+  void* out;
+  void* out2;
+  int64_t ldo;
+  int32_t m_split;
+  // EPI_GATEUP
+  uint16_t* z;
+  uint16_t* g_save;
+  uint16_t* h_save;
+  int64_t ldf;                // row pitch of z / g / h (= F)
+  const uint16_t* e_base;
+  int64_t e_pitch;
+  const int32_t* e_index;
+  int64_t e_rows;
+  int32_t e_mode;             // staple_embed_mode
+  // EPI_DZ
+  const uint16_t* g_in;
+  const uint16_t* h_in;
+  uint16_t* dgh;              // [M][2 * ldf]: dg in [0, F), dh in [F, 2F)
+  int32_t* err;
+};
+
+__device__ __forceinline__ void tile_coords(int t, const Params& p, int& mb, int& nb) {
+  const int per_group = p.group_m * p.tiles_n;
+  const int g = t / per_group;
+  const int first_m = g * p.group_m;
+  const int rows = min(p.group_m, p.tiles_m - first_m);
+  const int r = t - g * per_group;
+  mb = first_m + r % rows;
+  nb = r / rows;
+}
+
+// --------------------------------------------------------------------------
+// Epilogue helpers (one thread = one accumulator row, 32 columns per load)
+// --------------------------------------------------------------------------
+__device__ __forceinline__ void store_bf16x32(uint16_t* dst, const float* v) {
+  uint4* d = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    uint4 w;
+    w.x = pack_bf2(v[8 * i + 0], v[8 * i + 1]);
+    w.y = pack_bf2(v[8 * i + 2], v[8 * i + 3]);
+    w.z = pack_bf2(v[8 * i + 4], v[8 * i + 5]);
+    w.w = pack_bf2(v[8 * i + 6], v[8 * i + 7]);
+    d[i] = w;
+  }
+}
+
+__device__ __forceinline__ void load_bf16x32(const uint16_t* src, float* v) {
+  const uint4* s = reinterpret_cast<const uint4*>(src);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const uint4 w = __ldg(s + i);
+    v[8 * i + 0] = bf_lo(w.x);
+    v[8 * i + 1] = bf_hi(w.x);
+    v[8 * i + 2] = bf_lo(w.y);
+    v[8 * i + 3] = bf_hi(w.y);
+    v[8 * i + 4] = bf_lo(w.z);
+    v[8 * i + 5] = bf_hi(w.z);
+    v[8 * i + 6] = bf_lo(w.w);
+    v[8 * i + 7] = bf_hi(w.w);
+  }
+}
+
+template <int EPI>
+__device__ __forceinline__ void epilogue_tile(const Params& p, uint32_t tacc, int m, int nb) {
+  const bool row_ok = m < p.M;
+  if constexpr (EPI == EPI_BF16 || EPI == EPI_F32) {
+#pragma unroll 1
+    for (int c = 0; c < BN / 32; ++c) {
+      uint32_t r[32];
+      tmem_ld32(tacc + c * 32, r);
+      tmem_ld_wait(r);
+      const int n = nb * BN + c * 32;
+      if (row_ok && n < p.N) {
+        float v[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+        if constexpr (EPI == EPI_BF16) {
+          store_bf16x32(static_cast<uint16_t*>(p.out) + int64_t(m) * p.ldo + n, v);
+        } else {
+          float* base = m < p.m_split
+                            ? static_cast<float*>(p.out) + int64_t(m) * p.ldo
+                            : static_cast<float*>(p.out2) + int64_t(m - p.m_split) * p.ldo;
+          float4* d = reinterpret_cast<float4*>(base + n);
+#pragma unroll
+          for (int i = 0; i < 8; ++i)
+            d[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+        }
+      }
+    }
+  } else if constexpr (EPI == EPI_GATEUP) {
+    // Accumulator columns [0,128): g for features f0..f0+127; [128,256): u.
+    const uint16_t* erow = nullptr;
+    if (row_ok && p.e_mode != STAPLE_EMBED_NONE) {
+      const int64_t idx = p.e_index[m];
+      if (idx < 0 || idx >= p.e_rows) {
+        report(p.err, STAPLE_EIDRANGE);
+      } else {
+        erow = p.e_base + idx * p.e_pitch;
+      }
+    }
+    const int f0 = nb * (BN / 2);
+#pragma unroll 1
+    for (int c = 0; c < BN / 64; ++c) {
+      uint32_t rg[32], ru[32];
+      tmem_ld32(tacc + c * 32, rg);
+      tmem_ld32(tacc + BN / 2 + c * 32, ru);
+      tmem_ld_wait(rg);
+      reg_fence(ru);
+      const int f = f0 + c * 32;
+      if (row_ok && f < p.N) {
+        float e[32];
+        if (erow) {
+          load_bf16x32(erow + f, e);
+        } else {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) e[i] = 0.0f;
+        }
+        float g[32], h[32], z[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          g[i] = __uint_as_float(rg[i]);
+          h[i] = __uint_as_float(ru[i]) + e[i];
+          z[i] = g[i] * sigmoid_f(g[i]) * h[i];
+        }
+        const int64_t off = int64_t(m) * p.ldf + f;
+        store_bf16x32(p.z + off, z);
+        if (p.g_save) store_bf16x32(p.g_save + off, g);
+        if (p.h_save) store_bf16x32(p.h_save + off, h);
+      }
+    }
+  } else {  // EPI_DZ: accumulator = dz for features [nb*256, nb*256 + 256)
+#pragma unroll 1
+    for (int c = 0; c < BN / 32; ++c) {
+      uint32_t r[32];
+      tmem_ld32(tacc + c * 32, r);
+      tmem_ld_wait(r);
+      const int f = nb * BN + c * 32;
+      if (row_ok && f < p.N) {
+        const int64_t off = int64_t(m) * p.ldf + f;
+        float g[32], h[32], dg[32], dh[32];
+        load_bf16x32(p.g_in + off, g);
+        load_bf16x32(p.h_in + off, h);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          const float dz = __uint_as_float(r[i]);
+          const float s = sigmoid_f(g[i]);
+          dh[i] = dz * g[i] * s;
+          dg[i] = dz * h[i] * (s * (1.0f + g[i] * (1.0f - s)));
+        }
+        uint16_t* row = p.dgh + int64_t(m) * (2 * p.ldf);
+        store_bf16x32(row + f, dg);
+        store_bf16x32(row + p.ldf + f, dh);
+      }
+    }
+  }
+}
+
+// --------------------------------------------------------------------------
+// The kernel
+// --------------------------------------------------------------------------
+template <bool A_MN, bool B_MN, int BSRC, int EPI>
+__global__ void __launch_bounds__(kThreads, 1)
+    gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB0,
+                const __grid_constant__ CUtensorMap tmB1, const Params p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + STAGES * A_STAGE;
+  uint64_t* full = reinterpret_cast<uint64_t*>(sB + STAGES * B_STAGE);
+  uint64_t* empty = full + STAGES;
+  uint64_t* tfull = empty + STAGES;
+  uint64_t* tempty = tfull + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tempty + 2);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+#pragma unroll
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    mbar_init(&tfull[0], 1);
+    mbar_init(&tfull[1], 1);
+    mbar_init(&tempty[0], 4);
+    mbar_init(&tempty[1], 4);
+    *abort_flag = 0;
+    fence_barrier_init();
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB0);
+    if (BSRC != B_ONE) tma_prefetch_desc(&tmB1);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const int ntiles = p.tiles_m * p.tiles_n;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ------------------------------------------------------------ producer
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      int issued = 0;
+      for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
+        int mb, nb;
+        tile_coords(t, p, mb, nb);
+        const int m0 = mb * BM;
+        for (int kb = 0; kb < p.k_blocks; ++kb) {
+          if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag, p.err)) {
+            ok = false;
+            break;
+          }
+          uint64_t* bar = &full[stage];
+          mbar_arrive_expect_tx(bar, STAGE_BYTES);
+          uint8_t* a = sA + stage * A_STAGE;
+          uint8_t* b = sB + stage * B_STAGE;
+          const int k0 = kb * BK;
+          if (A_MN) {
+            tma_load_2d(&tmA, bar, a, m0, k0);
+            tma_load_2d(&tmA, bar, a + A_STAGE / 2, m0 + 64, k0);
+          } else {
+            tma_load_2d(&tmA, bar, a, k0, m0);
+          }
+          if (BSRC == B_NHALF) {
+            const int n0 = nb * (BN / 2);
+            tma_load_2d(&tmB0, bar, b, k0, n0);
+            tma_load_2d(&tmB1, bar, b + B_STAGE / 2, k0, n0);
+          } else {
+            const CUtensorMap* mp = &tmB0;
+            int kk = k0;
+            if (BSRC == B_KSPLIT && k0 >= p.ksplit) {
+              mp = &tmB1;
+              kk = k0 - p.ksplit;
+            }
+            const int n0 = nb * BN;
+            if (B_MN) {
+#pragma unroll
+              for (int i = 0; i < 4; ++i) tma_load_2d(mp, bar, b + i * (B_STAGE / 4), n0 + 64 * i, kk);
+            } else {
+              tma_load_2d(mp, bar, b, kk, n0);
+              tma_load_2d(mp, bar, b + B_STAGE / 2, kk, n0 + 128);
+            }
+          }
+          ++issued;
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+      }
+      if (!ok) {
+        // Let the copies already issued land before the block goes away.
+        for (int i = 0; i < STAGES && issued > 0; ++i, --issued) {
+          if (--stage < 0) {
+            stage = STAGES - 1;
+            phase ^= 1;
+          }
+          const uint64_t t0 = globaltimer();
+          while (!mbar_try_wait(&full[stage], phase) && globaltimer() - t0 < 1000000ull) {
+          }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ---------------------------------------------------------- MMA issuer
+      const uint32_t idesc = idesc_bf16_f32(BM, BN, A_MN, B_MN);
+      int stage = 0;
+      uint32_t phase = 0;
+      int iter = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x, ++iter) {
+        const int buf = iter & 1;
+        const uint32_t use = uint32_t(iter >> 1);
+        if (!mbar_wait(&tempty[buf], (use & 1) ^ 1, abort_flag, p.err)) break;
+        tc_fence_after();
+        const uint32_t dacc = tmem_base + uint32_t(buf * BN);
+        for (int kb = 0; kb < p.k_blocks; ++kb) {
+          if (!mbar_wait(&full[stage], phase, abort_flag, p.err)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a_addr = smem_u32(sA + stage * A_STAGE);
+          const uint32_t b_addr = smem_u32(sB + stage * B_STAGE);
+#pragma unroll
+          for (int k = 0; k < BK / 16; ++k) {
+            const uint64_t ad = A_MN ? sw128_desc(a_addr + k * 2048, A_STAGE / 2, 1024)
+                                     : sw128_desc(a_addr + k * 32, 16, 1024);
+            const uint64_t bd = B_MN ? sw128_desc(b_addr + k * 2048, B_STAGE / 4, 1024)
+                                     : sw128_desc(b_addr + k * 32, 16, 1024);
+            umma_bf16(dacc, ad, bd, idesc, (kb | k) != 0 ? 1u : 0u);
+          }
+          umma_commit(&empty[stage]);
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+        if (ok) umma_commit(&tfull[buf]);
+      }
+    }
+  } else {
+    // -------------------------------------------------------------- epilogue
+    const int q = warp & 3;
+    const int row = q * 32 + lane;
+    int iter = 0;
+    for (int t = blockIdx.x; t < ntiles; t += gridDim.x, ++iter) {
+      const int buf = iter & 1;
+      const uint32_t use = uint32_t(iter >> 1);
+      int mb, nb;
+      tile_coords(t, p, mb, nb);
+      const bool ok = mbar_wait(&tfull[buf], use & 1, abort_flag, p.err);
+      if (!__all_sync(0xffffffffu, ok)) break;
+      tc_fence_after();
+      const uint32_t tacc = tmem_base + (uint32_t(q * 32) << 16) + uint32_t(buf * BN);
+      epilogue_tile<EPI>(p, tacc, mb * BM + row, nb);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&tempty[buf]);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) {
+    __syncwarp();
+    tmem_dealloc(tmem_base, kTmemCols);
+  }
+}
+
+}  // namespace tc
+}  // namespace stp

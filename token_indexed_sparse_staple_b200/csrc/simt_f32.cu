@@ -1,0 +1,233 @@
+// K11: the STAPLE layer in fp32 on CUDA cores.
+//
+// The fp32 workload asks for agreement with the fp64 definition to 1e-5 of
+// the largest output; tf32 tensor-core products (10-bit mantissa) cannot meet
+// that, so fp32 runs as a plain tiled SIMT GEMM (64x64 block tile, 4x4 per
+// thread, fp32 accumulation) with the same fused epilogues as the bf16 path:
+// E-row add + SiLU gating for the gate/up pair, the SwiGLU backward for dz.
+#include "common.cuh"
+#include "internal.h"
+
+namespace stp {
+
+namespace {
+
+constexpr int ST = 64;   // block tile (M and N)
+constexpr int SK = 16;   // k tile
+
+enum SEpi { S_STORE = 0, S_GATEUP = 1, S_DZ = 2 };
+
+struct SParams {
+  int M, N, K;
+  const float* A;
+  int64_t lda;
+  const float* B0;
+  const float* B1;  // DUAL: second B operand; KSPLIT: operand for k >= ksplit
+  int64_t ldb;
+  int ksplit;       // 0 = no split
+  float* out;
+  float* out2;
+  int64_t ldo;
+  int m_split;
+  // gate/up
+  float* z;
+  float* g_save;
+  float* h_save;
+  int64_t ldf;
+  const float* e_base;
+  int64_t e_pitch;
+  const int32_t* e_index;
+  int64_t e_rows;
+  int e_mode;
+  // dz
+  const float* g_in;
+  const float* h_in;
+  float* dgh;
+  int32_t* err;
+};
+
+__device__ __forceinline__ float silu_acc(float g) { return g / (1.0f + expf(-g)); }
+
+template <bool A_MN, bool B_MN, int EPI, bool DUAL>
+__global__ void __launch_bounds__(256) sgemm_kernel(const SParams p) {
+  __shared__ float As[SK][ST];
+  __shared__ float Bs[SK][ST];
+  __shared__ float Cs[DUAL ? SK : 1][DUAL ? ST : 1];
+  const int tid = threadIdx.x;
+  const int tx = tid & 15, ty = tid >> 4;
+  const int m0 = blockIdx.y * ST, n0 = blockIdx.x * ST;
+  float acc[4][4] = {};
+  float acc2[DUAL ? 4 : 1][DUAL ? 4 : 1] = {};
+
+  for (int k0 = 0; k0 < p.K; k0 += SK) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int idx = tid + i * 256;
+      int mm, kk;
+      if (A_MN) { kk = idx / ST; mm = idx % ST; } else { mm = idx / SK; kk = idx % SK; }
+      const int m = m0 + mm, k = k0 + kk;
+      float v = 0.0f;
+      if (m < p.M && k < p.K) v = A_MN ? p.A[int64_t(k) * p.lda + m] : p.A[int64_t(m) * p.lda + k];
+      As[kk][mm] = v;
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int idx = tid + i * 256;
+      int nn, kk;
+      if (B_MN) { kk = idx / ST; nn = idx % ST; } else { nn = idx / SK; kk = idx % SK; }
+      const int n = n0 + nn, k = k0 + kk;
+      float v = 0.0f, v2 = 0.0f;
+      if (n < p.N && k < p.K) {
+        const bool second = p.ksplit > 0 && k >= p.ksplit;
+        const int kl = second ? k - p.ksplit : k;
+        const int64_t off = B_MN ? int64_t(kl) * p.ldb + n : int64_t(n) * p.ldb + kl;
+        v = (second ? p.B1 : p.B0)[off];
+        if (DUAL) v2 = p.B1[off];
+      }
+      Bs[kk][nn] = v;
+      if (DUAL) Cs[kk][nn] = v2;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int kk = 0; kk < SK; ++kk) {
+      float a[4], b[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) a[i] = As[kk][ty * 4 + i];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) b[j] = Bs[kk][tx * 4 + j];
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(a[i], b[j], acc[i][j]);
+      if constexpr (DUAL) {
+        float b2[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) b2[j] = Cs[kk][tx * 4 + j];
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+          for (int j = 0; j < 4; ++j) acc2[i][j] = fmaf(a[i], b2[j], acc2[i][j]);
+      }
+    }
+    __syncthreads();
+  }
+
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int m = m0 + ty * 4 + i;
+    if (m >= p.M) continue;
+    const float* erow = nullptr;
+    if constexpr (EPI == S_GATEUP) {
+      if (p.e_mode != STAPLE_EMBED_NONE) {
+        const int64_t idx = p.e_index[m];
+        if (idx < 0 || idx >= p.e_rows) report(p.err, STAPLE_EIDRANGE);
+        else erow = p.e_base + idx * p.e_pitch;
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int n = n0 + tx * 4 + j;
+      if (n >= p.N) continue;
+      if constexpr (EPI == S_STORE) {
+        float* row = m < p.m_split ? p.out + int64_t(m) * p.ldo
+                                   : p.out2 + int64_t(m - p.m_split) * p.ldo;
+        row[n] = acc[i][j];
+      } else if constexpr (EPI == S_GATEUP) {
+        const float g = acc[i][j];
+        const float h = acc2[DUAL ? i : 0][DUAL ? j : 0] + (erow ? erow[n] : 0.0f);
+        const int64_t off = int64_t(m) * p.ldf + n;
+        p.z[off] = silu_acc(g) * h;
+        if (p.g_save) p.g_save[off] = g;
+        if (p.h_save) p.h_save[off] = h;
+      } else {
+        const int64_t off = int64_t(m) * p.ldf + n;
+        const float dz = acc[i][j];
+        const float g = p.g_in[off], h = p.h_in[off];
+        const float s = 1.0f / (1.0f + expf(-g));
+        float* row = p.dgh + int64_t(m) * (2 * p.ldf);
+        row[n] = dz * h * (s * (1.0f + g * (1.0f - s)));
+        row[p.ldf + n] = dz * g * s;
+      }
+    }
+  }
+}
+
+template <bool A_MN, bool B_MN, int EPI, bool DUAL>
+staple_status run(const SParams& p, cudaStream_t st) {
+  if (p.M == 0 || p.N == 0) return STAPLE_OK;
+  const dim3 grid((p.N + ST - 1) / ST, (p.M + ST - 1) / ST);
+  sgemm_kernel<A_MN, B_MN, EPI, DUAL><<<grid, 256, 0, st>>>(p);
+  return cudaGetLastError() == cudaSuccess ? STAPLE_OK : STAPLE_ECUDA;
+}
+
+}  // namespace
+
+staple_status f32_ffn_fwd(int T, int D, int F, const float* x, const staple_embed* e,
+                          const float* wg, const float* wu, const float* wd, float* z, float* y,
+                          float* g_save, float* h_save, int32_t* err, cudaStream_t st) {
+  SParams p{};
+  // gate/up: [T][F] pair = x [T][D] . W^T, W [F][D] K-major
+  p.M = T; p.N = F; p.K = D;
+  p.A = x; p.lda = D; p.B0 = wg; p.B1 = wu; p.ldb = D;
+  p.z = z; p.g_save = g_save; p.h_save = h_save; p.ldf = F;
+  p.e_mode = e ? e->mode : STAPLE_EMBED_NONE;
+  if (e && e->mode != STAPLE_EMBED_NONE) {
+    p.e_base = static_cast<const float*>(e->base);
+    p.e_pitch = e->row_pitch;
+    p.e_index = e->index;
+    p.e_rows = e->n_rows;
+  }
+  p.err = err;
+  staple_status s = run<false, false, S_GATEUP, true>(p, st);
+  if (s != STAPLE_OK) return s;
+  SParams q{};
+  q.M = T; q.N = D; q.K = F;
+  q.A = z; q.lda = F; q.B0 = wd; q.ldb = F;
+  q.out = y; q.ldo = D; q.m_split = T;
+  return run<false, false, S_STORE, false>(q, st);
+}
+
+staple_status f32_dz(int T, int D, int F, const float* dy, const float* g_save,
+                     const float* h_save, const float* wd, float* dgh, cudaStream_t st) {
+  SParams p{};
+  // dz [T][F] = dY [T][D] . W_down [D][F]  (B MN-major: n = f contiguous)
+  p.M = T; p.N = F; p.K = D;
+  p.A = dy; p.lda = D; p.B0 = wd; p.ldb = F;
+  p.g_in = g_save; p.h_in = h_save; p.dgh = dgh; p.ldf = F;
+  return run<false, true, S_DZ, false>(p, st);
+}
+
+staple_status f32_ffn_bwd(int T, int D, int F, const float* dy, const float* x, const float* z,
+                          const float* dgh, const float* wg, const float* wu, float* dx,
+                          float* dwg, float* dwu, float* dwd, cudaStream_t st) {
+  staple_status s;
+  if (dx) {
+    // dx [T][D] = dgh [T][2F] . [W_gate; W_up] ([2F][D], n = d contiguous)
+    SParams p{};
+    p.M = T; p.N = D; p.K = 2 * F;
+    p.A = dgh; p.lda = 2 * F; p.B0 = wg; p.B1 = wu; p.ldb = D; p.ksplit = F;
+    p.out = dx; p.ldo = D; p.m_split = T;
+    if ((s = run<false, true, S_STORE, false>(p, st)) != STAPLE_OK) return s;
+  }
+  if (dwg || dwu) {
+    // dW [f][d] = sum_t dgh[t][f] x[t][d]  (A MN-major over dgh, B MN-major over x)
+    SParams p{};
+    const bool both = dwg && dwu;
+    p.M = both ? 2 * F : F; p.N = D; p.K = T;
+    p.A = dwg ? dgh : dgh + F; p.lda = 2 * F;
+    p.B0 = x; p.ldb = D;
+    p.out = dwg ? dwg : dwu; p.out2 = dwu; p.ldo = D; p.m_split = both ? F : p.M;
+    if ((s = run<true, true, S_STORE, false>(p, st)) != STAPLE_OK) return s;
+  }
+  if (dwd) {
+    // dW_down [d][f] = sum_t dY[t][d] z[t][f]
+    SParams p{};
+    p.M = D; p.N = F; p.K = T;
+    p.A = dy; p.lda = D; p.B0 = z; p.ldb = F;
+    p.out = dwd; p.ldo = F; p.m_split = D;
+    if ((s = run<true, true, S_STORE, false>(p, st)) != STAPLE_OK) return s;
+  }
+  return STAPLE_OK;
+}
+
+}  // namespace stp

@@ -1,0 +1,461 @@
+// The extern "C" entry points of libstaple: argument checks, host-side
+// bookkeeping (contexts, registered tables, the hot-row cache) and the
+// stream orchestration around the kernels.  Every compute step runs in the
+// CUDA kernels of the other translation units.
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstring>
+#include <new>
+#include <vector>
+
+#include "../../include/staple.h"
+#include "internal.h"
+
+struct staple_context {
+  stp::DeviceInfo di;
+  int32_t* d_err;          // device error word
+  cudaEvent_t ev_main;     // main -> side ordering
+  cudaEvent_t ev_side;     // side -> main ordering
+};
+
+struct staple_table {
+  void* base;              // caller's pointer (host or device)
+  const uint8_t* dev;      // device-visible address of the first row
+  size_t bytes;
+  int64_t V;
+  int32_t F;
+  int32_t groups;
+  staple_dtype dtype;
+  uint32_t flags;
+  bool registered;         // we called cudaHostRegister
+};
+
+struct staple_cache {
+  int device;
+  int32_t K;
+  int32_t cap;             // hash capacity (power of two)
+  int64_t row_bytes;       // groups * F * element size
+  void* rows;              // [K][groups * F]
+  int32_t* hkeys;          // [cap], -1 = empty
+  int32_t* hvals;          // [cap]
+  int32_t* hot_dev;        // [K] ids in slot order, followed by K itself
+  std::vector<int32_t> hot;
+};
+
+namespace {
+
+inline size_t esize(staple_dtype d) { return d == STAPLE_BF16 ? 2 : 4; }
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+inline cudaStream_t cs(staple_stream s) { return reinterpret_cast<cudaStream_t>(s); }
+
+staple_status set_device(const staple_context* ctx) {
+  return cudaSetDevice(ctx->di.device) == cudaSuccess ? STAPLE_OK : STAPLE_ECUDA;
+}
+
+#define STP_TRY(expr)                              \
+  do {                                             \
+    staple_status _s = (expr);                     \
+    if (_s != STAPLE_OK) return _s;                \
+  } while (0)
+#define STP_CUDA(expr)                                        \
+  do {                                                        \
+    if ((expr) != cudaSuccess) return STAPLE_ECUDA;           \
+  } while (0)
+
+staple_status check_embed(const staple_embed* e, staple_dtype dt, int F) {
+  if (!e || e->mode == STAPLE_EMBED_NONE) return STAPLE_OK;
+  if (e->mode != STAPLE_EMBED_TABLE && e->mode != STAPLE_EMBED_ROWS) return STAPLE_EINVAL;
+  if (!e->base || !e->index || e->n_rows <= 0 || e->row_pitch < F) return STAPLE_EINVAL;
+  if (dt == STAPLE_BF16 && (!aligned16(e->base) || (e->row_pitch % 8) != 0)) return STAPLE_EINVAL;
+  return STAPLE_OK;
+}
+
+staple_status check_dims(staple_dtype dt, int32_t T, int32_t D, int32_t F) {
+  if (dt != STAPLE_BF16 && dt != STAPLE_F32) return STAPLE_EINVAL;
+  if (T < 0 || D <= 0 || F <= 0) return STAPLE_EINVAL;
+  if (dt == STAPLE_BF16 && ((D % 64) != 0 || (F % 64) != 0)) return STAPLE_EINVAL;
+  if (dt == STAPLE_F32 && (F % 8) != 0) return STAPLE_EINVAL;
+  if (int64_t(T) * 2 * F > (int64_t(1) << 31) * 4) return STAPLE_EUNSUPPORTED;
+  return STAPLE_OK;
+}
+
+bool ptrs_ok(staple_dtype dt, std::initializer_list<const void*> ps) {
+  for (const void* p : ps) {
+    if (!p) return false;
+    if (dt == STAPLE_BF16 && !aligned16(p)) return false;
+  }
+  return true;
+}
+
+}  // namespace
+
+extern "C" {
+
+int staple_abi_version(void) { return STAPLE_ABI_VERSION; }
+
+const char* staple_status_string(staple_status s) {
+  switch (s) {
+    case STAPLE_OK: return "STAPLE_OK";
+    case STAPLE_EINVAL: return "STAPLE_EINVAL: invalid argument";
+    case STAPLE_EIDRANGE: return "STAPLE_EIDRANGE: token id outside [0, V)";
+    case STAPLE_ECUDA: return "STAPLE_ECUDA: CUDA runtime error";
+    case STAPLE_ENOMEM: return "STAPLE_ENOMEM: allocation failed";
+    case STAPLE_ETIMEOUT: return "STAPLE_ETIMEOUT: a bounded kernel wait ran out";
+    case STAPLE_EUNSUPPORTED: return "STAPLE_EUNSUPPORTED: not supported by this build";
+    case STAPLE_ENODEV: return "STAPLE_ENODEV: no sm_100 device";
+  }
+  return "STAPLE_UNKNOWN";
+}
+
+staple_status staple_context_create(int device, staple_context** out) {
+  if (!out) return STAPLE_EINVAL;
+  *out = nullptr;
+  int n = 0;
+  if (cudaGetDeviceCount(&n) != cudaSuccess || device < 0 || device >= n) return STAPLE_ENODEV;
+  cudaDeviceProp prop;
+  STP_CUDA(cudaGetDeviceProperties(&prop, device));
+  if (prop.major != 10) return STAPLE_ENODEV;
+  STP_CUDA(cudaSetDevice(device));
+  staple_context* c = new (std::nothrow) staple_context();
+  if (!c) return STAPLE_ENOMEM;
+  c->di.device = device;
+  c->di.num_sms = prop.multiProcessorCount;
+  if (cudaMalloc(&c->d_err, sizeof(int32_t)) != cudaSuccess) {
+    delete c;
+    return STAPLE_ENOMEM;
+  }
+  if (cudaMemset(c->d_err, 0, sizeof(int32_t)) != cudaSuccess ||
+      cudaEventCreateWithFlags(&c->ev_main, cudaEventDisableTiming) != cudaSuccess ||
+      cudaEventCreateWithFlags(&c->ev_side, cudaEventDisableTiming) != cudaSuccess) {
+    cudaFree(c->d_err);
+    delete c;
+    return STAPLE_ECUDA;
+  }
+  *out = c;
+  return STAPLE_OK;
+}
+
+staple_status staple_context_destroy(staple_context* ctx) {
+  if (!ctx) return STAPLE_OK;
+  cudaSetDevice(ctx->di.device);
+  cudaEventDestroy(ctx->ev_main);
+  cudaEventDestroy(ctx->ev_side);
+  cudaFree(ctx->d_err);
+  delete ctx;
+  return STAPLE_OK;
+}
+
+staple_status staple_get_error(staple_context* ctx, staple_stream stream, int32_t* device_error) {
+  if (!ctx || !device_error) return STAPLE_EINVAL;
+  STP_TRY(set_device(ctx));
+  STP_CUDA(cudaStreamSynchronize(cs(stream)));
+  int32_t h = 0;
+  STP_CUDA(cudaMemcpy(&h, ctx->d_err, sizeof(h), cudaMemcpyDeviceToHost));
+  STP_CUDA(cudaMemset(ctx->d_err, 0, sizeof(int32_t)));
+  *device_error = h;
+  return STAPLE_OK;
+}
+
+// ------------------------------------------------------------------ tables
+
+staple_status staple_table_register(staple_context* ctx, void* base, size_t bytes, int64_t V,
+                                    int32_t F, int32_t groups, staple_dtype dtype, uint32_t flags,
+                                    staple_table** out) {
+  if (!ctx || !base || !out || V <= 0 || F <= 0 || groups <= 0) return STAPLE_EINVAL;
+  if (dtype != STAPLE_BF16 && dtype != STAPLE_F32) return STAPLE_EINVAL;
+  const uint32_t loc = flags & (STAPLE_TABLE_DEVICE | STAPLE_TABLE_HOST_PINNED |
+                                STAPLE_TABLE_HOST_REGISTER);
+  if (loc != STAPLE_TABLE_DEVICE && loc != STAPLE_TABLE_HOST_PINNED &&
+      loc != STAPLE_TABLE_HOST_REGISTER)
+    return STAPLE_EINVAL;
+  const size_t need = size_t(V) * size_t(groups) * size_t(F) * esize(dtype);
+  if (bytes < need || !aligned16(base) || (size_t(F) * esize(dtype)) % 16 != 0) return STAPLE_EINVAL;
+  STP_TRY(set_device(ctx));
+  staple_table* t = new (std::nothrow) staple_table();
+  if (!t) return STAPLE_ENOMEM;
+  t->base = base;
+  t->bytes = bytes;
+  t->V = V;
+  t->F = F;
+  t->groups = groups;
+  t->dtype = dtype;
+  t->flags = loc;
+  t->registered = false;
+  if (loc == STAPLE_TABLE_DEVICE) {
+    t->dev = static_cast<const uint8_t*>(base);
+  } else {
+    if (loc == STAPLE_TABLE_HOST_REGISTER) {
+      if (cudaHostRegister(base, bytes, cudaHostRegisterMapped | cudaHostRegisterPortable) !=
+          cudaSuccess) {
+        cudaGetLastError();
+        delete t;
+        return STAPLE_ECUDA;
+      }
+      t->registered = true;
+    }
+    void* dp = nullptr;
+    if (cudaHostGetDevicePointer(&dp, base, 0) != cudaSuccess) {
+      cudaGetLastError();
+      if (t->registered) cudaHostUnregister(base);
+      delete t;
+      return STAPLE_ECUDA;
+    }
+    t->dev = static_cast<const uint8_t*>(dp);
+  }
+  *out = t;
+  return STAPLE_OK;
+}
+
+staple_status staple_table_unregister(staple_table* t) {
+  if (!t) return STAPLE_OK;
+  if (t->registered) cudaHostUnregister(t->base);
+  delete t;
+  return STAPLE_OK;
+}
+
+// ------------------------------------------------------------------- cache
+
+staple_status staple_cache_build(staple_context* ctx, const staple_table* table,
+                                 const int64_t* freq, double frac, staple_stream stream,
+                                 staple_cache** out) {
+  if (!ctx || !table || !freq || !out || !(frac >= 0.0 && frac <= 1.0)) return STAPLE_EINVAL;
+  *out = nullptr;
+  STP_TRY(set_device(ctx));
+  const int64_t V = table->V;
+  if (V > INT32_MAX) return STAPLE_EUNSUPPORTED;
+  int64_t K = frac > 0 ? int64_t(std::ceil(frac * double(V) - 1e-9)) : 0;
+  K = std::min<int64_t>(std::max<int64_t>(K, 0), V);
+  std::vector<int32_t> order(V);
+  for (int64_t i = 0; i < V; ++i) order[i] = int32_t(i);
+  std::partial_sort(order.begin(), order.begin() + K, order.end(), [&](int32_t a, int32_t b) {
+    return freq[a] > freq[b] || (freq[a] == freq[b] && a < b);
+  });
+  staple_cache* c = new (std::nothrow) staple_cache();
+  if (!c) return STAPLE_ENOMEM;
+  c->device = ctx->di.device;
+  c->K = int32_t(K);
+  int32_t cap = 16;
+  while (cap < 2 * K) cap <<= 1;
+  c->cap = cap;
+  c->row_bytes = int64_t(table->groups) * table->F * int64_t(esize(table->dtype));
+  c->hot.assign(order.begin(), order.begin() + K);
+  cudaStream_t st = cs(stream);
+  bool ok = cudaMalloc(&c->rows, size_t(std::max<int64_t>(K, 1)) * c->row_bytes) == cudaSuccess &&
+            cudaMalloc(&c->hkeys, size_t(cap) * 4) == cudaSuccess &&
+            cudaMalloc(&c->hvals, size_t(cap) * 4) == cudaSuccess &&
+            cudaMalloc(&c->hot_dev, size_t(K + 1) * 4) == cudaSuccess;
+  if (!ok) {
+    cudaGetLastError();
+    staple_cache_free(c);
+    return STAPLE_ENOMEM;
+  }
+  std::vector<int32_t> hk(c->hot);
+  hk.push_back(int32_t(K));
+  ok = cudaMemsetAsync(c->hkeys, 0xFF, size_t(cap) * 4, st) == cudaSuccess &&
+       cudaMemcpyAsync(c->hot_dev, hk.data(), hk.size() * 4, cudaMemcpyHostToDevice, st) ==
+           cudaSuccess &&
+       stp::launch_cache_fill(c->hot_dev, int(K), c->hkeys, c->hvals, uint32_t(cap - 1), st) ==
+           STAPLE_OK &&
+       stp::launch_copy_rows(table->dev, c->row_bytes, c->row_bytes, c->hot_dev,
+                             c->hot_dev + K, c->rows, ctx->di.num_sms, st) == STAPLE_OK &&
+       cudaStreamSynchronize(st) == cudaSuccess;
+  if (!ok) {
+    staple_cache_free(c);
+    return STAPLE_ECUDA;
+  }
+  *out = c;
+  return STAPLE_OK;
+}
+
+staple_status staple_cache_info(const staple_cache* c, int32_t* K, int32_t* cap) {
+  if (!c) return STAPLE_EINVAL;
+  if (K) *K = c->K;
+  if (cap) *cap = c->cap;
+  return STAPLE_OK;
+}
+
+staple_status staple_cache_hot_ids(const staple_cache* c, int32_t* hot_ids) {
+  if (!c || (!hot_ids && c->K > 0)) return STAPLE_EINVAL;
+  if (c->K > 0) std::memcpy(hot_ids, c->hot.data(), size_t(c->K) * 4);
+  return STAPLE_OK;
+}
+
+staple_status staple_cache_rows(const staple_cache* c, const void** rows) {
+  if (!c || !rows) return STAPLE_EINVAL;
+  *rows = c->rows;
+  return STAPLE_OK;
+}
+
+staple_status staple_cache_free(staple_cache* c) {
+  if (!c) return STAPLE_OK;
+  cudaSetDevice(c->device);
+  if (c->rows) cudaFree(c->rows);
+  if (c->hkeys) cudaFree(c->hkeys);
+  if (c->hvals) cudaFree(c->hvals);
+  if (c->hot_dev) cudaFree(c->hot_dev);
+  delete c;
+  return STAPLE_OK;
+}
+
+// --------------------------------------------------------------- workspace
+
+size_t staple_workspace_bytes(int32_t T, int32_t D, int32_t F, uint32_t flags) {
+  (void)D;
+  (void)flags;
+  if (T < 0 || F <= 0) return 0;
+  size_t b = stp::seg_reduce_workspace(T, F);
+  return (b + 255) & ~size_t(255);
+}
+
+// --------------------------------------------------------------- retrieval
+
+staple_status staple_dedup(staple_context* ctx, const int32_t* ids, int32_t T, int64_t V,
+                           int32_t* unique, int32_t* inverse, int32_t* seg_off,
+                           int32_t* sorted_pos, int32_t* U_dev, staple_stream stream) {
+  if (!ctx || T < 0 || V <= 0 || V > INT32_MAX || !seg_off || !U_dev) return STAPLE_EINVAL;
+  if (T > 0 && (!ids || !unique || !inverse || !sorted_pos)) return STAPLE_EINVAL;
+  if (T > stp::kMaxDedupT) return STAPLE_EUNSUPPORTED;
+  STP_TRY(set_device(ctx));
+  return stp::launch_dedup(ids, T, V, unique, inverse, seg_off, sorted_pos, U_dev, ctx->d_err,
+                           cs(stream));
+}
+
+staple_status staple_gather_unique_rows(staple_context* ctx, const staple_cache* cache,
+                                        const staple_table* table, const int32_t* unique,
+                                        const int32_t* U_dev, int32_t T, int32_t* slot,
+                                        int32_t* miss_list, int32_t* miss_count, void* rows,
+                                        staple_stream stream, staple_stream side) {
+  if (!ctx || !table || !U_dev || !slot || !miss_list || !miss_count || T < 0) return STAPLE_EINVAL;
+  if (T > 0 && (!unique || !rows)) return STAPLE_EINVAL;
+  if (!aligned16(rows)) return STAPLE_EINVAL;
+  const int64_t row_bytes = int64_t(table->groups) * table->F * int64_t(esize(table->dtype));
+  if (cache && cache->row_bytes != row_bytes) return STAPLE_EINVAL;
+  STP_TRY(set_device(ctx));
+  cudaStream_t st = cs(stream);
+  cudaStream_t sd = cs(side);
+  STP_TRY(stp::launch_probe(unique, U_dev, cache && cache->K > 0 ? cache->hkeys : nullptr,
+                            cache ? cache->hvals : nullptr,
+                            cache ? uint32_t(cache->cap - 1) : 0u, slot, miss_list, miss_count,
+                            st));
+  const bool split = sd != st;
+  if (split) {
+    STP_CUDA(cudaEventRecord(ctx->ev_main, st));
+    STP_CUDA(cudaStreamWaitEvent(sd, ctx->ev_main, 0));
+  }
+  STP_TRY(stp::launch_gather_misses(table->dev, row_bytes, row_bytes, unique, miss_list,
+                                    miss_count, rows, ctx->di.num_sms, split ? sd : st));
+  if (cache && cache->K > 0)
+    STP_TRY(stp::launch_gather_hits(cache->rows, row_bytes, U_dev, slot, rows, ctx->di.num_sms, st));
+  if (split) {
+    STP_CUDA(cudaEventRecord(ctx->ev_side, sd));
+    STP_CUDA(cudaStreamWaitEvent(st, ctx->ev_side, 0));
+  }
+  return STAPLE_OK;
+}
+
+staple_status staple_gather_rows(staple_context* ctx, const staple_cache* cache,
+                                 const staple_table* table, const int32_t* ids, int32_t T,
+                                 int32_t* unique, int32_t* inverse, int32_t* seg_off,
+                                 int32_t* sorted_pos, int32_t* U_dev, int32_t* slot,
+                                 int32_t* miss_list, int32_t* miss_count, void* rows,
+                                 staple_stream stream, staple_stream side) {
+  if (!table) return STAPLE_EINVAL;
+  STP_TRY(staple_dedup(ctx, ids, T, table->V, unique, inverse, seg_off, sorted_pos, U_dev,
+                       stream));
+  return staple_gather_unique_rows(ctx, cache, table, unique, U_dev, T, slot, miss_list,
+                                   miss_count, rows, stream, side);
+}
+
+// ------------------------------------------------------------ FFN forward
+
+staple_status staple_ffn_fwd(staple_context* ctx, staple_dtype dtype, int32_t T, int32_t D,
+                             int32_t F, const void* x, const staple_embed* embed,
+                             const void* w_gate, const void* w_up, const void* w_down, void* z,
+                             void* y, void* g_save, void* h_save, void* workspace,
+                             size_t workspace_bytes, staple_stream stream) {
+  (void)workspace;
+  (void)workspace_bytes;
+  if (!ctx) return STAPLE_EINVAL;
+  STP_TRY(check_dims(dtype, T, D, F));
+  STP_TRY(check_embed(embed, dtype, F));
+  if (!ptrs_ok(dtype, {w_gate, w_up, w_down})) return STAPLE_EINVAL;
+  if (T > 0 && !ptrs_ok(dtype, {x, z, y})) return STAPLE_EINVAL;
+  if ((g_save && !ptrs_ok(dtype, {g_save})) || (h_save && !ptrs_ok(dtype, {h_save})))
+    return STAPLE_EINVAL;
+  STP_TRY(set_device(ctx));
+  if (dtype == STAPLE_BF16)
+    return stp::tc_ffn_fwd(ctx->di, T, D, F, x, embed, w_gate, w_up, w_down, z, y, g_save, h_save,
+                           ctx->d_err, cs(stream));
+  return stp::f32_ffn_fwd(T, D, F, static_cast<const float*>(x), embed,
+                          static_cast<const float*>(w_gate), static_cast<const float*>(w_up),
+                          static_cast<const float*>(w_down), static_cast<float*>(z),
+                          static_cast<float*>(y), static_cast<float*>(g_save),
+                          static_cast<float*>(h_save), ctx->d_err, cs(stream));
+}
+
+// ----------------------------------------------------------- FFN backward
+
+staple_status staple_embed_bwd(staple_context* ctx, staple_dtype dtype, int32_t T, int32_t D,
+                               int32_t F, const void* dy, const void* g_save, const void* h_save,
+                               const void* w_down, const int32_t* sorted_pos,
+                               const int32_t* inverse, const int32_t* seg_off,
+                               const int32_t* U_dev, void* dgh, float* dE, void* workspace,
+                               size_t workspace_bytes, staple_stream stream) {
+  if (!ctx) return STAPLE_EINVAL;
+  STP_TRY(check_dims(dtype, T, D, F));
+  if (!ptrs_ok(dtype, {w_down})) return STAPLE_EINVAL;
+  if (T > 0 && !ptrs_ok(dtype, {dy, g_save, h_save, dgh})) return STAPLE_EINVAL;
+  if (dE) {
+    if (!sorted_pos || !inverse || !seg_off || !U_dev || !aligned16(dE)) return STAPLE_EINVAL;
+    const size_t need = stp::seg_reduce_workspace(T, F);
+    if (T > 0 && (!workspace || workspace_bytes < need || !aligned16(workspace)))
+      return STAPLE_EINVAL;
+  }
+  STP_TRY(set_device(ctx));
+  cudaStream_t st = cs(stream);
+  if (dtype == STAPLE_BF16)
+    STP_TRY(stp::tc_dz(ctx->di, T, D, F, dy, g_save, h_save, w_down, dgh, ctx->d_err, st));
+  else
+    STP_TRY(stp::f32_dz(T, D, F, static_cast<const float*>(dy), static_cast<const float*>(g_save),
+                        static_cast<const float*>(h_save), static_cast<const float*>(w_down),
+                        static_cast<float*>(dgh), st));
+  if (!dE) return STAPLE_OK;
+  const size_t es = esize(dtype);
+  const void* dh = static_cast<const uint8_t*>(dgh) + size_t(F) * es;
+  return stp::launch_seg_reduce(dtype == STAPLE_BF16, dh, 2 * int64_t(F), sorted_pos, inverse,
+                                seg_off, U_dev, T, F, dE, static_cast<float*>(workspace), st);
+}
+
+staple_status staple_ffn_bwd(staple_context* ctx, staple_dtype dtype, int32_t T, int32_t D,
+                             int32_t F, const void* dy, const void* x, const void* z,
+                             const void* dgh, const void* w_gate, const void* w_up, void* dx,
+                             float* dw_gate, float* dw_up, float* dw_down, void* workspace,
+                             size_t workspace_bytes, staple_stream stream) {
+  (void)workspace;
+  (void)workspace_bytes;
+  if (!ctx) return STAPLE_EINVAL;
+  STP_TRY(check_dims(dtype, T, D, F));
+  if (T > 0 && !ptrs_ok(dtype, {dy, x, z, dgh})) return STAPLE_EINVAL;
+  if (dx && !ptrs_ok(dtype, {dx, w_gate, w_up})) return STAPLE_EINVAL;
+  for (const float* p : {dw_gate, dw_up, dw_down})
+    if (p && !aligned16(p)) return STAPLE_EINVAL;
+  STP_TRY(set_device(ctx));
+  if (dtype == STAPLE_BF16)
+    return stp::tc_ffn_bwd(ctx->di, T, D, F, dy, x, z, dgh, w_gate, w_up, dx, dw_gate, dw_up,
+                           dw_down, ctx->d_err, cs(stream));
+  if (T == 0) {
+    cudaStream_t st = cs(stream);
+    if (dw_gate) STP_CUDA(cudaMemsetAsync(dw_gate, 0, size_t(F) * D * 4, st));
+    if (dw_up) STP_CUDA(cudaMemsetAsync(dw_up, 0, size_t(F) * D * 4, st));
+    if (dw_down) STP_CUDA(cudaMemsetAsync(dw_down, 0, size_t(F) * D * 4, st));
+    return STAPLE_OK;
+  }
+  return stp::f32_ffn_bwd(T, D, F, static_cast<const float*>(dy), static_cast<const float*>(x),
+                          static_cast<const float*>(z), static_cast<const float*>(dgh),
+                          static_cast<const float*>(w_gate), static_cast<const float*>(w_up),
+                          static_cast<float*>(dx), dw_gate, dw_up, dw_down, cs(stream));
+}
+
+}  // extern "C"
