@@ -1,0 +1,546 @@
+#!/usr/bin/env python
+"""Throughput of the STAPLE embedding-augmented SwiGLU FFN layer on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
+
+Default workload: one OLMo-2-1B-shaped layer decoding a batch of 64 tokens
+(d_model 2048, d_ff 8192, vocab 100352, bf16, the whole table E in HBM).  A
+step is one forward pass of the layer over one batch: the gate/up GEMM with
+the E-row add and SiLU gating fused in, then the down GEMM.  Four weight sets
+(403 MB, more than the 126 MB L2) and 64 token batches rotate from step to
+step, so no step finds its weights in L2.  The training layer (16384 tokens,
+host table with a 5% HBM cache, forward + full backward incl. the unique-row
+table gradient) is timed as well and reported under "train_layer", next to
+the same build's dense run (E path disabled).
+
+Multi-GPU (torchrun): every rank runs its own replica on its own batches (no
+collective on the data path); the time is the max over ranks.
+
+--impl reference times the CPU oracle (the plain fp64 definition) on a bounded
+sample of the same workload: each step is one token's forward restricted to a
+256-feature slice of d_ff, i.e. 1/32 of a token; tokens/s is scaled to match.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import synthetic as syn  # noqa: E402
+
+METRIC = "STAPLE FFN layer tokens/s (fwd+bwd and decode) at 1 B200; % of roofline"
+DEFAULT_WORKLOAD = "olmo2-1b-decode-layer"
+REF_SLICE = 256
+
+
+# --------------------------------------------------------------------------
+# Plumbing: ranks, peaks, clocks
+# --------------------------------------------------------------------------
+
+def dist_init():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+    return rank, world, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(v: float, world: int) -> float:
+    if world == 1:
+        return v
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained", d["bf16_tflops"]),
+                "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+            "source": "fallback"}
+
+
+class Clocks:
+    """nvidia-smi sampling of SM clocks and throttle reasons while it runs."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.Q}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            time.sleep(0.15)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self, t0: float, t1: float):
+        if self.proc is None or not self.path:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    rows.append((int(parts[1]), int(parts[2]), float(parts[3]), parts[4:]))
+                except ValueError:
+                    continue
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        # samples taken while the timed region ran: the ones drawing power
+        load = [r for r in rows if r[2] > 200.0] or rows
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({n for r in load for n, v in zip(names, r[3][1:]) if v == "Active"})
+        return {"sm_mhz": statistics.median(r[0] for r in load), "sm_max_mhz": max(r[1] for r in rows),
+                "power_w_max": max(r[2] for r in rows), "samples": len(load), "reasons": reasons}
+
+
+def bf16_randn(shape, std, seed):
+    """Seeded N(0, std) draws made on the GPU, rounded to bf16 (used for the
+    big tensors; the parity tests use the numpy generator of `synthetic`)."""
+    import torch
+    g = torch.Generator(device="cuda")
+    g.manual_seed(seed)
+    return (torch.randn(shape, generator=g, device="cuda", dtype=torch.float32) * std).to(torch.bfloat16)
+
+
+def kernel_table(trace, steps_seen):
+    out = {}
+    for name, ms in trace:
+        if ms < 0:
+            continue
+        d = out.setdefault(name, {"launches": 0, "total_ms": 0.0})
+        d["launches"] += 1
+        d["total_ms"] += ms
+    tot = sum(d["total_ms"] for d in out.values()) or 1.0
+    for d in out.values():
+        d["avg_us"] = round(1000.0 * d["total_ms"] / d["launches"], 3)
+        d["share"] = round(d["total_ms"] / tot, 4)
+        d["total_ms"] = round(d["total_ms"], 4)
+    return out
+
+
+# --------------------------------------------------------------------------
+# Decode layer (device table)
+# --------------------------------------------------------------------------
+
+def decode_setup(stp, w, local):
+    import torch
+    R, S = 4, 64
+    T, D, F, V = w.T, w.D, w.F, w.V
+    st = {"R": R, "S": S}
+    st["wg"] = [bf16_randn((F, D), w.w_std, syn.SEED_W + 3 * r) for r in range(R)]
+    st["wu"] = [bf16_randn((F, D), w.w_std, syn.SEED_W + 3 * r + 1) for r in range(R)]
+    st["wd"] = [bf16_randn((D, F), w.w_std, syn.SEED_W + 3 * r + 2) for r in range(R)]
+    st["table"] = bf16_randn((V, F), w.e_std, syn.SEED_E)
+    ids = np.stack([syn.zipf_ids(T, V, w.zipf_s, seed=syn.SEED_IDS + w.index + 7919 * s)
+                    for s in range(S)])
+    st["ids_host"] = torch.from_numpy(ids).pin_memory()
+    st["ids"] = st["ids_host"].cuda()
+    st["x"] = bf16_randn((S, T, D), w.x_std, syn.SEED_ACT)
+    st["x_host"] = st["x"].cpu().pin_memory()
+    st["z"] = torch.empty((T, F), dtype=torch.bfloat16, device="cuda")
+    st["y"] = torch.empty((T, D), dtype=torch.bfloat16, device="cuda")
+    st["y_host"] = torch.empty((S, T, D), dtype=torch.bfloat16).pin_memory()
+    st["emb"] = [stp.make_embed(stp.STAPLE_EMBED_TABLE, st["table"], F, st["ids"][s], V)
+                 for s in range(S)]
+    return st
+
+
+def decode_step(stp, ctx, w, st, s, stream):
+    r = s % st["R"]
+    b = s % st["S"]
+    stp.staple_ffn_fwd(ctx, stp.STAPLE_BF16, w.T, w.D, w.F, st["x"][b], st["emb"][b], st["wg"][r],
+                       st["wu"][r], st["wd"][r], st["z"], st["y"], stream=stream)
+
+
+def run_decode(stp, ctx, w, args, world, local):
+    import torch
+    st = decode_setup(stp, w, local)
+    stream = torch.cuda.Stream()
+    G = st["R"] * st["S"] // 4   # steps per captured graph (cycles weights 16x)
+    with torch.cuda.stream(stream):
+        for s in range(max(args.warmup, 3)):
+            decode_step(stp, ctx, w, st, s, stream)
+    torch.cuda.synchronize()
+    assert stp.staple_get_error(ctx, stream) == 0
+    # capture G steps once; replay to cover the K timed steps
+    stp.staple_trace_enable(ctx, True)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        for s in range(G):
+            decode_step(stp, ctx, w, st, s, stream)
+    reps = max(1, (args.steps + G - 1) // G)
+    K = reps * G
+    for _ in range(max(1, args.warmup // G)):
+        graph.replay()
+    torch.cuda.synchronize()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    with Clocks(local) as clk:
+        torch.cuda.synchronize()
+        t0 = time.time()
+        ev0.record(stream)
+        for _ in range(reps):
+            graph.replay()
+        ev1.record(stream)
+        torch.cuda.synchronize()
+        t1 = time.time()
+    ms = ev0.elapsed_time(ev1)
+    trace = stp.staple_trace_read(ctx)
+    stp.staple_trace_enable(ctx, False)
+    assert stp.staple_get_error(ctx, stream) == 0
+    ms_max = max_over_ranks(ms, world)
+    kern = kernel_table(trace, G)
+    res = {"K": K, "ms": ms_max, "ms_local": ms, "clocks": clk.summary(t0, t1), "kernels": kern,
+           "launches_per_step": sum(d["launches"] for d in kern.values()) / G}
+    del graph
+    # end to end through the public call with host buffers: H2D of x and ids
+    # from pinned memory, the layer, D2H of y, every step
+    Ke = min(K, 4096)
+    h2d = st["x"][0].numel() * 2 + st["ids"][0].numel() * 4
+    d2h = st["y"].numel() * 2
+    xd = torch.empty_like(st["x"][0])
+    idd = torch.empty_like(st["ids"][0])
+    embd = stp.make_embed(stp.STAPLE_EMBED_TABLE, st["table"], w.F, idd, w.V)
+
+    def e2e_step(s):
+        r, b = s % st["R"], s % st["S"]
+        xd.copy_(st["x_host"][b], non_blocking=True)
+        idd.copy_(st["ids_host"][b], non_blocking=True)
+        stp.staple_ffn_fwd(ctx, stp.STAPLE_BF16, w.T, w.D, w.F, xd, embd, st["wg"][r], st["wu"][r],
+                           st["wd"][r], st["z"], st["y"], stream=stream)
+        st["y_host"][b].copy_(st["y"], non_blocking=True)
+
+    with torch.cuda.stream(stream):
+        for s in range(8):
+            e2e_step(s)
+        torch.cuda.synchronize()
+        barrier(world)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for s in range(Ke):
+            e2e_step(s)
+        e1.record(stream)
+        torch.cuda.synchronize()
+    e_ms = max_over_ranks(e0.elapsed_time(e1), world)
+    res["e2e"] = {"K": Ke, "ms": e_ms, "h2d": h2d, "d2h": d2h}
+    # dominant kernel: algorithmic bytes of one gate/up launch
+    T, D, F = w.T, w.D, w.F
+    res["roofline_kernel"] = "k5_gateup"
+    res["alg_bytes"] = 2 * F * D * 2 + T * D * 2 + T * F * 2 + T * F * 2 + T * 4
+    res["alg_note"] = ("k5_gateup bytes per launch: W_gate + W_up (2*F*D*2) + x (T*D*2) + "
+                       "E rows (T*F*2) + z (T*F*2) + ids (T*4)")
+    return res
+
+
+# --------------------------------------------------------------------------
+# Training layer (host table + 5% cache)
+# --------------------------------------------------------------------------
+
+def run_train(stp, ctx, w, steps, warmup, world, local):
+    import torch
+    T, D, F, V = w.T, w.D, w.F, w.V
+    S = 4
+    wg = bf16_randn((F, D), w.w_std, syn.SEED_W)
+    wu = bf16_randn((F, D), w.w_std, syn.SEED_W + 1)
+    wd = bf16_randn((D, F), w.w_std, syn.SEED_W + 2)
+    table_host = bf16_randn((V, F), w.e_std, syn.SEED_E).cpu().pin_memory()
+    tab = stp.staple_table_register(ctx, table_host, V * F * 2, V, F, 1, stp.STAPLE_BF16,
+                                    stp.STAPLE_TABLE_HOST_PINNED)
+    freq = syn.calibration_freq(V)
+    cache = stp.staple_cache_build(ctx, tab, freq, w.cache_frac)
+    ids = torch.from_numpy(np.stack([syn.zipf_ids(T, V, w.zipf_s, seed=syn.SEED_IDS + w.index + 7919 * s)
+                                     for s in range(S)])).cuda()
+    x = [bf16_randn((T, D), w.x_std, syn.SEED_ACT + 2 * s) for s in range(S)]
+    dy = [bf16_randn((T, D), w.dy_std, syn.SEED_ACT + 2 * s + 1) for s in range(S)]
+    i32 = dict(dtype=torch.int32, device="cuda")
+    unique, inverse, sorted_pos, slot, miss = (torch.empty(T, **i32) for _ in range(5))
+    seg, U, mc = torch.empty(T + 1, **i32), torch.empty(1, **i32), torch.empty(1, **i32)
+    rows = torch.empty((T, F), dtype=torch.bfloat16, device="cuda")
+    z, g, h = (torch.empty((T, F), dtype=torch.bfloat16, device="cuda") for _ in range(3))
+    y = torch.empty((T, D), dtype=torch.bfloat16, device="cuda")
+    dgh = torch.empty((T, 2 * F), dtype=torch.bfloat16, device="cuda")
+    dE = torch.empty((T, F), dtype=torch.float32, device="cuda")
+    dx = torch.empty((T, D), dtype=torch.bfloat16, device="cuda")
+    dwg, dwu = (torch.empty((F, D), dtype=torch.float32, device="cuda") for _ in range(2))
+    dwd = torch.empty((D, F), dtype=torch.float32, device="cuda")
+    wsb = stp.staple_workspace_bytes(T, D, F)
+    ws = torch.empty(wsb, dtype=torch.uint8, device="cuda")
+    stream, side = torch.cuda.Stream(), torch.cuda.Stream()
+    emb_rows = stp.make_embed(stp.STAPLE_EMBED_ROWS, rows, F, inverse, T)
+    emb_none = stp.make_embed(stp.STAPLE_EMBED_NONE)
+
+    def step(s, staple=True):
+        b = s % S
+        if staple:
+            stp.staple_gather_rows(ctx, cache, tab, ids[b], T, unique, inverse, seg, sorted_pos, U,
+                                   slot, miss, mc, rows, stream=stream, side=side)
+        stp.staple_ffn_fwd(ctx, stp.STAPLE_BF16, T, D, F, x[b], emb_rows if staple else emb_none,
+                           wg, wu, wd, z, y, g, h, stream=stream)
+        stp.staple_embed_bwd(ctx, stp.STAPLE_BF16, T, D, F, dy[b], g, h, wd, sorted_pos, inverse,
+                             seg, U, dgh, dE if staple else None, ws, wsb, stream=stream)
+        stp.staple_ffn_bwd(ctx, stp.STAPLE_BF16, T, D, F, dy[b], x[b], z, dgh, wg, wu, dx, dwg, dwu,
+                           dwd, stream=stream)
+
+    out = {}
+    try:
+        for mode in ("staple", "dense"):
+            staple = mode == "staple"
+            with torch.cuda.stream(stream):
+                for s in range(max(warmup, 3)):
+                    step(s, staple)
+            torch.cuda.synchronize()
+            assert stp.staple_get_error(ctx, stream) == 0
+            if staple:
+                stp.staple_trace_enable(ctx, True)
+            barrier(world)
+            ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            with Clocks(local) as clk:
+                torch.cuda.synchronize()
+                t0 = time.time()
+                with torch.cuda.stream(stream):
+                    ev0.record(stream)
+                    for s in range(steps):
+                        step(s, staple)
+                    ev1.record(stream)
+                torch.cuda.synchronize()
+                t1 = time.time()
+            ms = max_over_ranks(ev0.elapsed_time(ev1), world)
+            assert stp.staple_get_error(ctx, stream) == 0
+            out[mode] = {"ms": ms, "clocks": clk.summary(t0, t1)}
+            if staple:
+                out[mode]["kernels"] = kernel_table(stp.staple_trace_read(ctx), steps)
+                stp.staple_trace_enable(ctx, False)
+                out["U"] = int(U.item())
+                out["misses"] = int(mc.item())
+    finally:
+        stp.staple_cache_free(cache)
+        stp.staple_table_unregister(tab)
+    return out
+
+
+def train_flops(w):
+    return 18 * w.T * w.D * w.F   # 3 forward + 6 backward GEMMs of 2*T*D*F
+
+
+# --------------------------------------------------------------------------
+# CPU oracle legs
+# --------------------------------------------------------------------------
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def oracle_decode_inputs(w):
+    inp = syn.make_layer_inputs(w, with_table=False)
+    rows = {}
+    for b in range(4):
+        ids = syn.zipf_ids(w.T, w.V, w.zipf_s, seed=syn.SEED_IDS + w.index + 7919 * b)
+        rows[b] = ids
+    E_rows = syn.bf16_normal((w.T, w.F), w.e_std, syn.SEED_E)[1].astype(np.float64)
+    return inp, E_rows
+
+
+def cpu_baseline_decode(w, seconds=12.0):
+    """The oracle's forward on whole 64-token batches for ~seconds of CPU time."""
+    import oracle
+    inp, E_rows = oracle_decode_inputs(w)
+    x, wg, wu, wd = (inp.f64(k) for k in ("x", "w_gate", "w_up", "w_down"))
+    ids = np.arange(w.T)  # rows of E_rows: each token's own (already gathered) table row
+    n = 0
+    t0 = time.time()
+    while time.time() - t0 < seconds or n == 0:
+        oracle.ffn_forward(x, ids, wg, wu, wd, E_rows)
+        n += 1
+    dt = time.time() - t0
+    return {"value": n * w.T / dt, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
+            "sample": f"{n} full decode batches of {w.T} tokens (fp64 numpy oracle), {dt:.1f} s"}
+
+
+def reference_arm(w, args):
+    """--impl reference: the oracle as the reference implementation.  Each step
+    is one token's forward on a REF_SLICE-feature slice of d_ff (REF_SLICE/F of
+    a token's work); tokens/s counts those fractions."""
+    import oracle
+    inp = syn.make_layer_inputs(w, T=1, with_table=False)
+    x, wg, wu, wd = (inp.f64(k) for k in ("x", "w_gate", "w_up", "w_down"))
+    E = syn.bf16_normal((1, w.F), w.e_std, syn.SEED_E)[1].astype(np.float64)
+    nsl = w.F // REF_SLICE
+
+    def step(s):
+        k = s % nsl
+        sl = slice(k * REF_SLICE, (k + 1) * REF_SLICE)
+        oracle.ffn_forward(x, [0], wg[sl], wu[sl], wd[:, sl], E[:, sl])
+
+    for s in range(args.warmup):
+        step(s)
+    t0 = time.time()
+    for s in range(args.steps):
+        step(s)
+    dt = time.time() - t0
+    tokens = args.steps * REF_SLICE / w.F
+    v = tokens / dt
+    return {"metric": METRIC, "value": v, "unit": "tokens/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000 * dt / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "impl": "reference",
+            "config": {"workload": w.name, "T": w.T, "d_model": w.D, "d_ff": w.F, "vocab": w.V},
+            "cpu_baseline": {"value": v, "unit": "tokens/s", "kind": "oracle", "cores": blas_threads(),
+                             "sample": f"per step: 1 token x {REF_SLICE} of {w.F} d_ff features "
+                                       f"(1/{nsl} token), fp64 numpy oracle"},
+            "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+# --------------------------------------------------------------------------
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=60000)
+    ap.add_argument("--warmup", type=int, default=256)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=[DEFAULT_WORKLOAD])
+    ap.add_argument("--train-steps", type=int, default=200)
+    ap.add_argument("--no-train", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    w = syn.WORKLOADS[args.workload]
+
+    rank, world, local = dist_init()
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(reference_arm(w, args)), flush=True)
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+        return
+
+    import torch
+
+    import token_indexed_sparse_staple_b200 as stp
+    torch.cuda.set_device(local)
+    ctx = stp.staple_context_create(local)
+    pk = peaks()
+    dec = run_decode(stp, ctx, w, args, world, local)
+    K = dec["K"]
+    value = world * w.T * K / (dec["ms"] / 1000.0)
+    kd = dec["kernels"].get(dec["roofline_kernel"], {})
+    ach = dec["alg_bytes"] / (kd.get("avg_us", float("nan")) * 1e-6) / 1e9
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K,
+        "warmup": args.warmup, "ms_per_step": dec["ms"] / K, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": w.name, "T": w.T, "d_model": w.D, "d_ff": w.F, "vocab": w.V,
+                   "table": "device (1.64 GB in HBM)", "weights": "random N(0,0.02) bf16",
+                   "l2": "inputs larger than L2: 4 rotating weight sets (403 MB) and 64 token batches",
+                   "graph": "steps replayed from one captured CUDA graph of 64 steps"},
+        "roofline": {"bound": "hbm", "kernel": dec["roofline_kernel"], "achieved": ach,
+                     "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": ach / pk["hbm_gbs"],
+                     "traffic": None, "peak_source": pk["source"] + " (copy bandwidth)",
+                     "alg_bytes_per_launch": dec["alg_bytes"], "note": dec["alg_note"]},
+        "e2e": {"value": world * w.T * dec["e2e"]["K"] / (dec["e2e"]["ms"] / 1000.0),
+                "unit": "tokens/s", "h2d_bytes_per_step": dec["e2e"]["h2d"],
+                "d2h_bytes_per_step": dec["e2e"]["d2h"], "steps": dec["e2e"]["K"],
+                "how": "per step: pinned H2D of x and ids, staple_ffn_fwd, D2H of y (Python loop)"},
+        "gpu_launches": int(round(dec["launches_per_step"] * K)),
+        "clocks": dec["clocks"],
+        "kernels": dec["kernels"],
+    }
+    if not args.no_train:
+        try:
+            wt = syn.WORKLOADS["olmo2-1b-train-layer"]
+            tr = run_train(stp, ctx, wt, args.train_steps, 5, world, local)
+            st_ms = tr["staple"]["ms"] / args.train_steps
+            de_ms = tr["dense"]["ms"] / args.train_steps
+            kern = tr["staple"]["kernels"]
+            top = max(kern.items(), key=lambda kv: kv[1]["total_ms"])
+            gemm_flops = {"k5_gateup": 4, "k6_down": 2, "k7_dz": 2, "k9_dx": 4, "k10_dw_gate_up": 4,
+                          "k10_dw_down": 2}
+            tf = None
+            if top[0] in gemm_flops:
+                tf = gemm_flops[top[0]] * wt.T * wt.D * wt.F / (top[1]["avg_us"] * 1e-6) / 1e12
+            line["train_layer"] = {
+                "workload": wt.name, "tokens_per_s": world * wt.T / (st_ms / 1000.0),
+                "ms_per_step": st_ms, "dense_ms_per_step": de_ms,
+                "e_path_overhead": (st_ms - de_ms) / de_ms, "steps": args.train_steps,
+                "U": tr["U"], "misses": tr["misses"],
+                "tflops": train_flops(wt) / (st_ms / 1000.0) / 1e12,
+                "roofline": {"bound": "tensor", "kernel": top[0], "achieved": tf,
+                             "peak": pk["bf16_tflops_sustained"], "unit": "TFLOP/s",
+                             "frac": None if tf is None else tf / pk["bf16_tflops_sustained"],
+                             "peak_source": pk["source"] + " (cuBLAS bf16, sustained)"},
+                "clocks": tr["staple"]["clocks"], "kernels": kern,
+            }
+        except Exception as ex:  # the decode line must still print
+            line["train_layer"] = {"error": repr(ex)}
+    if world == 1 and rank == 0 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline_decode(w)
+    stp.staple_context_destroy(ctx)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        barrier(world)
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

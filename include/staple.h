@@ -88,6 +88,21 @@ staple_status staple_context_destroy(staple_context* ctx);
  * it.  The only call that waits for the device. */
 staple_status staple_get_error(staple_context* ctx, staple_stream stream, int32_t* device_error);
 
+/* Per-kernel timing.  With tracing enabled, every kernel the library launches
+ * for this context is bracketed by two CUDA events on its launch stream (a
+ * record costs well under a microsecond of device time).  staple_trace_read
+ * waits for the recorded events, writes up to `capacity` records in launch
+ * order into out[], stores their number in *count, and forgets them (records
+ * beyond capacity are dropped).  Enabling allocates 2 * 65536 events once. */
+typedef struct staple_trace_record {
+  char kernel[40]; /* kernel name, e.g. "k5_gateup" */
+  float ms;        /* event-to-event device time of the launch */
+} staple_trace_record;
+
+staple_status staple_trace_enable(staple_context* ctx, int enable);
+staple_status staple_trace_read(staple_context* ctx, staple_trace_record* out, int32_t capacity,
+                                int32_t* count);
+
 /* ------------------------------------------------------------------ tables */
 
 #define STAPLE_TABLE_DEVICE 1u        /* `base` is device memory (the whole table in HBM) */

@@ -152,3 +152,20 @@ def test_bf16_rejects_unsupported_shapes(stp, ctx):
     with pytest.raises(stp.StapleError) as ex:
         stp.staple_ffn_fwd(ctx, stp.STAPLE_BF16, 4, 96, 64, t, e, t, t, t, t, t)
     assert ex.value.status == stp.STAPLE_EINVAL
+
+
+def test_trace_records_every_kernel(stp, ctx):
+    w = _bf16_workload(300, 128, 320, 1000)
+    inp = syn.make_layer_inputs(w)
+    stp.staple_trace_enable(ctx, True)
+    try:
+        run_layer(stp, ctx, inp, w.D, w.F, w.V, embed="table")
+        rec = stp.staple_trace_read(ctx)
+    finally:
+        stp.staple_trace_enable(ctx, False)
+    names = [n for n, _ in rec]
+    for k in ("k1_dedup", "k5_gateup", "k6_down", "k7_dz", "k8_seg_reduce", "k9_dx",
+              "k10_dw_gate_up", "k10_dw_down"):
+        assert k in names, (k, names)
+    assert all(ms > 0 for _, ms in rec)
+    assert stp.staple_trace_read(ctx) == []

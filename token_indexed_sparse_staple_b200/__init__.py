@@ -95,6 +95,18 @@ def staple_get_error(ctx: int, stream=None) -> int:
     return e.value
 
 
+def staple_trace_enable(ctx: int, enable: bool = True) -> None:
+    _ok(lib().staple_trace_enable(ctx, int(bool(enable))), "staple_trace_enable")
+
+
+def staple_trace_read(ctx: int, capacity: int = 1 << 16) -> list[tuple[str, float]]:
+    """[(kernel name, device ms)] for the launches since the last read."""
+    recs = (_lib.staple_trace_record * capacity)()
+    n = C.c_int32()
+    _ok(lib().staple_trace_read(ctx, recs, capacity, C.byref(n)), "staple_trace_read")
+    return [(recs[i].kernel.decode(), float(recs[i].ms)) for i in range(n.value)]
+
+
 # ------------------------------------------------------------------- tables
 
 def staple_table_register(ctx: int, base, nbytes: int, V: int, F: int, groups: int, dtype: int,

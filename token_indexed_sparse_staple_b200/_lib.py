@@ -19,6 +19,10 @@ sz = C.c_size_t
 P = C.POINTER
 
 
+class staple_trace_record(C.Structure):
+    _fields_ = [("kernel", C.c_char * 40), ("ms", C.c_float)]
+
+
 class staple_embed(C.Structure):
     _fields_ = [("mode", i32), ("reserved", i32), ("base", vp), ("row_pitch", i64),
                 ("index", vp), ("n_rows", i64)]
@@ -31,6 +35,8 @@ SIGNATURES = {
     "staple_context_create": (c_status, [C.c_int, P(vp)]),
     "staple_context_destroy": (c_status, [vp]),
     "staple_get_error": (c_status, [vp, vp, P(i32)]),
+    "staple_trace_enable": (c_status, [vp, C.c_int]),
+    "staple_trace_read": (c_status, [vp, vp, i32, P(i32)]),
     "staple_table_register": (c_status, [vp, vp, sz, i64, i32, i32, C.c_int, u32, P(vp)]),
     "staple_table_unregister": (c_status, [vp]),
     "staple_cache_build": (c_status, [vp, vp, vp, C.c_double, vp, P(vp)]),

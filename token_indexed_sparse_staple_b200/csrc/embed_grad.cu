@@ -139,13 +139,17 @@ staple_status launch_seg_reduce(bool bf16, const void* dh, int64_t ld, const int
   const int chunks = (T + kSegChunk - 1) / kSegChunk;
   const dim3 grid(chunks, (F + kSegSlice - 1) / kSegSlice);
   if (bf16)
-    seg_reduce_kernel<true><<<grid, kSegThreads, 0, st>>>(dh, ld, sorted_pos, inverse, seg_off, T,
-                                                          F, dE, part);
+    STP_LAUNCH("k8_seg_reduce", st,
+               seg_reduce_kernel<true><<<grid, kSegThreads, 0, st>>>(dh, ld, sorted_pos, inverse,
+                                                                     seg_off, T, F, dE, part));
   else
-    seg_reduce_kernel<false><<<grid, kSegThreads, 0, st>>>(dh, ld, sorted_pos, inverse, seg_off,
-                                                           T, F, dE, part);
+    STP_LAUNCH("k8_seg_reduce", st,
+               seg_reduce_kernel<false><<<grid, kSegThreads, 0, st>>>(dh, ld, sorted_pos, inverse,
+                                                                      seg_off, T, F, dE, part));
   if (chunks > 1)
-    seg_fixup_kernel<<<grid, kSegThreads, 0, st>>>(sorted_pos, inverse, seg_off, T, F, dE, part);
+    STP_LAUNCH("k8_seg_fixup", st,
+               seg_fixup_kernel<<<grid, kSegThreads, 0, st>>>(sorted_pos, inverse, seg_off, T, F,
+                                                              dE, part));
   return cudaGetLastError() == cudaSuccess ? STAPLE_OK : STAPLE_ECUDA;
 }
 

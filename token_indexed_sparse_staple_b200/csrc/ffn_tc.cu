@@ -10,6 +10,7 @@
 #include <cudaTypedefs.h>
 
 #include <algorithm>
+#include <atomic>
 #include <mutex>
 
 #include "gemm_tc.cuh"
@@ -59,22 +60,25 @@ bool mnmajor(CUtensorMap* m, const void* base, int k, int mn, int64_t ld) {
 }
 
 template <bool A_MN, bool B_MN, int BSRC, int EPI>
-staple_status launch(const DeviceInfo& di, const CUtensorMap& a, const CUtensorMap& b0,
-                     const CUtensorMap& b1, tc::Params p, cudaStream_t st) {
+staple_status launch(const char* name, const DeviceInfo& di, const CUtensorMap& a,
+                     const CUtensorMap& b0, const CUtensorMap& b1, tc::Params p, cudaStream_t st) {
   p.k_blocks = (p.K + tc::BK - 1) / tc::BK;
   const int ntiles = p.tiles_m * p.tiles_n;
   if (ntiles == 0) return STAPLE_OK;
   if (p.group_m <= 0) p.group_m = 16;
   auto kern = tc::gemm_kernel<A_MN, B_MN, BSRC, EPI>;
-  static bool attr_set = false;  // per instantiation
-  if (!attr_set) {
+  // the shared-memory opt-in is set once per device and instantiation, so
+  // that no runtime attribute call happens while a stream is being captured
+  static std::atomic<uint64_t> attr_done{0};
+  const uint64_t bit = uint64_t(1) << (di.device & 63);
+  if (!(attr_done.load() & bit)) {
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              tc::kSmemBytes) != cudaSuccess)
       return STAPLE_ECUDA;
-    attr_set = true;
+    attr_done.fetch_or(bit);
   }
   const int grid = std::min(ntiles, di.num_sms);
-  kern<<<grid, tc::kThreads, tc::kSmemBytes, st>>>(a, b0, b1, p);
+  STP_LAUNCH(name, st, kern<<<grid, tc::kThreads, tc::kSmemBytes, st>>>(a, b0, b1, p));
   return cudaGetLastError() == cudaSuccess ? STAPLE_OK : STAPLE_ECUDA;
 }
 
@@ -110,7 +114,7 @@ staple_status tc_ffn_fwd(const DeviceInfo& di, int T, int D, int F, const void* 
       p.e_rows = e->n_rows;
     }
     p.err = err;
-    staple_status s = launch<false, false, tc::B_NHALF, tc::EPI_GATEUP>(di, mx, mg, mu, p, st);
+    staple_status s = launch<false, false, tc::B_NHALF, tc::EPI_GATEUP>("k5_gateup", di, mx, mg, mu, p, st);
     if (s != STAPLE_OK) return s;
   }
   tc::Params q{};
@@ -123,7 +127,7 @@ staple_status tc_ffn_fwd(const DeviceInfo& di, int T, int D, int F, const void* 
   q.ldo = D;
   q.m_split = T;
   q.err = err;
-  return launch<false, false, tc::B_ONE, tc::EPI_BF16>(di, mz, md, md, q, st);
+  return launch<false, false, tc::B_ONE, tc::EPI_BF16>("k6_down", di, mz, md, md, q, st);
 }
 
 staple_status tc_dz(const DeviceInfo& di, int T, int D, int F, const void* dy, const void* g_save,
@@ -143,7 +147,7 @@ staple_status tc_dz(const DeviceInfo& di, int T, int D, int F, const void* dy, c
   p.h_in = static_cast<const uint16_t*>(h_save);
   p.dgh = static_cast<uint16_t*>(dgh);
   p.err = err;
-  return launch<false, true, tc::B_ONE, tc::EPI_DZ>(di, mdy, mwd, mwd, p, st);
+  return launch<false, true, tc::B_ONE, tc::EPI_DZ>("k7_dz", di, mdy, mwd, mwd, p, st);
 }
 
 staple_status tc_ffn_bwd(const DeviceInfo& di, int T, int D, int F, const void* dy,
@@ -175,7 +179,7 @@ staple_status tc_ffn_bwd(const DeviceInfo& di, int T, int D, int F, const void* 
     p.ldo = D;
     p.m_split = T;
     p.err = err;
-    if ((s = launch<false, true, tc::B_KSPLIT, tc::EPI_BF16>(di, ma, mb0, mb1, p, st)) !=
+    if ((s = launch<false, true, tc::B_KSPLIT, tc::EPI_BF16>("k9_dx", di, ma, mb0, mb1, p, st)) !=
         STAPLE_OK)
       return s;
   }
@@ -197,7 +201,7 @@ staple_status tc_ffn_bwd(const DeviceInfo& di, int T, int D, int F, const void* 
     p.ldo = D;
     p.m_split = both ? F : M;
     p.err = err;
-    if ((s = launch<true, true, tc::B_ONE, tc::EPI_F32>(di, ma, mb, mb, p, st)) != STAPLE_OK)
+    if ((s = launch<true, true, tc::B_ONE, tc::EPI_F32>("k10_dw_gate_up", di, ma, mb, mb, p, st)) != STAPLE_OK)
       return s;
   }
   if (dwd) {
@@ -214,7 +218,7 @@ staple_status tc_ffn_bwd(const DeviceInfo& di, int T, int D, int F, const void* 
     p.ldo = F;
     p.m_split = D;
     p.err = err;
-    if ((s = launch<true, true, tc::B_ONE, tc::EPI_F32>(di, ma, mb, mb, p, st)) != STAPLE_OK)
+    if ((s = launch<true, true, tc::B_ONE, tc::EPI_F32>("k10_dw_down", di, ma, mb, mb, p, st)) != STAPLE_OK)
       return s;
   }
   return STAPLE_OK;

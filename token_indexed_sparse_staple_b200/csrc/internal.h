@@ -17,6 +17,27 @@ struct DeviceInfo {
   int num_sms;
 };
 
+// trace.cu: optional per-kernel CUDA-event timing of a context
+constexpr int kTraceCapacity = 1 << 16;
+struct Tracer;
+Tracer* tracer_create(int device);
+void tracer_destroy(Tracer* t);
+bool tracer_enable(Tracer* t, bool on);
+int tracer_read(Tracer* t, staple_trace_record* out, int cap, int* dropped);
+int trace_begin(const char* name, cudaStream_t st);   // -1 when tracing is off
+void trace_end(int slot, cudaStream_t st);
+struct TraceScope {                                   // makes a tracer current for one API call
+  explicit TraceScope(Tracer* t);
+  ~TraceScope();
+  Tracer* prev;
+};
+#define STP_LAUNCH(name, st, ...)                     \
+  do {                                                \
+    const int _slot = ::stp::trace_begin(name, st);   \
+    __VA_ARGS__;                                      \
+    ::stp::trace_end(_slot, st);                      \
+  } while (0)
+
 // retrieval.cu
 staple_status launch_dedup(const int32_t* ids, int T, int64_t V, int32_t* unique,
                            int32_t* inverse, int32_t* seg_off, int32_t* sorted_pos,

@@ -7,6 +7,8 @@
 // probe the GPU cache; on a miss read the row from CUDA-registered host
 // memory with no CPU gather); AI Radio episode, paper summary (only the U
 // active rows are materialised on the GPU).
+#include <atomic>
+
 #include "common.cuh"
 #include "internal.h"
 
@@ -171,10 +173,21 @@ static cudaError_t launch_dedup_t(const int32_t* ids, int T, int64_t V, int key_
                                   int32_t* err, cudaStream_t st) {
   const size_t smem = (kDedupWarps * kRadix + 64) * sizeof(int32_t) + size_t(T) * sizeof(W);
   auto k = dedup_kernel<W, IPL>;
-  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
-  if (e != cudaSuccess) return e;
-  k<<<1, kDedupThreads, smem, st>>>(ids, T, V, key_bits, pos_bits, unique, inverse, seg_off,
-                                     sorted_pos, U_dev, err);
+  // opt in to the largest shared-memory size once per device and instantiation
+  static std::atomic<uint64_t> attr_done{0};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  const uint64_t bit = uint64_t(1) << (dev & 63);
+  if (!(attr_done.load() & bit)) {
+    const int max_smem = (kDedupWarps * kRadix + 64) * int(sizeof(int32_t)) + kMaxDedupT * int(sizeof(W));
+    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         max_smem < 227 * 1024 ? max_smem : 227 * 1024);
+    if (e != cudaSuccess) return e;
+    attr_done.fetch_or(bit);
+  }
+  STP_LAUNCH("k1_dedup", st,
+             k<<<1, kDedupThreads, smem, st>>>(ids, T, V, key_bits, pos_bits, unique, inverse,
+                                                seg_off, sorted_pos, U_dev, err));
   return cudaGetLastError();
 }
 
@@ -306,16 +319,18 @@ __global__ void __launch_bounds__(256)
 staple_status launch_probe(const int32_t* unique, const int32_t* U_dev, const int32_t* hkeys,
                            const int32_t* hvals, uint32_t hmask, int32_t* slot,
                            int32_t* miss_list, int32_t* miss_count, cudaStream_t st) {
-  probe_kernel<<<1, 1024, 0, st>>>(unique, U_dev, hkeys, hvals, hmask, slot, miss_list,
-                                   miss_count);
+  STP_LAUNCH("k2_probe", st,
+             probe_kernel<<<1, 1024, 0, st>>>(unique, U_dev, hkeys, hvals, hmask, slot, miss_list,
+                                              miss_count));
   return cudaGetLastError() == cudaSuccess ? STAPLE_OK : STAPLE_ECUDA;
 }
 
 staple_status launch_gather_hits(const void* cache_rows, int64_t row_bytes, const int32_t* U_dev,
                                  const int32_t* slot, void* rows, int num_sms, cudaStream_t st) {
-  gather_kernel<G_HITS><<<num_sms * 2, 256, 0, st>>>(
-      static_cast<const uint8_t*>(cache_rows), row_bytes, nullptr, U_dev, slot, nullptr,
-      static_cast<uint8_t*>(rows), row_bytes);
+  STP_LAUNCH("k3_gather_hits", st,
+             gather_kernel<G_HITS><<<num_sms * 2, 256, 0, st>>>(
+                 static_cast<const uint8_t*>(cache_rows), row_bytes, nullptr, U_dev, slot,
+                 nullptr, static_cast<uint8_t*>(rows), row_bytes));
   return cudaGetLastError() == cudaSuccess ? STAPLE_OK : STAPLE_ECUDA;
 }
 
@@ -323,9 +338,10 @@ staple_status launch_gather_misses(const void* table_dev, int64_t table_pitch_by
                                    int64_t row_bytes, const int32_t* unique,
                                    const int32_t* miss_list, const int32_t* miss_count,
                                    void* rows, int num_sms, cudaStream_t st) {
-  gather_kernel<G_MISSES><<<num_sms, 256, 0, st>>>(
-      static_cast<const uint8_t*>(table_dev), table_pitch_bytes, unique, miss_count, nullptr,
-      miss_list, static_cast<uint8_t*>(rows), row_bytes);
+  STP_LAUNCH("k4_gather_misses", st,
+             gather_kernel<G_MISSES><<<num_sms, 256, 0, st>>>(
+                 static_cast<const uint8_t*>(table_dev), table_pitch_bytes, unique, miss_count,
+                 nullptr, miss_list, static_cast<uint8_t*>(rows), row_bytes));
   return cudaGetLastError() == cudaSuccess ? STAPLE_OK : STAPLE_ECUDA;
 }
 

@@ -156,7 +156,8 @@ template <bool A_MN, bool B_MN, int EPI, bool DUAL>
 staple_status run(const SParams& p, cudaStream_t st) {
   if (p.M == 0 || p.N == 0) return STAPLE_OK;
   const dim3 grid((p.N + ST - 1) / ST, (p.M + ST - 1) / ST);
-  sgemm_kernel<A_MN, B_MN, EPI, DUAL><<<grid, 256, 0, st>>>(p);
+  STP_LAUNCH(EPI == S_GATEUP ? "k11_f32_gateup" : (EPI == S_DZ ? "k11_f32_dz" : "k11_f32_gemm"),
+             st, sgemm_kernel<A_MN, B_MN, EPI, DUAL><<<grid, 256, 0, st>>>(p));
   return cudaGetLastError() == cudaSuccess ? STAPLE_OK : STAPLE_ECUDA;
 }
 

@@ -18,6 +18,7 @@ struct staple_context {
   int32_t* d_err;          // device error word
   cudaEvent_t ev_main;     // main -> side ordering
   cudaEvent_t ev_side;     // side -> main ordering
+  stp::Tracer* tracer;     // optional per-kernel timing
 };
 
 struct staple_table {
@@ -133,7 +134,22 @@ staple_status staple_context_create(int device, staple_context** out) {
     delete c;
     return STAPLE_ECUDA;
   }
+  c->tracer = stp::tracer_create(device);
   *out = c;
+  return STAPLE_OK;
+}
+
+staple_status staple_trace_enable(staple_context* ctx, int enable) {
+  if (!ctx) return STAPLE_EINVAL;
+  STP_TRY(set_device(ctx));
+  return stp::tracer_enable(ctx->tracer, enable != 0) ? STAPLE_OK : STAPLE_ECUDA;
+}
+
+staple_status staple_trace_read(staple_context* ctx, staple_trace_record* out, int32_t capacity,
+                                int32_t* count) {
+  if (!ctx || !count || capacity < 0 || (capacity > 0 && !out)) return STAPLE_EINVAL;
+  STP_TRY(set_device(ctx));
+  *count = stp::tracer_read(ctx->tracer, out, capacity, nullptr);
   return STAPLE_OK;
 }
 
@@ -142,6 +158,7 @@ staple_status staple_context_destroy(staple_context* ctx) {
   cudaSetDevice(ctx->di.device);
   cudaEventDestroy(ctx->ev_main);
   cudaEventDestroy(ctx->ev_side);
+  stp::tracer_destroy(ctx->tracer);
   cudaFree(ctx->d_err);
   delete ctx;
   return STAPLE_OK;
@@ -223,6 +240,7 @@ staple_status staple_cache_build(staple_context* ctx, const staple_table* table,
   if (!ctx || !table || !freq || !out || !(frac >= 0.0 && frac <= 1.0)) return STAPLE_EINVAL;
   *out = nullptr;
   STP_TRY(set_device(ctx));
+  stp::TraceScope trace_scope(ctx->tracer);
   const int64_t V = table->V;
   if (V > INT32_MAX) return STAPLE_EUNSUPPORTED;
   int64_t K = frac > 0 ? int64_t(std::ceil(frac * double(V) - 1e-9)) : 0;
@@ -318,6 +336,7 @@ staple_status staple_dedup(staple_context* ctx, const int32_t* ids, int32_t T, i
   if (T > 0 && (!ids || !unique || !inverse || !sorted_pos)) return STAPLE_EINVAL;
   if (T > stp::kMaxDedupT) return STAPLE_EUNSUPPORTED;
   STP_TRY(set_device(ctx));
+  stp::TraceScope trace_scope(ctx->tracer);
   return stp::launch_dedup(ids, T, V, unique, inverse, seg_off, sorted_pos, U_dev, ctx->d_err,
                            cs(stream));
 }
@@ -333,6 +352,7 @@ staple_status staple_gather_unique_rows(staple_context* ctx, const staple_cache*
   const int64_t row_bytes = int64_t(table->groups) * table->F * int64_t(esize(table->dtype));
   if (cache && cache->row_bytes != row_bytes) return STAPLE_EINVAL;
   STP_TRY(set_device(ctx));
+  stp::TraceScope trace_scope(ctx->tracer);
   cudaStream_t st = cs(stream);
   cudaStream_t sd = cs(side);
   STP_TRY(stp::launch_probe(unique, U_dev, cache && cache->K > 0 ? cache->hkeys : nullptr,
@@ -385,6 +405,7 @@ staple_status staple_ffn_fwd(staple_context* ctx, staple_dtype dtype, int32_t T,
   if ((g_save && !ptrs_ok(dtype, {g_save})) || (h_save && !ptrs_ok(dtype, {h_save})))
     return STAPLE_EINVAL;
   STP_TRY(set_device(ctx));
+  stp::TraceScope trace_scope(ctx->tracer);
   if (dtype == STAPLE_BF16)
     return stp::tc_ffn_fwd(ctx->di, T, D, F, x, embed, w_gate, w_up, w_down, z, y, g_save, h_save,
                            ctx->d_err, cs(stream));
@@ -414,6 +435,7 @@ staple_status staple_embed_bwd(staple_context* ctx, staple_dtype dtype, int32_t 
       return STAPLE_EINVAL;
   }
   STP_TRY(set_device(ctx));
+  stp::TraceScope trace_scope(ctx->tracer);
   cudaStream_t st = cs(stream);
   if (dtype == STAPLE_BF16)
     STP_TRY(stp::tc_dz(ctx->di, T, D, F, dy, g_save, h_save, w_down, dgh, ctx->d_err, st));
@@ -442,6 +464,7 @@ staple_status staple_ffn_bwd(staple_context* ctx, staple_dtype dtype, int32_t T,
   for (const float* p : {dw_gate, dw_up, dw_down})
     if (p && !aligned16(p)) return STAPLE_EINVAL;
   STP_TRY(set_device(ctx));
+  stp::TraceScope trace_scope(ctx->tracer);
   if (dtype == STAPLE_BF16)
     return stp::tc_ffn_bwd(ctx->di, T, D, F, dy, x, z, dgh, w_gate, w_up, dx, dw_gate, dw_up,
                            dw_down, ctx->d_err, cs(stream));
