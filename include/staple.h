@@ -262,6 +262,33 @@ staple_status staple_ffn_bwd(staple_context* ctx, staple_dtype dtype, int32_t T,
                              float* dw_gate, float* dw_up, float* dw_down, void* workspace,
                              size_t workspace_bytes, staple_stream stream);
 
+/* ------------------------------------------- allocation-free table gradient */
+
+/* dE from dh without any device allocation, by the caller or the library.
+ * The paper has no counterpart: this is the table-gradient reduction of
+ * staple_embed_bwd (same kernels, same result) for callers that cannot
+ * allocate device memory -- a process whose device memory is all owned by
+ * another allocator, code that must not call cudaMalloc because it
+ * synchronizes the device, or a plug-in host that only passes its input and
+ * output buffers.  Its partial-sum scratch is a 16 MiB array built into the
+ * library's device image, which every GPU that loads the library holds until
+ * the process exits.
+ *   dh          device, T rows of F values (dtype) with row pitch ld elements
+ *               (e.g. the dh half of staple_embed_bwd's dgh: base + F, ld = 2F)
+ *   sorted_pos, inverse, seg_off   from staple_dedup for the same ids
+ *   dE          out, fp32 [>= U][F]; rows >= U untouched
+ * Runs on the current device, on `stream`.  The first call on a device looks
+ * up the array's device address (cudaGetSymbolAddress); make that first call
+ * before any stream capture.  Every call shares the one array, so calls that
+ * overlap on the GPU race; nothing in it needs to start at zero.
+ * Returns STAPLE_EINVAL for bad arguments and for a size beyond the array:
+ * 2 * ceil(T / 64) * F * 4 bytes must not exceed 16 MiB (T <= 16384 at
+ * F = 8192).  F must be a multiple of 8. */
+staple_status staple_embed_grad_static(staple_dtype dtype, int32_t T, int32_t F, const void* dh,
+                                       int64_t ld, const int32_t* sorted_pos,
+                                       const int32_t* inverse, const int32_t* seg_off, float* dE,
+                                       staple_stream stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -206,3 +206,11 @@ def staple_ffn_bwd(ctx, dtype, T, D, F, dy, x, z, dgh, w_gate, w_up, dx, dw_gate
     _ok(lib().staple_ffn_bwd(ctx, dtype, T, D, F, _p(dy), _p(x), _p(z), _p(dgh), _p(w_gate),
                              _p(w_up), _p(dx), _p(dw_gate), _p(dw_up), _p(dw_down),
                              _p(workspace), workspace_bytes, _stream(stream)), "staple_ffn_bwd")
+
+
+def staple_embed_grad_static(dtype, T, F, dh, ld, sorted_pos, inverse, seg_off, dE, stream=None):
+    """Table gradient from dh with the library's built-in scratch: no device
+    allocation by the caller or the library (see include/staple.h)."""
+    _ok(lib().staple_embed_grad_static(dtype, T, F, _p(dh), ld, _p(sorted_pos), _p(inverse),
+                                       _p(seg_off), _p(dE), _stream(stream)),
+        "staple_embed_grad_static")
