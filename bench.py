@@ -196,6 +196,8 @@ def decode_setup(stp, w, local):
     st["y_host"] = torch.empty((S, T, D), dtype=torch.bfloat16).pin_memory()
     st["emb"] = [stp.make_embed(stp.STAPLE_EMBED_TABLE, st["table"], F, st["ids"][s], V)
                  for s in range(S)]
+    st["wsb"] = stp.staple_workspace_bytes(T, D, F)
+    st["ws"] = torch.zeros(st["wsb"], dtype=torch.uint8, device="cuda")
     return st
 
 
@@ -203,7 +205,8 @@ def decode_step(stp, ctx, w, st, s, stream):
     r = s % st["R"]
     b = s % st["S"]
     stp.staple_ffn_fwd(ctx, stp.STAPLE_BF16, w.T, w.D, w.F, st["x"][b], st["emb"][b], st["wg"][r],
-                       st["wu"][r], st["wd"][r], st["z"], st["y"], stream=stream)
+                       st["wu"][r], st["wd"][r], st["z"], st["y"], None, None, st["ws"], st["wsb"],
+                       stream=stream)
 
 
 def run_decode(stp, ctx, w, args, world, local):
@@ -224,18 +227,20 @@ def run_decode(stp, ctx, w, args, world, local):
             decode_step(stp, ctx, w, st, s, stream)
     reps = max(1, (args.steps + G - 1) // G)
     K = reps * G
-    for _ in range(max(1, args.warmup // G)):
-        graph.replay()
+    with torch.cuda.stream(stream):       # replay() launches on the current stream
+        for _ in range(max(1, args.warmup // G)):
+            graph.replay()
     torch.cuda.synchronize()
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier(world)
     with Clocks(local) as clk:
         torch.cuda.synchronize()
         t0 = time.time()
-        ev0.record(stream)
-        for _ in range(reps):
-            graph.replay()
-        ev1.record(stream)
+        with torch.cuda.stream(stream):
+            ev0.record(stream)
+            for _ in range(reps):
+                graph.replay()
+            ev1.record(stream)
         torch.cuda.synchronize()
         t1 = time.time()
     ms = ev0.elapsed_time(ev1)
@@ -261,7 +266,8 @@ def run_decode(stp, ctx, w, args, world, local):
         xd.copy_(st["x_host"][b], non_blocking=True)
         idd.copy_(st["ids_host"][b], non_blocking=True)
         stp.staple_ffn_fwd(ctx, stp.STAPLE_BF16, w.T, w.D, w.F, xd, embd, st["wg"][r], st["wu"][r],
-                           st["wd"][r], st["z"], st["y"], stream=stream)
+                           st["wd"][r], st["z"], st["y"], None, None, st["ws"], st["wsb"],
+                           stream=stream)
         st["y_host"][b].copy_(st["y"], non_blocking=True)
 
     with torch.cuda.stream(stream):
@@ -329,7 +335,7 @@ def run_train(stp, ctx, w, steps, warmup, world, local):
             stp.staple_gather_rows(ctx, cache, tab, ids[b], T, unique, inverse, seg, sorted_pos, U,
                                    slot, miss, mc, rows, stream=stream, side=side)
         stp.staple_ffn_fwd(ctx, stp.STAPLE_BF16, T, D, F, x[b], emb_rows if staple else emb_none,
-                           wg, wu, wd, z, y, g, h, stream=stream)
+                           wg, wu, wd, z, y, g, h, ws, wsb, stream=stream)
         stp.staple_embed_bwd(ctx, stp.STAPLE_BF16, T, D, F, dy[b], g, h, wd, sorted_pos, inverse,
                              seg, U, dgh, dE if staple else None, ws, wsb, stream=stream)
         stp.staple_ffn_bwd(ctx, stp.STAPLE_BF16, T, D, F, dy[b], x[b], z, dgh, wg, wu, dx, dwg, dwu,

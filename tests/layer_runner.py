@@ -52,9 +52,11 @@ def run_layer(stp, ctx, inp, D, F, V, *, embed="table", training=True, rows_tabl
         e = stp.make_embed(stp.STAPLE_EMBED_ROWS, rows, F, inverse, max(T, 1))
         keep.append(rows)
         out["miss_count"] = int(mc.item())
+    wsb = stp.staple_workspace_bytes(T, D, F)
+    ws = torch.empty(max(wsb, 256), dtype=torch.uint8, device="cuda")
     try:
         stp.staple_ffn_fwd(ctx, sdt, T, D, F, x, e, wg, wu, wd, z, y,
-                           g if training else None, h if training else None)
+                           g if training else None, h if training else None, ws, wsb)
         err = stp.staple_get_error(ctx)
         assert err == 0, stp.staple_status_string(err)
         out.update(z=f64(z), y=f64(y))
@@ -67,8 +69,6 @@ def run_layer(stp, ctx, inp, D, F, V, *, embed="table", training=True, rows_tabl
             dy = dev(inp.dy, dt)
             dgh = empty((T, 2 * F), dt)
             dE = torch.zeros((max(T, 1), F), dtype=torch.float32, device="cuda")
-            wsb = stp.staple_workspace_bytes(T, D, F)
-            ws = torch.empty(max(wsb, 256), dtype=torch.uint8, device="cuda")
             stp.staple_embed_bwd(ctx, sdt, T, D, F, dy, g, h, wd, sorted_pos, inverse, seg, U, dgh,
                                  dE, ws, wsb)
             dx = empty((T, D), dt)

@@ -169,3 +169,45 @@ def test_trace_records_every_kernel(stp, ctx):
         assert k in names, (k, names)
     assert all(ms > 0 for _, ms in rec)
     assert stp.staple_trace_read(ctx) == []
+
+
+# ----------------------------------------------------- decode-shaped path
+
+@pytest.mark.parametrize("T", [1, 17, 64, 200, 256])
+def test_bf16_decode_sizes_match_oracle(stp, ctx, T):
+    """T <= 256 runs the weight-streaming kernels (weights on the MMA's M side,
+    split-K down projection with a last-block reduction)."""
+    w = _bf16_workload(T, 256, 576, 4000)
+    inp = syn.make_layer_inputs(w, with_dy=False)
+    got = run_layer(stp, ctx, inp, w.D, w.F, w.V, embed="table", training=False)
+    ref = oracle_layer(inp, training=False)
+    compare(got, ref, TOL["bf16"], FWD)
+
+
+def test_bf16_decode_saves_g_and_h(stp, ctx):
+    w = _bf16_workload(64, 256, 512, 1000)
+    inp = syn.make_layer_inputs(w)
+    got = run_layer(stp, ctx, inp, w.D, w.F, w.V, embed="table")
+    compare(got, oracle_layer(inp), TOL["bf16"], FWD + SAVED + BWD)
+
+
+@pytest.mark.parametrize("D,F", [(2048, 1024), (1024, 8192), (4096, 11008)])
+def test_bf16_decode_cluster_split_shapes(stp, ctx, D, F):
+    """Down projections whose K is split over 2..8 blocks of a cluster, and
+    the 7B shape (d_ff 11008 = 172 k blocks of 64)."""
+    w = _bf16_workload(64, D, F, 2000)
+    inp = syn.make_layer_inputs(w, with_dy=False)
+    got = run_layer(stp, ctx, inp, w.D, w.F, w.V, embed="table", training=False)
+    compare(got, oracle_layer(inp, training=False), TOL["bf16"], FWD)
+
+
+def test_olmo2_1b_decode_layer_full_size(stp, ctx):
+    """The bench workload itself: T = 64, d_model 2048, d_ff 8192, vocab 100352,
+    the whole table in HBM, every output row checked against the oracle."""
+    w = syn.WORKLOADS["olmo2-1b-decode-layer"]
+    inp = syn.make_layer_inputs(w)
+    got = run_layer(stp, ctx, inp, w.D, w.F, w.V, embed="table", training=False)
+    x, wg, wu, wd = (inp.f64(k) for k in ("x", "w_gate", "w_up", "w_down"))
+    E_rows = syn.bf16_bits_to_f32(inp.table[inp.ids]).astype(np.float64)
+    ref = oracle.ffn_forward(x, np.arange(w.T), wg, wu, wd, E_rows)
+    compare(got, ref, TOL["bf16"], FWD)

@@ -395,17 +395,21 @@ staple_status staple_ffn_fwd(staple_context* ctx, staple_dtype dtype, int32_t T,
                              const void* w_gate, const void* w_up, const void* w_down, void* z,
                              void* y, void* g_save, void* h_save, void* workspace,
                              size_t workspace_bytes, staple_stream stream) {
-  (void)workspace;
-  (void)workspace_bytes;
   if (!ctx) return STAPLE_EINVAL;
   STP_TRY(check_dims(dtype, T, D, F));
   STP_TRY(check_embed(embed, dtype, F));
+  (void)workspace;
+  (void)workspace_bytes;
+  const bool decode = dtype == STAPLE_BF16 && T >= 1 && T <= stp::kMaxDecodeT;
   if (!ptrs_ok(dtype, {w_gate, w_up, w_down})) return STAPLE_EINVAL;
   if (T > 0 && !ptrs_ok(dtype, {x, z, y})) return STAPLE_EINVAL;
   if ((g_save && !ptrs_ok(dtype, {g_save})) || (h_save && !ptrs_ok(dtype, {h_save})))
     return STAPLE_EINVAL;
   STP_TRY(set_device(ctx));
   stp::TraceScope trace_scope(ctx->tracer);
+  if (decode)
+    return stp::tc_decode_fwd(ctx->di, T, D, F, x, embed, w_gate, w_up, w_down, z, y, g_save,
+                              h_save, ctx->d_err, cs(stream));
   if (dtype == STAPLE_BF16)
     return stp::tc_ffn_fwd(ctx->di, T, D, F, x, embed, w_gate, w_up, w_down, z, y, g_save, h_save,
                            ctx->d_err, cs(stream));
