@@ -324,7 +324,7 @@ def run_train(stp, ctx, w, steps, warmup, world, local):
     dwg, dwu = (torch.empty((F, D), dtype=torch.float32, device="cuda") for _ in range(2))
     dwd = torch.empty((D, F), dtype=torch.float32, device="cuda")
     wsb = stp.staple_workspace_bytes(T, D, F)
-    ws = torch.empty(wsb, dtype=torch.uint8, device="cuda")
+    ws = torch.zeros(wsb, dtype=torch.uint8, device="cuda")
     stream, side = torch.cuda.Stream(), torch.cuda.Stream()
     emb_rows = stp.make_embed(stp.STAPLE_EMBED_ROWS, rows, F, inverse, T)
     emb_none = stp.make_embed(stp.STAPLE_EMBED_NONE)

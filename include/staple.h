@@ -23,9 +23,9 @@
  *    the device (an id >= V, a kernel wait that ran out of time) are recorded
  *    in the context's device error word; staple_get_error() reads it.
  *  - The caller owns every tensor.  The library allocates device memory only
- *    in staple_context_create, staple_table_register (flag DEVICE_COPY) and
- *    staple_cache_build; the per-step calls allocate nothing and take scratch
- *    from a caller workspace sized by staple_workspace_bytes().
+ *    in staple_context_create and staple_cache_build (and events in
+ *    staple_trace_enable); the per-step calls allocate nothing and take
+ *    scratch from a caller workspace sized by staple_workspace_bytes().
  *  - Pointers are device pointers unless the argument says "host".
  *    Matrices are row-major and dense (leading dimension = row length).
  *    bf16 tensors are passed as raw 16-bit storage.
@@ -152,9 +152,13 @@ staple_status staple_cache_free(staple_cache* cache);
 /* --------------------------------------------------------------- workspace */
 
 /* Bytes of caller-owned device scratch the per-step calls need for T tokens,
- * d_model D, d_ff F (flags reserved, pass 0).  A workspace of this size (or
- * larger), 256-byte aligned, may be reused by every call with the same or
- * smaller sizes, one call at a time per workspace. */
+ * d_model D, d_ff F (flags reserved, pass 0).  Zero-fill the workspace once
+ * (e.g. cudaMemset) before its first use: its first bytes hold the decode
+ * kernel's tile counters and ready flags, which every call leaves at zero
+ * again (after a call that reported an error, zero-fill it again).  A
+ * workspace of this size (or larger), 256-byte aligned, may be reused by
+ * every call with the same D and F and the same or smaller T, one call at a
+ * time per workspace. */
 size_t staple_workspace_bytes(int32_t T, int32_t D, int32_t F, uint32_t flags);
 
 /* ------------------------------------------------------- retrieval (K1..K4) */
@@ -225,7 +229,11 @@ typedef struct staple_embed {
  *   g_save, h_save [T][F]  out (training): g and h for the backward pass;
  *               both NULL for inference
  * bf16 needs D and F multiples of 64 and 16-byte aligned pointers;
- * T >= 0.  fp32 accepts any sizes. */
+ * T >= 0.  fp32 needs F a multiple of 8.
+ * bf16 with 1 <= T <= 256 (decode sizes) runs one persistent kernel that
+ * streams both projections' weights across all SMs and needs the workspace
+ * (staple_workspace_bytes, zero-filled once); larger T runs the tiled GEMMs
+ * and ignores it. */
 staple_status staple_ffn_fwd(staple_context* ctx, staple_dtype dtype, int32_t T, int32_t D,
                              int32_t F, const void* x, const staple_embed* embed,
                              const void* w_gate, const void* w_up, const void* w_down, void* z,

@@ -53,7 +53,7 @@ def run_layer(stp, ctx, inp, D, F, V, *, embed="table", training=True, rows_tabl
         keep.append(rows)
         out["miss_count"] = int(mc.item())
     wsb = stp.staple_workspace_bytes(T, D, F)
-    ws = torch.empty(max(wsb, 256), dtype=torch.uint8, device="cuda")
+    ws = torch.zeros(max(wsb, 256), dtype=torch.uint8, device="cuda")
     try:
         stp.staple_ffn_fwd(ctx, sdt, T, D, F, x, e, wg, wu, wd, z, y,
                            g if training else None, h if training else None, ws, wsb)

@@ -1,0 +1,556 @@
+// One persistent tcgen05 kernel for the STAPLE layer at decode sizes
+// (T <= 256 tokens): gate/up with the fused E-row add and SiLU gating, then
+// the down projection, in a single launch.
+//
+// With a handful of tokens the layer streams its weights once per step and
+// is bound by HBM bandwidth, so the kernel is organised around that stream:
+//
+//  * The weights take the MMA's M side (128 rows per tile) and the tokens its
+//    N side (T rounded up to 16).  A gate/up tile stacks 64 W_gate and the
+//    matching 64 W_up rows (64 features); a down tile is 128 W_down rows.
+//    Every stage carries `sub` 64-wide k blocks, so each weight row is read
+//    in runs of sub * 128 bytes (short runs per row leave HBM far below its
+//    bandwidth).  Weights and activations have separate rings: the weight
+//    ring is deep (HBM latency), the activation ring shallow (it hits L2).
+//  * Phase 1, gate/up: whole tiles are spread over the blocks.  A block
+//    finishes a tile straight from tensor memory, 16 tokens at a time: g and
+//    u rows go to shared memory, then all 128 epilogue threads compute
+//    h = u + E[id_t][f] (E rows prefetched into shared memory during the main
+//    loop), z = SiLU(g) h (g and h saved when asked) over consecutive
+//    features, and the tile's ready flag goes up.  (A compact loop: the
+//    epilogue runs while every SM's memory queues are full, where a large
+//    unrolled body stalls on instruction fetch.)
+//  * Phase 2, down: the down units (tile x `sub` k blocks) are split evenly
+//    over the blocks (stream-K), so every SM streams the same share of
+//    W_down.  A unit's activation loads wait (bounded spin) on the ready
+//    flags of the gate/up tiles that produced its z columns; its weight
+//    loads do not wait.  Each block's piece of a tile leaves an fp32 partial
+//    in the workspace (L2-resident) and bumps the tile's counter.
+//  * The down sums are spread over all blocks: once a block has finished its
+//    own pieces, its epilogue warps take 16-row chunks from an atomic work
+//    queue, wait (bounded) until the chunk's tile is complete, sum the
+//    partials in piece order (deterministic) and write y = bf16(sum).
+//  * Every block finishes its gate/up tiles before it needs anybody's z, so
+//    all waits end while all blocks are resident (grid <= SMs, one block
+//    per SM).  Counters, flags and queue counters live in the first bytes of
+//    the workspace; the last event of a call resets them, so a zero-filled
+//    workspace stays valid across calls and graph replays.
+//
+// Warps: 0 weight (A) loads, 1 MMA issue + tensor memory, 2 activation (B)
+// loads, 3..6 epilogue (each owns one 32-lane quarter of tensor memory).
+// Every mbarrier wait and flag spin is bounded (STAPLE_ETIMEOUT).  The
+// kernel is launched as a programmatic dependent: weights stream before
+// griddepcontrol.wait; activations, outputs and counters only after it.
+#pragma once
+
+#include "common.cuh"
+
+namespace stp {
+namespace fused {
+
+constexpr int BM = 128;
+constexpr int BK = 64;
+constexpr int kMaxStages = 8;
+constexpr int kThreads = 224;
+constexpr int A_BLOCK = BM * BK * 2;  // 128 weight rows x 64 k: 16 KiB
+constexpr int kMaxN = 256;
+constexpr int kStagesB = 3;
+constexpr int kChunkRows = 16;        // rows of a down tile per reduction chunk
+constexpr int kXStride = 17;          // fp32 words per row of the g/u exchange chunk
+// shared memory after the rings: barriers + flags (512 B), token ids,
+// g/u exchange chunk [128][17] fp32; then the E tile [N][64] bf16
+constexpr int kTailFixed = 512 + kMaxN * 4 + 128 * kXStride * 4;
+
+struct Params {
+  int32_t T, N, D, F;
+  int32_t sub;         // k blocks per unit (and per pipeline stage)
+  int32_t stages;      // depth of the weight ring
+  int32_t stages_b;    // depth of the activation ring
+  int32_t G;           // gate/up tiles (F / 64)
+  int32_t Dt;          // down tiles (ceil(D / 128))
+  int32_t ug, ud;      // units per gate/up tile, per down tile
+  int32_t Ud;          // down units (Dt * ud)
+  int32_t maxp_d;      // partial slots per down tile
+  // activations / outputs
+  uint16_t* z;
+  uint16_t* g_save;
+  uint16_t* h_save;
+  uint16_t* y;
+  const uint16_t* e_base;
+  int64_t e_pitch;
+  const int32_t* e_index;
+  int64_t e_rows;
+  int32_t e_mode;
+  // workspace
+  uint32_t* cnt;       // [Dt] pieces finished per down tile
+  uint32_t* ready;     // [G] gate/up tile finished
+  uint32_t* queue;     // [2]: next chunk to reduce, events seen
+  float* part;         // [Dt * maxp_d][N][128]
+  int32_t* err;
+};
+
+__host__ __device__ inline int range_start(int c, int U, int grid) {
+  return int((int64_t(c) * U) / grid);
+}
+// The block whose range holds unit x.
+__host__ __device__ inline int owner(int x, int U, int grid) {
+  int c = int((int64_t(x) * grid) / U);
+  while (c + 1 < grid && range_start(c + 1, U, grid) <= x) ++c;
+  while (c > 0 && range_start(c, U, grid) > x) --c;
+  return c;
+}
+
+__device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void grid_dep_launch() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void epi_bar() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+__device__ __forceinline__ uint32_t ld_acquire(const uint32_t* a) {
+  uint32_t v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(a) : "memory");
+  return v;
+}
+__device__ __forceinline__ void st_release(uint32_t* a, uint32_t v) {
+  asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(a), "r"(v) : "memory");
+}
+__device__ __forceinline__ void fence_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+__device__ __forceinline__ float4 ldcg4(const float* a) {
+  return __ldcg(reinterpret_cast<const float4*>(a));
+}
+__device__ __forceinline__ void add4(float4& a, const float4 b) {
+  a.x += b.x;
+  a.y += b.y;
+  a.z += b.z;
+  a.w += b.w;
+}
+// Bounded spin until *a >= want (acquire).  False (and *abort set, the
+// error word written) after kWaitLimitNs.
+__device__ __forceinline__ bool spin_until(const uint32_t* a, uint32_t want, volatile int* abort,
+                                           int32_t* err) {
+  if (ld_acquire(a) >= want) return true;
+  const uint64_t t0 = globaltimer();
+  while (ld_acquire(a) < want) {
+    __nanosleep(64);
+    if (*abort) return false;
+    if (globaltimer() - t0 > kWaitLimitNs) {
+      *abort = 1;
+      report(err, STAPLE_ETIMEOUT);
+      return false;
+    }
+  }
+  return true;
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    decode_fused_kernel(const __grid_constant__ CUtensorMap tm_wg,
+                        const __grid_constant__ CUtensorMap tm_wu,
+                        const __grid_constant__ CUtensorMap tm_wd,
+                        const __grid_constant__ CUtensorMap tm_x,
+                        const __grid_constant__ CUtensorMap tm_z, const Params p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  const int b_block = p.N * BK * 2;
+  const int a_stage = p.sub * A_BLOCK;
+  const int b_stage = p.sub * b_block;
+  const int S = p.stages;
+  const int SB = p.stages_b;
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + S * a_stage;
+  uint8_t* tail = sB + SB * b_stage;
+  uint64_t* fullA = reinterpret_cast<uint64_t*>(tail);
+  uint64_t* fullB = fullA + kMaxStages;
+  uint64_t* emptyA = fullB + kMaxStages;
+  uint64_t* emptyB = emptyA + kMaxStages;
+  uint64_t* tfull = emptyB + kMaxStages;  // [2]
+  uint64_t* tempty = tfull + 2;           // [2]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tempty + 2);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  int* s_flag = const_cast<int*>(abort_flag + 1);
+  // set by an epilogue warp whose wait failed, read by all four after a
+  // barrier, so every epilogue warp takes the same path through bar.sync
+  int* s_epi_fail = s_flag + 1;
+  int32_t* s_ids = reinterpret_cast<int32_t*>(tail + 512);            // [kMaxN]
+  float* s_x = reinterpret_cast<float*>(s_ids + kMaxN);               // [128][kXStride]
+  uint16_t* s_e = reinterpret_cast<uint16_t*>(s_x + 128 * kXStride);  // [N][64]
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int grid = gridDim.x;
+  // this block's work: gate/up tiles [t0, t1) (ug units each), then down
+  // units [d0, d1); local step i < ngs is gate/up, the rest down
+  const int t0 = range_start(blockIdx.x, p.G, grid), t1 = range_start(blockIdx.x + 1, p.G, grid);
+  const int d0 = range_start(blockIdx.x, p.Ud, grid), d1 = range_start(blockIdx.x + 1, p.Ud, grid);
+  const int ngs = (t1 - t0) * p.ug;
+  const int nsteps = ngs + (d1 - d0);
+  const uint32_t ncols = p.N <= 32 ? 32 : (p.N <= 64 ? 64 : (p.N <= 128 ? 128 : 256));
+  const uint32_t tmem_cols = 2 * ncols;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(&fullA[s], 1);
+      mbar_init(&emptyA[s], 1);
+    }
+    for (int s = 0; s < SB; ++s) {
+      mbar_init(&fullB[s], 1);
+      mbar_init(&emptyB[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&tfull[b], 1);
+      mbar_init(&tempty[b], 4);
+    }
+    *abort_flag = 0;
+    *s_epi_fail = 0;
+    fence_barrier_init();
+    tma_prefetch_desc(&tm_wg);
+    tma_prefetch_desc(&tm_wu);
+    tma_prefetch_desc(&tm_wd);
+    tma_prefetch_desc(&tm_x);
+    tma_prefetch_desc(&tm_z);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, tmem_cols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  grid_dep_launch();
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ---------------------------------------------------- weight (A) loads
+      const uint64_t once = l2_policy_evict_first();  // weights are read once per call
+      int s = 0;
+      uint32_t ph = 0;
+      for (int i = 0; i < nsteps; ++i) {
+        if (!mbar_wait(&emptyA[s], ph ^ 1, abort_flag, p.err)) break;
+        mbar_arrive_expect_tx(&fullA[s], a_stage);
+        uint8_t* a = sA + s * a_stage;
+        for (int j = 0; j < p.sub; ++j) {
+          if (i < ngs) {
+            const int tile = t0 + i / p.ug, u = i % p.ug;
+            const int k0 = (u * p.sub + j) * BK;
+            tma_load_2d_hint(&tm_wg, &fullA[s], a + j * A_BLOCK, k0, tile * 64, once);
+            tma_load_2d_hint(&tm_wu, &fullA[s], a + j * A_BLOCK + A_BLOCK / 2, k0, tile * 64, once);
+          } else {
+            const int x = d0 + i - ngs, tile = x / p.ud, u = x % p.ud;
+            tma_load_2d_hint(&tm_wd, &fullA[s], a + j * A_BLOCK, (u * p.sub + j) * BK, tile * BM,
+                             once);
+          }
+        }
+        if (++s == S) {
+          s = 0;
+          ph ^= 1;
+        }
+      }
+    }
+  } else if (warp == 2) {
+    if (lane == 0) {
+      // -------------------------------------------------- activation (B) loads
+      grid_dep_wait();
+      int s = 0;
+      uint32_t ph = 0;
+      for (int i = 0; i < nsteps; ++i) {
+        if (!mbar_wait(&emptyB[s], ph ^ 1, abort_flag, p.err)) break;
+        uint8_t* b = sB + s * b_stage;
+        if (i < ngs) {
+          const int u = i % p.ug;
+          mbar_arrive_expect_tx(&fullB[s], b_stage);
+          for (int j = 0; j < p.sub; ++j)
+            tma_load_2d(&tm_x, &fullB[s], b + j * b_block, (u * p.sub + j) * BK, 0);
+        } else {
+          const int u = (d0 + i - ngs) % p.ud;
+          // z columns [f_lo, f_hi) come from gate/up tiles f_lo/64 .. (f_hi-1)/64
+          const int f_lo = u * p.sub * BK;
+          const int f_hi = min(p.F, f_lo + p.sub * BK);
+          bool ok = true;
+          for (int t = f_lo / 64; t <= (f_hi - 1) / 64 && ok; ++t)
+            ok = spin_until(&p.ready[t], 1u, abort_flag, p.err);
+          if (!ok) break;
+          fence_async_global();
+          mbar_arrive_expect_tx(&fullB[s], b_stage);
+          for (int j = 0; j < p.sub; ++j)
+            tma_load_2d(&tm_z, &fullB[s], b + j * b_block, (u * p.sub + j) * BK, 0);
+        }
+        if (++s == SB) {
+          s = 0;
+          ph ^= 1;
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ---------------------------------------------------------------- MMA
+      const uint32_t idesc = idesc_bf16_f32(BM, p.N, false, false);
+      int sa = 0, sb = 0;
+      uint32_t pha = 0, phb = 0;
+      int piece = 0;
+      bool ok = true;
+      for (int i0 = 0; i0 < nsteps && ok; ++piece) {
+        int nunits;
+        if (i0 < ngs) {
+          nunits = p.ug;
+        } else {
+          const int x = d0 + i0 - ngs;
+          nunits = min(d1, (x / p.ud + 1) * p.ud) - x;
+        }
+        const int buf = piece & 1;
+        if (!mbar_wait(&tempty[buf], ((piece >> 1) & 1) ^ 1, abort_flag, p.err)) break;
+        tc_fence_after();
+        const uint32_t dacc = tmem_base + uint32_t(buf) * ncols;
+        for (int i = 0; i < nunits; ++i) {
+          if (!mbar_wait(&fullA[sa], pha, abort_flag, p.err) ||
+              !mbar_wait(&fullB[sb], phb, abort_flag, p.err)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a_addr = smem_u32(sA + sa * a_stage);
+          const uint32_t b_addr = smem_u32(sB + sb * b_stage);
+          for (int j = 0; j < p.sub; ++j) {
+#pragma unroll
+            for (int k = 0; k < BK / 16; ++k)
+              umma_bf16(dacc, sw128_desc(a_addr + j * A_BLOCK + k * 32, 16, 1024),
+                        sw128_desc(b_addr + j * b_block + k * 32, 16, 1024), idesc,
+                        (i | j | k) != 0 ? 1u : 0u);
+          }
+          umma_commit(&emptyA[sa]);
+          umma_commit(&emptyB[sb]);
+          if (++sa == S) {
+            sa = 0;
+            pha ^= 1;
+          }
+          if (++sb == SB) {
+            sb = 0;
+            phb ^= 1;
+          }
+        }
+        i0 += nunits;
+        if (ok) umma_commit(&tfull[buf]);
+      }
+    }
+  } else {
+    // ----------------------------------------------------------- epilogue
+    const int q = warp & 3;
+    const int row = q * 32 + lane;
+    const int et = threadIdx.x - 96;  // 0..127
+    grid_dep_wait();
+    for (int t = et; t < p.T; t += 128) {
+      int32_t id = -1;
+      if (p.e_mode != STAPLE_EMBED_NONE) {
+        const int64_t v = p.e_index[t];
+        if (v < 0 || v >= p.e_rows) report(p.err, STAPLE_EIDRANGE);
+        else id = int32_t(v);
+      }
+      s_ids[t] = id;
+    }
+    epi_bar();
+    int piece = 0;
+    bool alive = true;
+    // ---- phase 1: whole gate/up tiles, finished from tensor memory
+    for (int tile = t0; tile < t1 && alive; ++tile, ++piece) {
+      const int f0 = tile * 64;
+      // E[id_t][f0 .. f0+63] for every token: 128 bytes per row, 16-byte loads
+      // issued while the tile's main loop is still streaming.  Up to 8 loads
+      // per thread are put in flight before any of them is stored (behind a
+      // saturated weight stream each round trip is long).
+      for (int vb = et; vb < p.T * 8; vb += 8 * 128) {
+        uint4 w[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          const int v = vb + k * 128;
+          w[k] = make_uint4(0u, 0u, 0u, 0u);
+          if (v < p.T * 8) {
+            const int id = s_ids[v >> 3];
+            if (id >= 0)
+              w[k] = __ldg(reinterpret_cast<const uint4*>(p.e_base + int64_t(id) * p.e_pitch + f0) +
+                           (v & 7));
+          }
+        }
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          const int v = vb + k * 128;
+          if (v < p.T * 8) reinterpret_cast<uint4*>(s_e)[v] = w[k];
+        }
+      }
+      const int buf = piece & 1;
+      const bool ok = mbar_wait(&tfull[buf], (piece >> 1) & 1, abort_flag, p.err);
+      if (!__all_sync(0xffffffffu, ok) && lane == 0) *s_epi_fail = 1;
+      epi_bar();
+      if (*s_epi_fail) {
+        alive = false;
+        break;
+      }
+      tc_fence_after();
+      const uint32_t tacc = tmem_base + (uint32_t(q * 32) << 16) + uint32_t(buf) * ncols;
+      for (int c = 0; c < p.N; c += 16) {
+        uint32_t r[16];
+        tmem_ld16(tacc + c, r);
+        tmem_ld_wait16(r);
+#pragma unroll
+        for (int j = 0; j < 16; ++j) s_x[row * kXStride + j] = __uint_as_float(r[j]);
+        epi_bar();
+        const int tn = min(16, p.T - c);
+        for (int e = et; e < 64 * tn; e += 128) {
+          const int fl = e & 63, j = e >> 6, t = c + j;
+          const float g = s_x[fl * kXStride + j];
+          const float h = s_x[(64 + fl) * kXStride + j] + bf2f(s_e[t * 64 + fl]);
+          const int64_t off = int64_t(t) * p.F + f0 + fl;
+          p.z[off] = __bfloat16_as_ushort(__float2bfloat16_rn(g * sigmoid_f(g) * h));
+          if (p.g_save) p.g_save[off] = __bfloat16_as_ushort(__float2bfloat16_rn(g));
+          if (p.h_save) p.h_save[off] = __bfloat16_as_ushort(__float2bfloat16_rn(h));
+        }
+        epi_bar();
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&tempty[buf]);
+      __threadfence();
+      fence_async_global();
+      epi_bar();
+      if (et == 0) st_release(&p.ready[tile], 1u);
+    }
+    // ---- phase 2: down pieces -> fp32 partial slots
+    for (int x = d0; x < d1 && alive; ++piece) {
+      const int tile = x / p.ud;
+      const int x_end = min(d1, (tile + 1) * p.ud);
+      const int idx = blockIdx.x - owner(tile * p.ud, p.Ud, grid);
+      x = x_end;
+      const int buf = piece & 1;
+      const bool ok = mbar_wait(&tfull[buf], (piece >> 1) & 1, abort_flag, p.err);
+      if (!__all_sync(0xffffffffu, ok) && lane == 0) *s_epi_fail = 1;
+      epi_bar();
+      if (*s_epi_fail) {
+        alive = false;
+        break;
+      }
+      tc_fence_after();
+      float* mine = p.part + int64_t(tile * p.maxp_d + idx) * p.N * BM;
+      const uint32_t tacc = tmem_base + (uint32_t(q * 32) << 16) + uint32_t(buf) * ncols;
+      for (int c = 0; c < p.N; c += 32) {
+        uint32_t r[32];
+        tmem_ld32(tacc + c, r);
+        tmem_ld_wait(r);
+        const int cn = min(32, p.N - c);  // the slot holds N token rows
+#pragma unroll
+        for (int j = 0; j < 32; ++j)
+          if (j < cn) mine[(c + j) * BM + row] = __uint_as_float(r[j]);
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&tempty[buf]);
+      __threadfence();
+      epi_bar();
+      if (et == 0) atomicAdd(&p.cnt[tile], 1u);
+    }
+
+    // ---- down sums: 16-row chunks from the shared work queue.  queue[0]
+    // hands out chunks; queue[1] counts events: each reduced chunk and each
+    // block's final fetch past the end.  The event that completes the count
+    // (nchunks + grid) is the last use of any counter or flag of this call,
+    // so that thread resets them all for the next call.
+    const int chunks_per_tile = BM / kChunkRows;
+    const uint32_t nchunks = uint32_t(p.Dt * chunks_per_tile);
+    const uint32_t nevents = nchunks + uint32_t(grid);
+    const int64_t pstride = int64_t(p.N) * BM;
+    auto event = [&]() {
+      if (atomicAdd(&p.queue[1], 1u) == nevents - 1) {
+        for (int k = 0; k < p.Dt; ++k) p.cnt[k] = 0u;
+        for (int k = 0; k < p.G; ++k) p.ready[k] = 0u;
+        p.queue[0] = 0u;
+        p.queue[1] = 0u;
+        __threadfence();
+      }
+    };
+    while (alive) {
+      // one thread takes a chunk and waits for its tile; all follow its verdict
+      epi_bar();
+      if (et == 0) {
+        int code = int(atomicAdd(&p.queue[0], 1u));
+        if (code < int(nchunks)) {
+          const int tl = code / chunks_per_tile;
+          const int first = owner(tl * p.ud, p.Ud, grid);
+          const int np = owner((tl + 1) * p.ud - 1, p.Ud, grid) - first + 1;
+          if (!spin_until(&p.cnt[tl], uint32_t(np), abort_flag, p.err)) code = -1;
+        }
+        *s_flag = code;
+      }
+      epi_bar();
+      const int code = *s_flag;
+      if (code < 0) break;
+      const uint32_t c = uint32_t(code);
+      if (c >= nchunks) {
+        if (et == 0) event();
+        break;
+      }
+      const int tile = int(c) / chunks_per_tile;
+      const int r0 = (int(c) % chunks_per_tile) * kChunkRows;
+      const int o0 = owner(tile * p.ud, p.Ud, grid);
+      const int npieces = owner((tile + 1) * p.ud - 1, p.Ud, grid) - o0 + 1;
+      __threadfence();
+      const float* parts = p.part + int64_t(tile * p.maxp_d) * pstride;
+      // groups of 4 consecutive rows: T * 4 groups, one per thread per pass;
+      // all partials of a group are loaded before the first add
+      const int ngroups = p.T * (kChunkRows / 4);
+      for (int gi = et; gi < ngroups; gi += 128) {
+        const int t = gi >> 2, r = r0 + (gi & 3) * 4;
+        const float* src = parts + t * BM + r;
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int i0 = 0; i0 < npieces; i0 += 16) {
+          float4 v[16];
+#pragma unroll
+          for (int k = 0; k < 16; ++k)
+            v[k] = i0 + k < npieces ? ldcg4(src + (i0 + k) * pstride) : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+          for (int k = 0; k < 16; ++k)
+            if (i0 + k < npieces) add4(acc, v[k]);
+        }
+        const int d = tile * BM + r;
+        uint16_t* dst = p.y + int64_t(t) * p.D + d;
+        if (d + 3 < p.D) {
+          uint2 w;
+          w.x = pack_bf2(acc.x, acc.y);
+          w.y = pack_bf2(acc.z, acc.w);
+          *reinterpret_cast<uint2*>(dst) = w;
+        } else {
+          const float a[4] = {acc.x, acc.y, acc.z, acc.w};
+          for (int k = 0; k < 4 && d + k < p.D; ++k)
+            dst[k] = __bfloat16_as_ushort(__float2bfloat16_rn(a[k]));
+        }
+      }
+      __threadfence();
+      epi_bar();
+      if (et == 0) event();
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) {
+    __syncwarp();
+    tmem_dealloc(tmem_base, tmem_cols);
+  }
+}
+
+// Shared memory after the rings for N tokens.
+inline int tail_bytes(int N) { return kTailFixed + N * 64 * 2; }
+// Ring depths: the activation ring keeps kStagesB stages (it is fed from
+// L2), the weight ring takes the rest of shared memory.
+inline int stages_b(int N, int sub) { (void)N; (void)sub; return kStagesB; }
+inline int ring_stages(int N, int sub) {
+  const int budget = 227 * 1024 - 1024 - tail_bytes(N) - stages_b(N, sub) * sub * N * BK * 2;
+  const int s = budget / (sub * A_BLOCK);
+  return s > kMaxStages ? kMaxStages : s;
+}
+inline int smem_bytes(int N, int sub) {
+  return 1024 + ring_stages(N, sub) * sub * A_BLOCK + stages_b(N, sub) * sub * N * BK * 2 +
+         tail_bytes(N);
+}
+
+}  // namespace fused
+}  // namespace stp

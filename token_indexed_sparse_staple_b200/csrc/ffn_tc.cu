@@ -13,7 +13,7 @@
 #include <atomic>
 #include <mutex>
 
-#include "decode_tc.cuh"
+#include "decode_fused.cuh"
 #include "gemm_tc.cuh"
 #include "internal.h"
 
@@ -90,11 +90,101 @@ bool kmajor_rows(CUtensorMap* m, const void* base, int rows, int k, int64_t ld, 
   return make_map(m, base, uint64_t(k), uint64_t(rows), uint64_t(ld), tc::BK, uint32_t(box_rows));
 }
 
-template <int MODE>
-staple_status launch_decode(const char* name, const DeviceInfo& di, int grid, int cluster,
-                            const CUtensorMap& a0, const CUtensorMap& a1, const CUtensorMap& b,
-                            const dec::Params& p, cudaStream_t st) {
-  auto kern = dec::decode_kernel<MODE>;
+}  // namespace
+
+// ---------------------------------------------------------------- decode
+namespace {
+
+struct DecodePlan {
+  int N, sub, G, Dt, ug, ud, Ud, grid, maxp_d;
+  size_t counter_bytes, part_bytes;
+};
+
+// Partial slots per down tile for every grid up to kMaxDecodeGrid: a block's
+// range holds at least floor(Ud / kMaxDecodeGrid) units, so a tile of `units`
+// units meets at most (units - 1) / that + 2 ranges.  (The exact count is not
+// monotone in the grid size, so the bound is what sizes the workspace and
+// strides the slots.)
+int piece_bound(int units, int U) {
+  const int minlen = std::max(1, U / kMaxDecodeGrid);
+  return std::min(kMaxDecodeGrid, (units - 1) / minlen + 2);
+}
+
+DecodePlan plan_decode(int T, int D, int F, int num_sms) {
+  DecodePlan pl{};
+  pl.N = cdiv(T, 16) * 16;
+  pl.sub = ((D / 64) % 2 == 0 && (F / 64) % 2 == 0 && fused::ring_stages(pl.N, 2) >= 3) ? 2 : 1;
+  pl.G = F / 64;
+  pl.Dt = cdiv(D, fused::BM);
+  pl.ug = (D / 64) / pl.sub;
+  pl.ud = (F / 64) / pl.sub;
+  pl.Ud = pl.Dt * pl.ud;
+  // every block needs at least one down unit (so the blocks covering a down
+  // tile are consecutive and each writes its partial slot)
+  pl.grid = std::max(1, std::min(std::min(num_sms, kMaxDecodeGrid), pl.Ud));
+  pl.maxp_d = piece_bound(pl.ud, pl.Ud);
+  pl.counter_bytes = decode_counter_bytes(D, F);
+  pl.part_bytes = size_t(pl.Dt * pl.maxp_d) * pl.N * fused::BM * sizeof(float);
+  return pl;
+}
+
+}  // namespace
+
+size_t decode_counter_bytes(int D, int F) {
+  const size_t words = size_t((F / 64) + cdiv(D, fused::BM) + 2);
+  return (words * sizeof(uint32_t) + 255) & ~size_t(255);
+}
+
+size_t decode_scratch_bytes(int T, int D, int F) {
+  if (T < 1 || T > kMaxDecodeT || D % 64 || F % 64) return 0;
+  // the largest grid the launcher may use gives the most pieces per tile
+  const DecodePlan pl = plan_decode(T, D, F, kMaxDecodeGrid);
+  return pl.part_bytes;
+}
+
+staple_status tc_decode_fwd(const DeviceInfo& di, int T, int D, int F, const void* x,
+                            const staple_embed* e, const void* wg, const void* wu, const void* wd,
+                            void* z, void* y, void* g_save, void* h_save, void* ws,
+                            int32_t* err, cudaStream_t st) {
+  const DecodePlan pl = plan_decode(T, D, F, di.num_sms);
+  CUtensorMap mg, mu, md, mx, mz;
+  if (!kmajor_rows(&mg, wg, F, D, D, 64) || !kmajor_rows(&mu, wu, F, D, D, 64) ||
+      !kmajor_rows(&md, wd, D, F, F, fused::BM) || !kmajor_rows(&mx, x, T, D, D, pl.N) ||
+      !kmajor_rows(&mz, z, T, F, F, pl.N))
+    return STAPLE_ECUDA;
+  fused::Params p{};
+  p.T = T;
+  p.N = pl.N;
+  p.D = D;
+  p.F = F;
+  p.sub = pl.sub;
+  p.stages = fused::ring_stages(pl.N, pl.sub);
+  p.stages_b = fused::stages_b(pl.N, pl.sub);
+  p.G = pl.G;
+  p.Dt = pl.Dt;
+  p.ug = pl.ug;
+  p.ud = pl.ud;
+  p.Ud = pl.Ud;
+  p.maxp_d = pl.maxp_d;
+  p.z = static_cast<uint16_t*>(z);
+  p.g_save = static_cast<uint16_t*>(g_save);
+  p.h_save = static_cast<uint16_t*>(h_save);
+  p.y = static_cast<uint16_t*>(y);
+  p.e_mode = e ? e->mode : STAPLE_EMBED_NONE;
+  if (e && e->mode != STAPLE_EMBED_NONE) {
+    p.e_base = static_cast<const uint16_t*>(e->base);
+    p.e_pitch = e->row_pitch;
+    p.e_index = e->index;
+    p.e_rows = e->n_rows;
+  }
+  uint32_t* words = static_cast<uint32_t*>(ws);
+  p.cnt = words;
+  p.ready = words + pl.Dt;
+  p.queue = words + pl.Dt + pl.G;
+  p.part = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + pl.counter_bytes);
+  p.err = err;
+
+  auto kern = fused::decode_fused_kernel;
   static std::atomic<uint64_t> attr_done{0};
   const uint64_t bit = uint64_t(1) << (di.device & 63);
   if (!(attr_done.load() & bit)) {
@@ -104,106 +194,18 @@ staple_status launch_decode(const char* name, const DeviceInfo& di, int grid, in
     attr_done.fetch_or(bit);
   }
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(grid);
-  cfg.blockDim = dim3(dec::kThreads);
-  cfg.dynamicSmemBytes = dec::smem_bytes(p.N, p.sub);
+  cfg.gridDim = dim3(pl.grid);
+  cfg.blockDim = dim3(fused::kThreads);
+  cfg.dynamicSmemBytes = fused::smem_bytes(pl.N, pl.sub);
   cfg.stream = st;
-  cudaLaunchAttribute attr[2];
+  cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
-  attr[1].id = cudaLaunchAttributeClusterDimension;
-  attr[1].val.clusterDim.x = unsigned(cluster);
-  attr[1].val.clusterDim.y = 1;
-  attr[1].val.clusterDim.z = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = cluster > 1 ? 2 : 1;
-  cudaError_t e = cudaSuccess;
-  STP_LAUNCH(name, st, e = cudaLaunchKernelEx(&cfg, kern, a0, a1, b, p));
-  return e == cudaSuccess ? STAPLE_OK : STAPLE_ECUDA;
-}
-
-// Largest k blocks per stage (4, 2, 1) that divides a split, keeps a ring of
-// at least three stages and leaves room in the ring for the epilogue's
-// exchange tile (rows x (N rounded to 32, plus one) fp32).
-// (With one split, a stage that runs past K reads zeros, so any size fits.)
-int pick_sub(int N, int kb_per, int splits, int exchange_rows) {
-  const int need = exchange_rows * (((N + 31) & ~31) + 1) * 4;
-  for (int s : {4, 2, 1}) {
-    if (splits > 1 && kb_per % s) continue;
-    const int st = dec::ring_stages(N, s);
-    if (st >= 3 && st * s * (dec::A_BLOCK + N * dec::BK * 2) >= need) return s;
-  }
-  return 1;
-}
-
-}  // namespace
-
-// K split of the down projection: as many blocks per 128-row tile as the
-// SMs allow (at most one cluster of kMaxDecodeSplits), k blocks per split
-// rounded up to a multiple of 4 so that stages stay 512 bytes per row.
-void decode_splits(int num_sms, int D, int F, int* splits_out, int* kb_per_out) {
-  const int tiles_m = cdiv(D, dec::BM);
-  const int k_blocks = F / dec::BK;
-  int splits = std::max(1, std::min(kMaxDecodeSplits, num_sms / tiles_m));
-  splits = std::min(splits, k_blocks);
-  int kb_per = cdiv(k_blocks, splits);
-  if (splits > 1) kb_per = cdiv(kb_per, 4) * 4;
-  *kb_per_out = kb_per;
-  *splits_out = cdiv(k_blocks, kb_per);
-}
-
-staple_status tc_decode_fwd(const DeviceInfo& di, int T, int D, int F, const void* x,
-                            const staple_embed* e, const void* wg, const void* wu, const void* wd,
-                            void* z, void* y, void* g_save, void* h_save, int32_t* err,
-                            cudaStream_t st) {
-  const int N = cdiv(T, 16) * 16;
-  CUtensorMap mg, mu, mx, md, mz;
-  if (!kmajor_rows(&mg, wg, F, D, D, 64) || !kmajor_rows(&mu, wu, F, D, D, 64) ||
-      !kmajor_rows(&mx, x, T, D, D, N) || !kmajor_rows(&md, wd, D, F, F, dec::BM) ||
-      !kmajor_rows(&mz, z, T, F, F, N))
-    return STAPLE_ECUDA;
-  const int tiles_d = cdiv(D, dec::BM);
-  int splits = 1, kb_per = 1;
-  decode_splits(di.num_sms, D, F, &splits, &kb_per);
-
-  dec::Params p{};
-  p.T = T;
-  p.N = N;
-  p.err = err;
-  // gate/up: F / 64 feature blocks over the whole K = D
-  p.M = F;
-  p.K = D;
-  p.k_blocks = D / dec::BK;
-  p.kb_per = p.k_blocks;
-  p.splits = 1;
-  p.sub = pick_sub(N, p.kb_per, 1, 64);
-  p.stages = dec::ring_stages(N, p.sub);
-  p.z = static_cast<uint16_t*>(z);
-  p.g_save = static_cast<uint16_t*>(g_save);
-  p.h_save = static_cast<uint16_t*>(h_save);
-  p.ldf = F;
-  p.e_mode = e ? e->mode : STAPLE_EMBED_NONE;
-  if (e && e->mode != STAPLE_EMBED_NONE) {
-    p.e_base = static_cast<const uint16_t*>(e->base);
-    p.e_pitch = e->row_pitch;
-    p.e_index = e->index;
-    p.e_rows = e->n_rows;
-  }
-  staple_status s =
-      launch_decode<dec::GATEUP>("k5_gateup_decode", di, F / 64, 1, mg, mu, mx, p, st);
-  if (s != STAPLE_OK) return s;
-  // down: D / 128 row tiles, K = F split over the blocks of a cluster
-  dec::Params q = p;
-  q.M = D;
-  q.K = F;
-  q.k_blocks = F / dec::BK;
-  q.kb_per = kb_per;
-  q.splits = splits;
-  q.sub = pick_sub(N, q.kb_per, splits, splits > 1 ? dec::BM : 0);
-  q.stages = dec::ring_stages(N, q.sub);
-  q.y = static_cast<uint16_t*>(y);
-  return launch_decode<dec::DOWN>("k6_down_decode", di, tiles_d * splits, splits, md, md, mz, q,
-                                  st);
+  cfg.numAttrs = 1;
+  cudaError_t ce = cudaSuccess;
+  STP_LAUNCH("k5k6_decode_fused", st, ce = cudaLaunchKernelEx(&cfg, kern, mg, mu, md, mx, mz, p));
+  return ce == cudaSuccess ? STAPLE_OK : STAPLE_ECUDA;
 }
 
 staple_status tc_ffn_fwd(const DeviceInfo& di, int T, int D, int F, const void* x,

@@ -78,12 +78,15 @@ staple_status tc_ffn_bwd(const DeviceInfo& di, int T, int D, int F, const void* 
 
 // decode path (ffn_tc.cu): 1 <= T <= kMaxDecodeT tokens, bf16
 constexpr int kMaxDecodeT = 256;
-constexpr int kMaxDecodeSplits = 4;   // the down projection's K splits form one cluster
-void decode_splits(int num_sms, int D, int F, int* splits, int* kb_per);
+constexpr int kMaxDecodeGrid = 160;   // blocks of the persistent decode kernel (<= one per SM)
+// Workspace layout: [decode counters, decode_counter_bytes(D, F), zero-filled
+// once by the caller and left at zero by every call][shared scratch].
+size_t decode_counter_bytes(int D, int F);
+size_t decode_scratch_bytes(int T, int D, int F);
 staple_status tc_decode_fwd(const DeviceInfo& di, int T, int D, int F, const void* x,
                             const staple_embed* e, const void* wg, const void* wu, const void* wd,
-                            void* z, void* y, void* g_save, void* h_save, int32_t* err,
-                            cudaStream_t st);
+                            void* z, void* y, void* g_save, void* h_save, void* ws,
+                            int32_t* err, cudaStream_t st);
 
 // simt_f32.cu (fp32 on CUDA cores)
 staple_status f32_ffn_fwd(int T, int D, int F, const float* x, const staple_embed* e,

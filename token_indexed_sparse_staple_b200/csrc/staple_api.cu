@@ -320,11 +320,10 @@ staple_status staple_cache_free(staple_cache* c) {
 // --------------------------------------------------------------- workspace
 
 size_t staple_workspace_bytes(int32_t T, int32_t D, int32_t F, uint32_t flags) {
-  (void)D;
   (void)flags;
-  if (T < 0 || F <= 0) return 0;
-  size_t b = stp::seg_reduce_workspace(T, F);
-  return (b + 255) & ~size_t(255);
+  if (T < 0 || F <= 0 || D <= 0) return 0;
+  const size_t b = std::max(stp::seg_reduce_workspace(T, F), stp::decode_scratch_bytes(T, D, F));
+  return stp::decode_counter_bytes(D, F) + ((b + 255) & ~size_t(255));
 }
 
 // --------------------------------------------------------------- retrieval
@@ -398,9 +397,11 @@ staple_status staple_ffn_fwd(staple_context* ctx, staple_dtype dtype, int32_t T,
   if (!ctx) return STAPLE_EINVAL;
   STP_TRY(check_dims(dtype, T, D, F));
   STP_TRY(check_embed(embed, dtype, F));
-  (void)workspace;
-  (void)workspace_bytes;
   const bool decode = dtype == STAPLE_BF16 && T >= 1 && T <= stp::kMaxDecodeT;
+  if (decode && (!workspace || !aligned16(workspace) ||
+                 workspace_bytes < stp::decode_counter_bytes(D, F) +
+                                       stp::decode_scratch_bytes(T, D, F)))
+    return STAPLE_EINVAL;
   if (!ptrs_ok(dtype, {w_gate, w_up, w_down})) return STAPLE_EINVAL;
   if (T > 0 && !ptrs_ok(dtype, {x, z, y})) return STAPLE_EINVAL;
   if ((g_save && !ptrs_ok(dtype, {g_save})) || (h_save && !ptrs_ok(dtype, {h_save})))
@@ -409,7 +410,7 @@ staple_status staple_ffn_fwd(staple_context* ctx, staple_dtype dtype, int32_t T,
   stp::TraceScope trace_scope(ctx->tracer);
   if (decode)
     return stp::tc_decode_fwd(ctx->di, T, D, F, x, embed, w_gate, w_up, w_down, z, y, g_save,
-                              h_save, ctx->d_err, cs(stream));
+                              h_save, workspace, ctx->d_err, cs(stream));
   if (dtype == STAPLE_BF16)
     return stp::tc_ffn_fwd(ctx->di, T, D, F, x, embed, w_gate, w_up, w_down, z, y, g_save, h_save,
                            ctx->d_err, cs(stream));
@@ -432,9 +433,10 @@ staple_status staple_embed_bwd(staple_context* ctx, staple_dtype dtype, int32_t 
   STP_TRY(check_dims(dtype, T, D, F));
   if (!ptrs_ok(dtype, {w_down})) return STAPLE_EINVAL;
   if (T > 0 && !ptrs_ok(dtype, {dy, g_save, h_save, dgh})) return STAPLE_EINVAL;
+  const size_t head = stp::decode_counter_bytes(D, F);  // left untouched
   if (dE) {
     if (!sorted_pos || !inverse || !seg_off || !U_dev || !aligned16(dE)) return STAPLE_EINVAL;
-    const size_t need = stp::seg_reduce_workspace(T, F);
+    const size_t need = head + stp::seg_reduce_workspace(T, F);
     if (T > 0 && (!workspace || workspace_bytes < need || !aligned16(workspace)))
       return STAPLE_EINVAL;
   }
@@ -451,7 +453,9 @@ staple_status staple_embed_bwd(staple_context* ctx, staple_dtype dtype, int32_t 
   const size_t es = esize(dtype);
   const void* dh = static_cast<const uint8_t*>(dgh) + size_t(F) * es;
   return stp::launch_seg_reduce(dtype == STAPLE_BF16, dh, 2 * int64_t(F), sorted_pos, inverse,
-                                seg_off, U_dev, T, F, dE, static_cast<float*>(workspace), st);
+                                seg_off, U_dev, T, F, dE,
+                                reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + head),
+                                st);
 }
 
 staple_status staple_ffn_bwd(staple_context* ctx, staple_dtype dtype, int32_t T, int32_t D,
