@@ -23,6 +23,7 @@ sample of the same workload: each step is one token's forward restricted to a
 from __future__ import annotations
 
 import argparse
+import hashlib
 import json
 import os
 import statistics
@@ -147,6 +148,34 @@ class Clocks:
                 "power_w_max": max(r[2] for r in rows), "samples": len(load), "reasons": reasons}
 
 
+# DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of one launch,
+# from the ncu capture summarised in the named profile.  It describes the
+# kernel as captured, so it is reported only while the kernel's sources hash
+# to the captured value; otherwise the roofline's traffic is null.
+CAPTURED_TRAFFIC = {
+    "k5k6_decode_fused": {
+        "bytes": 104_795_008,   # mean of two launches: 104,419,840 and 105,170,176
+        "sources": ["token_indexed_sparse_staple_b200/csrc/decode_fused.cuh",
+                    "token_indexed_sparse_staple_b200/csrc/common.cuh"],
+        "sha256": "ec425cc20cbff1a5e5b33be8d745bdb6ebf5816610cdc65a3906bc5acb7c4d0e",
+        "profile": "profiles/decode_fused_olmo2_1b_T64.md",
+    },
+}
+
+
+def captured_traffic(kernel):
+    c = CAPTURED_TRAFFIC.get(kernel)
+    if c is None:
+        return None, "no capture"
+    h = hashlib.sha256()
+    for f in c["sources"]:
+        with open(os.path.join(ROOT, f), "rb") as fh:
+            h.update(fh.read())
+    if h.hexdigest() != c["sha256"]:
+        return None, "kernel changed since the capture in " + c["profile"]
+    return c["bytes"], c["profile"]
+
+
 def bf16_randn(shape, std, seed):
     """Seeded N(0, std) draws made on the GPU, rounded to bf16 (used for the
     big tensors; the parity tests use the numpy generator of `synthetic`)."""
@@ -219,8 +248,7 @@ def run_decode(stp, ctx, w, args, world, local):
             decode_step(stp, ctx, w, st, s, stream)
     torch.cuda.synchronize()
     assert stp.staple_get_error(ctx, stream) == 0
-    # capture G steps once; replay to cover the K timed steps
-    stp.staple_trace_enable(ctx, True)
+    # capture G steps once; replay to cover the K timed steps (untraced)
     graph = torch.cuda.CUDAGraph()
     with torch.cuda.graph(graph, stream=stream):
         for s in range(G):
@@ -244,14 +272,28 @@ def run_decode(stp, ctx, w, args, world, local):
         torch.cuda.synchronize()
         t1 = time.time()
     ms = ev0.elapsed_time(ev1)
+    assert stp.staple_get_error(ctx, stream) == 0
+    ms_max = max_over_ranks(ms, world)
+    del graph
+    # the same steps again with per-kernel CUDA events recorded around every
+    # launch: the kernel list and shares (events between launches stop the
+    # programmatic overlap of consecutive launches, so these steps are slower)
+    stp.staple_trace_enable(ctx, True)
+    tgraph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(tgraph, stream=stream):
+        for s in range(G):
+            decode_step(stp, ctx, w, st, s, stream)
+    with torch.cuda.stream(stream):
+        for _ in range(4):
+            tgraph.replay()
+    torch.cuda.synchronize()
     trace = stp.staple_trace_read(ctx)
     stp.staple_trace_enable(ctx, False)
     assert stp.staple_get_error(ctx, stream) == 0
-    ms_max = max_over_ranks(ms, world)
+    del tgraph
     kern = kernel_table(trace, G)
     res = {"K": K, "ms": ms_max, "ms_local": ms, "clocks": clk.summary(t0, t1), "kernels": kern,
            "launches_per_step": sum(d["launches"] for d in kern.values()) / G}
-    del graph
     # end to end through the public call with host buffers: H2D of x and ids
     # from pinned memory, the layer, D2H of y, every step
     Ke = min(K, 4096)
@@ -283,12 +325,14 @@ def run_decode(stp, ctx, w, args, world, local):
         torch.cuda.synchronize()
     e_ms = max_over_ranks(e0.elapsed_time(e1), world)
     res["e2e"] = {"K": Ke, "ms": e_ms, "h2d": h2d, "d2h": d2h}
-    # dominant kernel: algorithmic bytes of one gate/up launch
+    # dominant (and only) kernel: the fused decode launch.  Algorithmic bytes
+    # of one launch: the three weight matrices, x, the T gathered E rows, ids,
+    # and the z and y outputs
     T, D, F = w.T, w.D, w.F
-    res["roofline_kernel"] = "k5_gateup"
-    res["alg_bytes"] = 2 * F * D * 2 + T * D * 2 + T * F * 2 + T * F * 2 + T * 4
-    res["alg_note"] = ("k5_gateup bytes per launch: W_gate + W_up (2*F*D*2) + x (T*D*2) + "
-                       "E rows (T*F*2) + z (T*F*2) + ids (T*4)")
+    res["roofline_kernel"] = "k5k6_decode_fused"
+    res["alg_bytes"] = 3 * F * D * 2 + T * D * 2 + T * F * 2 + T * 4 + T * F * 2 + T * D * 2
+    res["alg_note"] = ("k5k6_decode_fused bytes per launch: W_gate + W_up + W_down (3*F*D*2) + "
+                       "x (T*D*2) + E rows (T*F*2) + ids (T*4) + z (T*F*2) + y (T*D*2)")
     return res
 
 
@@ -489,7 +533,12 @@ def main():
     K = dec["K"]
     value = world * w.T * K / (dec["ms"] / 1000.0)
     kd = dec["kernels"].get(dec["roofline_kernel"], {})
-    ach = dec["alg_bytes"] / (kd.get("avg_us", float("nan")) * 1e-6) / 1e9
+    # one launch per step: the untraced timed step bounds the launch duration
+    # from above; the traced average is reported beside it
+    one = abs(dec["launches_per_step"] - 1.0) < 1e-9 and kd
+    launch_us = dec["ms_local"] * 1000.0 / K if one else kd.get("avg_us", float("nan"))
+    ach = dec["alg_bytes"] / (launch_us * 1e-6) / 1e9
+    traffic, traffic_src = captured_traffic(dec["roofline_kernel"])
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K,
         "warmup": args.warmup, "ms_per_step": dec["ms"] / K, "higher_is_better": True,
@@ -500,8 +549,12 @@ def main():
                    "graph": "steps replayed from one captured CUDA graph of 64 steps"},
         "roofline": {"bound": "hbm", "kernel": dec["roofline_kernel"], "achieved": ach,
                      "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": ach / pk["hbm_gbs"],
-                     "traffic": None, "peak_source": pk["source"] + " (copy bandwidth)",
-                     "alg_bytes_per_launch": dec["alg_bytes"], "note": dec["alg_note"]},
+                     "traffic": traffic, "traffic_source": traffic_src,
+                     "peak_source": pk["source"] + " (copy bandwidth)",
+                     "alg_bytes_per_launch": dec["alg_bytes"], "note": dec["alg_note"],
+                     "launch_us": launch_us, "traced_launch_us": kd.get("avg_us"),
+                     "duration": ("untraced timed step (one launch per step)" if one else
+                                  "traced per-launch CUDA events")},
         "e2e": {"value": world * w.T * dec["e2e"]["K"] / (dec["e2e"]["ms"] / 1000.0),
                 "unit": "tokens/s", "h2d_bytes_per_step": dec["e2e"]["h2d"],
                 "d2h_bytes_per_step": dec["e2e"]["d2h"], "steps": dec["e2e"]["K"],
