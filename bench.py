@@ -357,9 +357,21 @@ def run_train(stp, ctx, w, steps, warmup, world, local):
     x = [bf16_randn((T, D), w.x_std, syn.SEED_ACT + 2 * s) for s in range(S)]
     dy = [bf16_randn((T, D), w.dy_std, syn.SEED_ACT + 2 * s + 1) for s in range(S)]
     i32 = dict(dtype=torch.int32, device="cuda")
-    unique, inverse, sorted_pos, slot, miss = (torch.empty(T, **i32) for _ in range(5))
-    seg, U, mc = torch.empty(T + 1, **i32), torch.empty(1, **i32), torch.empty(1, **i32)
-    rows = torch.empty((T, F), dtype=torch.bfloat16, device="cuda")
+
+    class Retrieval:
+        """One microbatch's retrieval outputs (two of them alternate)."""
+
+        def __init__(self):
+            self.unique, self.inverse, self.sorted_pos, self.slot, self.miss = (
+                torch.empty(T, **i32) for _ in range(5))
+            self.seg, self.U, self.mc = (torch.empty(T + 1, **i32), torch.empty(1, **i32),
+                                         torch.empty(1, **i32))
+            self.rows = torch.empty((T, F), dtype=torch.bfloat16, device="cuda")
+            self.emb = stp.make_embed(stp.STAPLE_EMBED_ROWS, self.rows, F, self.inverse, T)
+            self.ready = torch.cuda.Event()   # rows gathered (prefetch streams)
+            self.free = torch.cuda.Event()    # last reader done (main stream)
+
+    buf = [Retrieval(), Retrieval()]
     z, g, h = (torch.empty((T, F), dtype=torch.bfloat16, device="cuda") for _ in range(3))
     y = torch.empty((T, D), dtype=torch.bfloat16, device="cuda")
     dgh = torch.empty((T, 2 * F), dtype=torch.bfloat16, device="cuda")
@@ -369,19 +381,36 @@ def run_train(stp, ctx, w, steps, warmup, world, local):
     dwd = torch.empty((D, F), dtype=torch.float32, device="cuda")
     wsb = stp.staple_workspace_bytes(T, D, F)
     ws = torch.zeros(wsb, dtype=torch.uint8, device="cuda")
-    stream, side = torch.cuda.Stream(), torch.cuda.Stream()
-    emb_rows = stp.make_embed(stp.STAPLE_EMBED_ROWS, rows, F, inverse, T)
+    stream = torch.cuda.Stream()
+    pf, pf_side = torch.cuda.Stream(), torch.cuda.Stream()   # prefetch: main and miss streams
     emb_none = stp.make_embed(stp.STAPLE_EMBED_NONE)
+
+    def prefetch(s):
+        """Retrieval for microbatch s (dedup, probe, hit and miss gathers) on
+        the prefetch streams, into the buffer whose previous reader (step
+        s - 2) has finished.  Successive microbatches are pipelined this way
+        (retrieval-path table, Prefill row); there is no optimizer in this
+        layer benchmark, so no row the prefetch reads is updated in between."""
+        r = buf[s % 2]
+        pf.wait_event(r.free)
+        stp.staple_gather_rows(ctx, cache, tab, ids[s % S], T, r.unique, r.inverse, r.seg,
+                               r.sorted_pos, r.U, r.slot, r.miss, r.mc, r.rows, stream=pf,
+                               side=pf_side)
+        r.ready.record(pf)
 
     def step(s, staple=True):
         b = s % S
+        r = buf[s % 2]
         if staple:
-            stp.staple_gather_rows(ctx, cache, tab, ids[b], T, unique, inverse, seg, sorted_pos, U,
-                                   slot, miss, mc, rows, stream=stream, side=side)
-        stp.staple_ffn_fwd(ctx, stp.STAPLE_BF16, T, D, F, x[b], emb_rows if staple else emb_none,
+            prefetch(s + 1)
+            stream.wait_event(r.ready)
+        stp.staple_ffn_fwd(ctx, stp.STAPLE_BF16, T, D, F, x[b], r.emb if staple else emb_none,
                            wg, wu, wd, z, y, g, h, ws, wsb, stream=stream)
-        stp.staple_embed_bwd(ctx, stp.STAPLE_BF16, T, D, F, dy[b], g, h, wd, sorted_pos, inverse,
-                             seg, U, dgh, dE if staple else None, ws, wsb, stream=stream)
+        stp.staple_embed_bwd(ctx, stp.STAPLE_BF16, T, D, F, dy[b], g, h, wd, r.sorted_pos,
+                             r.inverse, r.seg, r.U, dgh, dE if staple else None, ws, wsb,
+                             stream=stream)
+        if staple:
+            r.free.record(stream)
         stp.staple_ffn_bwd(ctx, stp.STAPLE_BF16, T, D, F, dy[b], x[b], z, dgh, wg, wu, dx, dwg, dwu,
                            dwd, stream=stream)
 
@@ -389,8 +418,11 @@ def run_train(stp, ctx, w, steps, warmup, world, local):
     try:
         for mode in ("staple", "dense"):
             staple = mode == "staple"
+            nw = max(warmup, 3)
             with torch.cuda.stream(stream):
-                for s in range(max(warmup, 3)):
+                if staple:
+                    prefetch(0)
+                for s in range(nw):
                     step(s, staple)
             torch.cuda.synchronize()
             assert stp.staple_get_error(ctx, stream) == 0
@@ -403,8 +435,10 @@ def run_train(stp, ctx, w, steps, warmup, world, local):
                 t0 = time.time()
                 with torch.cuda.stream(stream):
                     ev0.record(stream)
-                    for s in range(steps):
+                    for s in range(nw, nw + steps):
                         step(s, staple)
+                    if staple:   # the last prefetch ends inside the timed region too
+                        stream.wait_event(buf[(nw + steps) % 2].ready)
                     ev1.record(stream)
                 torch.cuda.synchronize()
                 t1 = time.time()
@@ -414,8 +448,8 @@ def run_train(stp, ctx, w, steps, warmup, world, local):
             if staple:
                 out[mode]["kernels"] = kernel_table(stp.staple_trace_read(ctx), steps)
                 stp.staple_trace_enable(ctx, False)
-                out["U"] = int(U.item())
-                out["misses"] = int(mc.item())
+                out["U"] = int(buf[0].U.item())
+                out["misses"] = int(buf[0].mc.item())
     finally:
         stp.staple_cache_free(cache)
         stp.staple_table_unregister(tab)

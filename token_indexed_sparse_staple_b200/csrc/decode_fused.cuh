@@ -28,8 +28,10 @@
 //    in the workspace (L2-resident) and bumps the tile's counter.
 //  * The down sums are spread over all blocks: once a block has finished its
 //    own pieces, its epilogue warps take 16-row chunks from an atomic work
-//    queue, wait (bounded) until the chunk's tile is complete, sum the
-//    partials in piece order (deterministic) and write y = bf16(sum).
+//    queue, wait (bounded) until the chunk's tile is complete, bring every
+//    piece's 16 x N slice into the (then idle) ring memory with TMA loads
+//    that are all in flight at once, sum them in piece order
+//    (deterministic) and write y = bf16(sum).
 //  * Every block finishes its gate/up tiles before it needs anybody's z, so
 //    all waits end while all blocks are resident (grid <= SMs, one block
 //    per SM).  Counters, flags and queue counters live in the first bytes of
@@ -71,6 +73,7 @@ struct Params {
   int32_t ug, ud;      // units per gate/up tile, per down tile
   int32_t Ud;          // down units (Dt * ud)
   int32_t maxp_d;      // partial slots per down tile
+  int32_t rcap;        // partial slices per reduction batch (ring memory / slice)
   // activations / outputs
   uint16_t* z;
   uint16_t* g_save;
@@ -148,7 +151,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                         const __grid_constant__ CUtensorMap tm_wu,
                         const __grid_constant__ CUtensorMap tm_wd,
                         const __grid_constant__ CUtensorMap tm_x,
-                        const __grid_constant__ CUtensorMap tm_z, const Params p) {
+                        const __grid_constant__ CUtensorMap tm_z,
+                        const __grid_constant__ CUtensorMap tm_part, const Params p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -172,6 +176,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   // set by an epilogue warp whose wait failed, read by all four after a
   // barrier, so every epilogue warp takes the same path through bar.sync
   int* s_epi_fail = s_flag + 1;
+  uint64_t* rbar = reinterpret_cast<uint64_t*>(tail + 320);  // partial slices landed
   int32_t* s_ids = reinterpret_cast<int32_t*>(tail + 512);            // [kMaxN]
   float* s_x = reinterpret_cast<float*>(s_ids + kMaxN);               // [128][kXStride]
   uint16_t* s_e = reinterpret_cast<uint16_t*>(s_x + 128 * kXStride);  // [N][64]
@@ -201,6 +206,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&tfull[b], 1);
       mbar_init(&tempty[b], 4);
     }
+    mbar_init(rbar, 1);
     *abort_flag = 0;
     *s_epi_fail = 0;
     fence_barrier_init();
@@ -209,6 +215,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     tma_prefetch_desc(&tm_wd);
     tma_prefetch_desc(&tm_x);
     tma_prefetch_desc(&tm_z);
+    tma_prefetch_desc(&tm_part);
   }
   if (warp == 1) {
     tmem_alloc(tmem_slot, tmem_cols);
@@ -394,15 +401,30 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int j = 0; j < 16; ++j) s_x[row * kXStride + j] = __uint_as_float(r[j]);
         epi_bar();
-        const int tn = min(16, p.T - c);
-        for (int e = et; e < 64 * tn; e += 128) {
-          const int fl = e & 63, j = e >> 6, t = c + j;
-          const float g = s_x[fl * kXStride + j];
-          const float h = s_x[(64 + fl) * kXStride + j] + bf2f(s_e[t * 64 + fl]);
-          const int64_t off = int64_t(t) * p.F + f0 + fl;
-          p.z[off] = __bfloat16_as_ushort(__float2bfloat16_rn(g * sigmoid_f(g) * h));
-          if (p.g_save) p.g_save[off] = __bfloat16_as_ushort(__float2bfloat16_rn(g));
-          if (p.h_save) p.h_save[off] = __bfloat16_as_ushort(__float2bfloat16_rn(h));
+        // thread -> token c + et / 8, features 8 (et % 8) .. +7: one 16-byte
+        // store per output row piece (the memory system is saturated by the
+        // weight stream here, so the number of stores is what costs)
+        const int j = et >> 3, fl0 = (et & 7) * 8, t = c + j;
+        if (t < p.T) {
+          const uint4 ev = *reinterpret_cast<const uint4*>(s_e + t * 64 + fl0);
+          const uint32_t ew[4] = {ev.x, ev.y, ev.z, ev.w};
+          uint32_t zw[4], gw[4], hw[4];
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const int f = fl0 + 2 * k;
+            const float g0 = s_x[f * kXStride + j], g1 = s_x[(f + 1) * kXStride + j];
+            const float h0 = s_x[(64 + f) * kXStride + j] + bf_lo(ew[k]);
+            const float h1 = s_x[(65 + f) * kXStride + j] + bf_hi(ew[k]);
+            zw[k] = pack_bf2(g0 * sigmoid_f(g0) * h0, g1 * sigmoid_f(g1) * h1);
+            gw[k] = pack_bf2(g0, g1);
+            hw[k] = pack_bf2(h0, h1);
+          }
+          const int64_t off = int64_t(t) * p.F + f0 + fl0;
+          *reinterpret_cast<uint4*>(p.z + off) = make_uint4(zw[0], zw[1], zw[2], zw[3]);
+          if (p.g_save)
+            *reinterpret_cast<uint4*>(p.g_save + off) = make_uint4(gw[0], gw[1], gw[2], gw[3]);
+          if (p.h_save)
+            *reinterpret_cast<uint4*>(p.h_save + off) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
         }
         epi_bar();
       }
@@ -456,7 +478,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int chunks_per_tile = BM / kChunkRows;
     const uint32_t nchunks = uint32_t(p.Dt * chunks_per_tile);
     const uint32_t nevents = nchunks + uint32_t(grid);
-    const int64_t pstride = int64_t(p.N) * BM;
+    // slices land in the ring memory, idle once this block's MMAs are done
+    uint8_t* rbuf = sA;
+    const int slice = p.N * kChunkRows * 4;   // bytes of one piece's [N][16] fp32 slice
+    uint32_t rph = 0;
     auto event = [&]() {
       if (atomicAdd(&p.queue[1], 1u) == nevents - 1) {
         for (int k = 0; k < p.Dt; ++k) p.cnt[k] = 0u;
@@ -466,8 +491,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         __threadfence();
       }
     };
+    // thread et owns the float4 groups g = et + 128 m (token g / 4, rows
+    // 4 (g % 4) .. +3 of the chunk); kMaxN * 4 groups at most
+    constexpr int kGroups = kMaxN * (kChunkRows / 4) / 128;
     while (alive) {
-      // one thread takes a chunk and waits for its tile; all follow its verdict
+      // one thread takes a chunk, waits for its tile and puts the first batch
+      // of slice loads in flight; all follow its verdict
       epi_bar();
       if (et == 0) {
         int code = int(atomicAdd(&p.queue[0], 1u));
@@ -475,7 +504,16 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int tl = code / chunks_per_tile;
           const int first = owner(tl * p.ud, p.Ud, grid);
           const int np = owner((tl + 1) * p.ud - 1, p.Ud, grid) - first + 1;
-          if (!spin_until(&p.cnt[tl], uint32_t(np), abort_flag, p.err)) code = -1;
+          if (!spin_until(&p.cnt[tl], uint32_t(np), abort_flag, p.err)) {
+            code = -1;
+          } else {
+            fence_async_global();
+            const int nb = min(np, p.rcap);
+            const int r0 = (code % chunks_per_tile) * kChunkRows;
+            mbar_arrive_expect_tx(rbar, uint32_t(nb * slice));
+            for (int i = 0; i < nb; ++i)
+              tma_load_2d(&tm_part, rbar, rbuf + i * slice, r0, (tl * p.maxp_d + i) * p.N);
+          }
         }
         *s_flag = code;
       }
@@ -491,39 +529,57 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int r0 = (int(c) % chunks_per_tile) * kChunkRows;
       const int o0 = owner(tile * p.ud, p.Ud, grid);
       const int npieces = owner((tile + 1) * p.ud - 1, p.Ud, grid) - o0 + 1;
-      __threadfence();
-      const float* parts = p.part + int64_t(tile * p.maxp_d) * pstride;
-      // groups of 4 consecutive rows: T * 4 groups, one per thread per pass;
-      // all partials of a group are loaded before the first add
       const int ngroups = p.T * (kChunkRows / 4);
-      for (int gi = et; gi < ngroups; gi += 128) {
-        const int t = gi >> 2, r = r0 + (gi & 3) * 4;
-        const float* src = parts + t * BM + r;
-        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-        for (int i0 = 0; i0 < npieces; i0 += 16) {
-          float4 v[16];
+      float4 acc[kGroups];
 #pragma unroll
-          for (int k = 0; k < 16; ++k)
-            v[k] = i0 + k < npieces ? ldcg4(src + (i0 + k) * pstride) : make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-          for (int k = 0; k < 16; ++k)
-            if (i0 + k < npieces) add4(acc, v[k]);
+      for (int m = 0; m < kGroups; ++m) acc[m] = make_float4(0.f, 0.f, 0.f, 0.f);
+      bool ok = true;
+      for (int i0 = 0; i0 < npieces; i0 += p.rcap) {
+        const int nb = min(npieces - i0, p.rcap);
+        if (i0 > 0) {
+          epi_bar();  // the previous batch has been read
+          if (et == 0) {
+            mbar_arrive_expect_tx(rbar, uint32_t(nb * slice));
+            for (int i = 0; i < nb; ++i)
+              tma_load_2d(&tm_part, rbar, rbuf + i * slice, r0,
+                          (tile * p.maxp_d + i0 + i) * p.N);
+          }
         }
-        const int d = tile * BM + r;
+        ok = mbar_wait(rbar, rph, abort_flag, p.err);
+        rph ^= 1u;
+        if (!__all_sync(0xffffffffu, ok) && lane == 0) *s_epi_fail = 1;
+        epi_bar();
+        if (*s_epi_fail) {
+          ok = false;
+          break;
+        }
+        for (int i = 0; i < nb; ++i) {
+          const float4* sl = reinterpret_cast<const float4*>(rbuf + i * slice);
+#pragma unroll
+          for (int m = 0; m < kGroups; ++m) {
+            const int gi = et + 128 * m;
+            if (gi < ngroups) add4(acc[m], sl[gi]);
+          }
+        }
+      }
+      if (!ok) break;
+#pragma unroll
+      for (int m = 0; m < kGroups; ++m) {
+        const int gi = et + 128 * m;
+        if (gi >= ngroups) continue;
+        const int t = gi >> 2, d = tile * BM + r0 + (gi & 3) * 4;
         uint16_t* dst = p.y + int64_t(t) * p.D + d;
         if (d + 3 < p.D) {
           uint2 w;
-          w.x = pack_bf2(acc.x, acc.y);
-          w.y = pack_bf2(acc.z, acc.w);
+          w.x = pack_bf2(acc[m].x, acc[m].y);
+          w.y = pack_bf2(acc[m].z, acc[m].w);
           *reinterpret_cast<uint2*>(dst) = w;
         } else {
-          const float a[4] = {acc.x, acc.y, acc.z, acc.w};
+          const float a[4] = {acc[m].x, acc[m].y, acc[m].z, acc[m].w};
           for (int k = 0; k < 4 && d + k < p.D; ++k)
             dst[k] = __bfloat16_as_ushort(__float2bfloat16_rn(a[k]));
         }
       }
-      __threadfence();
-      epi_bar();
       if (et == 0) event();
     }
   }
@@ -546,6 +602,11 @@ inline int ring_stages(int N, int sub) {
   const int budget = 227 * 1024 - 1024 - tail_bytes(N) - stages_b(N, sub) * sub * N * BK * 2;
   const int s = budget / (sub * A_BLOCK);
   return s > kMaxStages ? kMaxStages : s;
+}
+// Partial slices (one piece's [N][16] fp32) that fit in the two rings.
+inline int reduce_slices(int N, int sub) {
+  const int ring = ring_stages(N, sub) * sub * A_BLOCK + stages_b(N, sub) * sub * N * BK * 2;
+  return ring / (N * kChunkRows * 4);
 }
 inline int smem_bytes(int N, int sub) {
   return 1024 + ring_stages(N, sub) * sub * A_BLOCK + stages_b(N, sub) * sub * N * BK * 2 +

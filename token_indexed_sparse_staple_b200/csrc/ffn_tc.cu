@@ -51,6 +51,21 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows, ui
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// 2-D fp32 tensor map without swizzle: `rows` rows of `cols` floats
+// (leading dimension ld floats), box = box_cols x box_rows.
+bool make_map_f32(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows, uint64_t ld,
+                  uint32_t box_cols, uint32_t box_rows) {
+  auto enc = encoder();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {ld * 4};
+  cuuint32_t box[2] = {box_cols, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<void*>(base), dims, strides, box,
+             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // K-major operand [rows][k]: box 64 (k) x 128 (rows).
 bool kmajor(CUtensorMap* m, const void* base, int rows, int k, int64_t ld) {
   return make_map(m, base, uint64_t(k), uint64_t(rows), uint64_t(ld), tc::BK, 128);
@@ -147,10 +162,15 @@ staple_status tc_decode_fwd(const DeviceInfo& di, int T, int D, int F, const voi
                             void* z, void* y, void* g_save, void* h_save, void* ws,
                             int32_t* err, cudaStream_t st) {
   const DecodePlan pl = plan_decode(T, D, F, di.num_sms);
-  CUtensorMap mg, mu, md, mx, mz;
+  void* part = static_cast<uint8_t*>(ws) + pl.counter_bytes;
+  CUtensorMap mg, mu, md, mx, mz, mp;
   if (!kmajor_rows(&mg, wg, F, D, D, 64) || !kmajor_rows(&mu, wu, F, D, D, 64) ||
       !kmajor_rows(&md, wd, D, F, F, fused::BM) || !kmajor_rows(&mx, x, T, D, D, pl.N) ||
-      !kmajor_rows(&mz, z, T, F, F, pl.N))
+      !kmajor_rows(&mz, z, T, F, F, pl.N) ||
+      // partial slots [Dt * maxp_d * N][128] fp32; a box is one piece's
+      // 16-row slice for all N tokens
+      !make_map_f32(&mp, part, fused::BM, uint64_t(pl.Dt) * pl.maxp_d * pl.N, fused::BM,
+                    fused::kChunkRows, uint32_t(pl.N)))
     return STAPLE_ECUDA;
   fused::Params p{};
   p.T = T;
@@ -166,6 +186,7 @@ staple_status tc_decode_fwd(const DeviceInfo& di, int T, int D, int F, const voi
   p.ud = pl.ud;
   p.Ud = pl.Ud;
   p.maxp_d = pl.maxp_d;
+  p.rcap = fused::reduce_slices(pl.N, pl.sub);
   p.z = static_cast<uint16_t*>(z);
   p.g_save = static_cast<uint16_t*>(g_save);
   p.h_save = static_cast<uint16_t*>(h_save);
@@ -181,7 +202,7 @@ staple_status tc_decode_fwd(const DeviceInfo& di, int T, int D, int F, const voi
   p.cnt = words;
   p.ready = words + pl.Dt;
   p.queue = words + pl.Dt + pl.G;
-  p.part = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + pl.counter_bytes);
+  p.part = static_cast<float*>(part);
   p.err = err;
 
   auto kern = fused::decode_fused_kernel;
@@ -204,7 +225,7 @@ staple_status tc_decode_fwd(const DeviceInfo& di, int T, int D, int F, const voi
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   cudaError_t ce = cudaSuccess;
-  STP_LAUNCH("k5k6_decode_fused", st, ce = cudaLaunchKernelEx(&cfg, kern, mg, mu, md, mx, mz, p));
+  STP_LAUNCH("k5k6_decode_fused", st, ce = cudaLaunchKernelEx(&cfg, kern, mg, mu, md, mx, mz, mp, p));
   return ce == cudaSuccess ? STAPLE_OK : STAPLE_ECUDA;
 }
 
