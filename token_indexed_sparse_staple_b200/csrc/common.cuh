@@ -48,6 +48,15 @@ __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
 
+// The first 1024-byte-aligned address in a dynamic shared-memory array.  The
+// result is formed by pointer arithmetic on the array itself (not through an
+// integer), so the compiler still knows every pointer derived from it is in
+// shared memory and emits shared-space loads and stores; generic ones would
+// share the global-memory pipeline and queue behind its traffic.
+__device__ __forceinline__ uint8_t* align_smem_1024(uint8_t* raw) {
+  return raw + ((1024u - (smem_u32(raw) & 1023u)) & 1023u);
+}
+
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count)
                : "memory");

@@ -22,9 +22,9 @@
 //    unrolled body stalls on instruction fetch.)
 //  * Phase 2, down: the down units (tile x `sub` k blocks) are split evenly
 //    over the blocks (stream-K), so every SM streams the same share of
-//    W_down.  A unit's activation loads wait (bounded spin) on the ready
-//    flags of the gate/up tiles that produced its z columns; its weight
-//    loads do not wait.  Each block's piece of a tile leaves an fp32 partial
+//    W_down.  The activation loads wait (bounded spin, all flags of the
+//    block polled at once by one warp) on the ready flags of the gate/up
+//    tiles that produced the block's z columns; weight loads do not wait.  Each block's piece of a tile leaves an fp32 partial
 //    in the workspace (L2-resident) and bumps the tile's counter.
 //  * The down sums are spread over all blocks: once a block has finished its
 //    own pieces, its epilogue warps take 16-row chunks from an atomic work
@@ -154,8 +154,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         const __grid_constant__ CUtensorMap tm_z,
                         const __grid_constant__ CUtensorMap tm_part, const Params p) {
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                             ~uintptr_t(1023));
+  uint8_t* smem = align_smem_1024(smem_raw);
   const int b_block = p.N * BK * 2;
   const int a_stage = p.sub * A_BLOCK;
   const int b_stage = p.sub * b_block;
@@ -256,33 +255,52 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
   } else if (warp == 2) {
+    // ---------------------------------------------------- activation (B) loads
+    grid_dep_wait();
+    int s = 0;
+    uint32_t ph = 0;
+    bool ok = true;
+    // x for the gate/up steps
     if (lane == 0) {
-      // -------------------------------------------------- activation (B) loads
-      grid_dep_wait();
-      int s = 0;
-      uint32_t ph = 0;
-      for (int i = 0; i < nsteps; ++i) {
-        if (!mbar_wait(&emptyB[s], ph ^ 1, abort_flag, p.err)) break;
+      for (int i = 0; i < ngs && ok; ++i) {
+        ok = mbar_wait(&emptyB[s], ph ^ 1, abort_flag, p.err);
+        if (!ok) break;
+        const int u = i % p.ug;
         uint8_t* b = sB + s * b_stage;
-        if (i < ngs) {
-          const int u = i % p.ug;
-          mbar_arrive_expect_tx(&fullB[s], b_stage);
-          for (int j = 0; j < p.sub; ++j)
-            tma_load_2d(&tm_x, &fullB[s], b + j * b_block, (u * p.sub + j) * BK, 0);
-        } else {
-          const int u = (d0 + i - ngs) % p.ud;
-          // z columns [f_lo, f_hi) come from gate/up tiles f_lo/64 .. (f_hi-1)/64
-          const int f_lo = u * p.sub * BK;
-          const int f_hi = min(p.F, f_lo + p.sub * BK);
-          bool ok = true;
-          for (int t = f_lo / 64; t <= (f_hi - 1) / 64 && ok; ++t)
-            ok = spin_until(&p.ready[t], 1u, abort_flag, p.err);
-          if (!ok) break;
-          fence_async_global();
-          mbar_arrive_expect_tx(&fullB[s], b_stage);
-          for (int j = 0; j < p.sub; ++j)
-            tma_load_2d(&tm_z, &fullB[s], b + j * b_block, (u * p.sub + j) * BK, 0);
+        mbar_arrive_expect_tx(&fullB[s], b_stage);
+        for (int j = 0; j < p.sub; ++j)
+          tma_load_2d(&tm_x, &fullB[s], b + j * b_block, (u * p.sub + j) * BK, 0);
+        if (++s == SB) {
+          s = 0;
+          ph ^= 1;
         }
+      }
+    }
+    ok = __shfl_sync(0xffffffffu, ok, 0);
+    // z for the down steps.  Every gate/up tile that feeds one of this
+    // block's down units must have raised its ready flag.  The whole warp
+    // polls those flags at once: checked one unit at a time, each check is
+    // an L2 round trip on the issue path of every unit.
+    if (ok && d1 > d0) {
+      bool mine = true;
+      for (int x = d0 + lane; x < d1 && mine; x += 32) {
+        // unit x reads z columns [f_lo, f_hi), made by tiles f_lo/64 .. (f_hi-1)/64
+        const int f_lo = (x % p.ud) * p.sub * BK;
+        const int f_hi = min(p.F, f_lo + p.sub * BK);
+        for (int t = f_lo / 64; t <= (f_hi - 1) / 64 && mine; ++t)
+          mine = spin_until(&p.ready[t], 1u, abort_flag, p.err);
+      }
+      ok = __all_sync(0xffffffffu, mine);
+    }
+    if (lane == 0 && ok) {
+      fence_async_global();
+      for (int i = ngs; i < nsteps; ++i) {
+        if (!mbar_wait(&emptyB[s], ph ^ 1, abort_flag, p.err)) break;
+        const int u = (d0 + i - ngs) % p.ud;
+        uint8_t* b = sB + s * b_stage;
+        mbar_arrive_expect_tx(&fullB[s], b_stage);
+        for (int j = 0; j < p.sub; ++j)
+          tma_load_2d(&tm_z, &fullB[s], b + j * b_block, (u * p.sub + j) * BK, 0);
         if (++s == SB) {
           s = 0;
           ph ^= 1;
