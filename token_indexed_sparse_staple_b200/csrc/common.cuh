@@ -38,8 +38,13 @@ __device__ __forceinline__ uint32_t pack_bf2(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&p);
 }
 
-// SiLU and its derivative in fp32 (the fast exponential intrinsic).
-__device__ __forceinline__ float sigmoid_f(float g) { return 1.0f / (1.0f + __expf(-g)); }
+// The logistic function for the bf16 paths: the fast exponential and the
+// fast division intrinsics.  An IEEE division would add a slow-path branch
+// to every call, which serialises the epilogues' independent evaluations.
+// Both intrinsics err by a few fp32 ulps, far below bf16 output rounding.
+// __fdividef returns 0 for a divisor above 2^126 (g < -87), where the
+// logistic function is 0 to fp32 precision anyway.
+__device__ __forceinline__ float sigmoid_f(float g) { return __fdividef(1.0f, 1.0f + __expf(-g)); }
 
 // ---------------------------------------------------------------------------
 // Shared-memory addresses, mbarriers
