@@ -49,7 +49,10 @@ REF_SLICE = 256
 # Plumbing: ranks, peaks, clocks
 # --------------------------------------------------------------------------
 
-def dist_init():
+def dist_init(backend: str | None = None):
+    """Ranks from the torchrun environment.  For more than one rank the
+    process group uses NCCL (one GPU per rank) unless `backend` says
+    otherwise (gloo runs the same plumbing on CPU)."""
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
@@ -58,8 +61,10 @@ def dist_init():
 
         import torch
         import torch.distributed as dist
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+        backend = backend or "nccl"
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=300))
     return rank, world, local
 
 
@@ -70,13 +75,22 @@ def barrier(world):
 
 
 def max_over_ranks(v: float, world: int) -> float:
+    """The largest of the ranks' values (each rank's device time): the job
+    takes as long as its slowest rank."""
     if world == 1:
         return v
     import torch
     import torch.distributed as dist
-    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([v], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def job_value(units_per_rank: float, ms_max: float, world: int) -> float:
+    """Whole-job throughput: the units all ranks processed over the slowest
+    rank's time (weak scaling: every rank runs its own replica)."""
+    return world * units_per_rank / (ms_max / 1000.0)
 
 
 def peaks():
@@ -548,7 +562,8 @@ def main():
     args = ap.parse_args()
     w = syn.WORKLOADS[args.workload]
 
-    rank, world, local = dist_init()
+    # the reference arm runs on host cores only, so its ranks need no GPU
+    rank, world, local = dist_init("gloo" if args.impl == "reference" else None)
     if args.impl == "reference":
         if rank == 0:
             print(json.dumps(reference_arm(w, args)), flush=True)
@@ -565,7 +580,7 @@ def main():
     pk = peaks()
     dec = run_decode(stp, ctx, w, args, world, local)
     K = dec["K"]
-    value = world * w.T * K / (dec["ms"] / 1000.0)
+    value = job_value(w.T * K, dec["ms"], world)
     kd = dec["kernels"].get(dec["roofline_kernel"], {})
     # one launch per step: the untraced timed step bounds the launch duration
     # from above; the traced average is reported beside it
@@ -589,7 +604,7 @@ def main():
                      "launch_us": launch_us, "traced_launch_us": kd.get("avg_us"),
                      "duration": ("untraced timed step (one launch per step)" if one else
                                   "traced per-launch CUDA events")},
-        "e2e": {"value": world * w.T * dec["e2e"]["K"] / (dec["e2e"]["ms"] / 1000.0),
+        "e2e": {"value": job_value(w.T * dec["e2e"]["K"], dec["e2e"]["ms"], world),
                 "unit": "tokens/s", "h2d_bytes_per_step": dec["e2e"]["h2d"],
                 "d2h_bytes_per_step": dec["e2e"]["d2h"], "steps": dec["e2e"]["K"],
                 "how": "per step: pinned H2D of x and ids, staple_ffn_fwd, D2H of y (Python loop)"},
@@ -611,7 +626,7 @@ def main():
             if top[0] in gemm_flops:
                 tf = gemm_flops[top[0]] * wt.T * wt.D * wt.F / (top[1]["avg_us"] * 1e-6) / 1e12
             line["train_layer"] = {
-                "workload": wt.name, "tokens_per_s": world * wt.T / (st_ms / 1000.0),
+                "workload": wt.name, "tokens_per_s": job_value(wt.T, st_ms, world),
                 "ms_per_step": st_ms, "dense_ms_per_step": de_ms,
                 "e_path_overhead": (st_ms - de_ms) / de_ms, "steps": args.train_steps,
                 "U": tr["U"], "misses": tr["misses"],
