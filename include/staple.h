@@ -257,6 +257,28 @@ staple_status staple_embed_bwd(staple_context* ctx, staple_dtype dtype, int32_t 
                                const int32_t* U_dev, void* dgh, float* dE, void* workspace,
                                size_t workspace_bytes, staple_stream stream);
 
+/* Return one layer's table gradient to host memory, where the tables and
+ * their optimizer live (the pages keep the tables in host DRAM and
+ * materialise only the U active rows of a batch: AI Radio episode, paper
+ * summary; Table 4's caption for the 12 offloaded tables).
+ *   dE          device, fp32 [capacity][F] from staple_embed_bwd
+ *   unique      device, int32 [capacity] from staple_dedup
+ *   U_dev       device int32: the number of rows to return
+ *   host_dE     out, host fp32 [capacity][F]: rows [0, U) written
+ *   host_unique out, host int32 [capacity]: ids [0, U) written
+ *   host_U      out, host int32: U
+ * The three host buffers must be page-locked and mapped into the device's
+ * address space (cudaHostAlloc, or cudaHostRegister with the mapped flag);
+ * otherwise STAPLE_EINVAL.  U is read on the device, so only U rows cross the
+ * host link and the host never waits for U.  F a multiple of 4, dE and
+ * host_dE 16-byte aligned.  Asynchronous on `stream`: the host buffers hold
+ * the result once the stream's work up to this call has completed. */
+staple_status staple_embed_grad_to_host(staple_context* ctx, int32_t F, int32_t capacity,
+                                        const float* dE, const int32_t* unique,
+                                        const int32_t* U_dev, float* host_dE,
+                                        int32_t* host_unique, int32_t* host_U,
+                                        staple_stream stream);
+
 /* Rest of the layer backward, consuming dgh from staple_embed_bwd:
  *   dx[T][D]       = dg W_gate + dh W_up                      (dtype)
  *   dw_gate[F][D]  = sum_t dg_t x_t^T       (fp32; NULL: not computed)

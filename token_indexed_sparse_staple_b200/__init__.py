@@ -201,6 +201,15 @@ def staple_embed_bwd(ctx, dtype, T, D, F, dy, g_save, h_save, w_down, sorted_pos
         "staple_embed_bwd")
 
 
+def staple_embed_grad_to_host(ctx, F, capacity, dE, unique, U_dev, host_dE, host_unique, host_U,
+                              stream=None):
+    """Rows [0, U) of dE and the U ids to page-locked, mapped host buffers
+    (U read on the device; see include/staple.h)."""
+    _ok(lib().staple_embed_grad_to_host(ctx, F, capacity, _p(dE), _p(unique), _p(U_dev),
+                                        _p(host_dE), _p(host_unique), _p(host_U),
+                                        _stream(stream)), "staple_embed_grad_to_host")
+
+
 def staple_ffn_bwd(ctx, dtype, T, D, F, dy, x, z, dgh, w_gate, w_up, dx, dw_gate, dw_up, dw_down,
                    workspace=None, workspace_bytes=0, stream=None):
     _ok(lib().staple_ffn_bwd(ctx, dtype, T, D, F, _p(dy), _p(x), _p(z), _p(dgh), _p(w_gate),

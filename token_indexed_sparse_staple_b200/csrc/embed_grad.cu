@@ -153,4 +153,39 @@ staple_status launch_seg_reduce(bool bf16, const void* dh, int64_t ld, const int
   return cudaGetLastError() == cudaSuccess ? STAPLE_OK : STAPLE_ECUDA;
 }
 
+// ---------------------------------------------------------------------------
+// Table-gradient return to host memory: the U rows only, U read on the device
+// ---------------------------------------------------------------------------
+
+// Rows [0, U) of dE (fp32, F floats per row) to mapped host memory with
+// 16-byte loads and stores.  Stores to host memory are posted writes over the
+// host link, so a grid that keeps many in flight runs at the link's rate.
+// Block 0 also writes the U ids and U itself.
+__global__ void __launch_bounds__(256)
+    grad_to_host_kernel(const float* __restrict__ dE, const int32_t* __restrict__ unique,
+                        const int32_t* __restrict__ U_dev, int F, int cap, float* host_dE,
+                        int32_t* host_unique, int32_t* host_U) {
+  const int U = min(*U_dev, cap);
+  const int64_t vecs = int64_t(U) * (F / 4);
+  const float4* src = reinterpret_cast<const float4*>(dE);
+  float4* dst = reinterpret_cast<float4*>(host_dE);
+  for (int64_t v = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; v < vecs;
+       v += int64_t(gridDim.x) * blockDim.x)
+    dst[v] = __ldcs(src + v);
+  if (blockIdx.x == 0) {
+    for (int j = threadIdx.x; j < U; j += blockDim.x) host_unique[j] = unique[j];
+    if (threadIdx.x == 0) *host_U = U;
+  }
+}
+
+staple_status launch_grad_to_host(const float* dE, const int32_t* unique, const int32_t* U_dev,
+                                  int F, int cap, float* host_dE, int32_t* host_unique,
+                                  int32_t* host_U, int num_sms, cudaStream_t st) {
+  if (cap == 0) return STAPLE_OK;
+  STP_LAUNCH("k12_grad_to_host", st,
+             grad_to_host_kernel<<<2 * num_sms, 256, 0, st>>>(dE, unique, U_dev, F, cap, host_dE,
+                                                              host_unique, host_U));
+  return cudaGetLastError() == cudaSuccess ? STAPLE_OK : STAPLE_ECUDA;
+}
+
 }  // namespace stp

@@ -63,6 +63,9 @@ staple_status launch_seg_reduce(bool bf16, const void* dh, int64_t ld, const int
                                 const int32_t* inverse, const int32_t* seg_off,
                                 const int32_t* U_dev, int T, int F, float* dE, float* part,
                                 cudaStream_t st);
+staple_status launch_grad_to_host(const float* dE, const int32_t* unique, const int32_t* U_dev,
+                                  int F, int cap, float* host_dE, int32_t* host_unique,
+                                  int32_t* host_U, int num_sms, cudaStream_t st);
 
 // ffn_tc.cu (bf16, tcgen05)
 staple_status tc_ffn_fwd(const DeviceInfo& di, int T, int D, int F, const void* x,

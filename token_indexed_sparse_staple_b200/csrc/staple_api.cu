@@ -458,6 +458,35 @@ staple_status staple_embed_bwd(staple_context* ctx, staple_dtype dtype, int32_t 
                                 st);
 }
 
+staple_status staple_embed_grad_to_host(staple_context* ctx, int32_t F, int32_t capacity,
+                                        const float* dE, const int32_t* unique,
+                                        const int32_t* U_dev, float* host_dE,
+                                        int32_t* host_unique, int32_t* host_U,
+                                        staple_stream stream) {
+  if (!ctx || F <= 0 || F % 4 || capacity < 0) return STAPLE_EINVAL;
+  if (capacity == 0) return STAPLE_OK;
+  if (!dE || !unique || !U_dev || !host_dE || !host_unique || !host_U || !aligned16(dE) ||
+      !aligned16(host_dE))
+    return STAPLE_EINVAL;
+  STP_TRY(set_device(ctx));
+  // the host buffers must be page-locked and mapped: their device-side
+  // addresses are what the kernel stores to
+  void* d_rows = nullptr;
+  void* d_ids = nullptr;
+  void* d_u = nullptr;
+  if (cudaHostGetDevicePointer(&d_rows, host_dE, 0) != cudaSuccess ||
+      cudaHostGetDevicePointer(&d_ids, host_unique, 0) != cudaSuccess ||
+      cudaHostGetDevicePointer(&d_u, host_U, 0) != cudaSuccess) {
+    cudaGetLastError();
+    return STAPLE_EINVAL;
+  }
+  if (!aligned16(d_rows)) return STAPLE_EINVAL;
+  stp::TraceScope trace_scope(ctx->tracer);
+  return stp::launch_grad_to_host(dE, unique, U_dev, F, capacity, static_cast<float*>(d_rows),
+                                  static_cast<int32_t*>(d_ids), static_cast<int32_t*>(d_u),
+                                  ctx->di.num_sms, cs(stream));
+}
+
 staple_status staple_ffn_bwd(staple_context* ctx, staple_dtype dtype, int32_t T, int32_t D,
                              int32_t F, const void* dy, const void* x, const void* z,
                              const void* dgh, const void* w_gate, const void* w_up, void* dx,
