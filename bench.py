@@ -470,6 +470,193 @@ def run_train(stp, ctx, w, steps, warmup, world, local):
     return out
 
 
+# --------------------------------------------------------------------------
+# Stacks of layers (tables grouped G layers per host row)
+# --------------------------------------------------------------------------
+
+def pinned_group_tables(n_groups, G, V, F, std, seed0, chunk_rows=4096):
+    """Page-locked host tables, one [V][G * F] bf16 array per group (layer
+    G*k + j in columns [j F, (j+1) F)).  Values are seeded N(0, std) draws
+    made on the GPU (one generator per layer, seed seed0 + layer), rounded to
+    bf16 and copied down in row chunks."""
+    import torch
+    out = []
+    for gi in range(n_groups):
+        t = torch.empty((V, G * F), dtype=torch.bfloat16, pin_memory=True)
+        gens = []
+        for j in range(G):
+            g = torch.Generator(device="cuda")
+            g.manual_seed(seed0 + gi * G + j)
+            gens.append(g)
+        blk = torch.empty((chunk_rows, G, F), dtype=torch.bfloat16, device="cuda")
+        for r0 in range(0, V, chunk_rows):
+            n = min(chunk_rows, V - r0)
+            for j in range(G):
+                blk[:n, j] = (torch.randn((n, F), generator=gens[j], device="cuda") * std).to(torch.bfloat16)
+            t[r0:r0 + n].copy_(blk[:n].view(n, G * F))
+        out.append(t)
+    torch.cuda.synchronize()
+    return out
+
+
+def release_pinned():
+    """Return cached page-locked host blocks to the system (torch keeps freed
+    pinned blocks for reuse)."""
+    import gc
+
+    import torch
+    gc.collect()
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+    f = getattr(torch._C, "_host_emptyCache", None)
+    if f is not None:
+        f()
+
+
+def stack_weights(L, D, F, std, seed0=syn.SEED_W):
+    from token_indexed_sparse_staple_b200.stack import LayerWeights
+    return [LayerWeights(bf16_randn((F, D), std, seed0 + 3 * l), bf16_randn((F, D), std, seed0 + 3 * l + 1),
+                         bf16_randn((D, F), std, seed0 + 3 * l + 2)) for l in range(L)]
+
+
+def run_stack_decode(stp, ctx, w, steps, world, local):
+    """16 stacked 7B-shaped layers decoding 64 tokens per step: one dedup and
+    four group gathers (side streams) per step, the 16 fused decode layers,
+    the whole step replayed from one CUDA graph."""
+    import torch
+
+    from token_indexed_sparse_staple_b200.stack import DecodeStack, GroupedTables
+    T, D, F, V, L, G = w.T, w.D, w.F, w.V, w.layers, w.group
+    t0 = time.time()
+    W = stack_weights(L, D, F, w.w_std)
+    host = pinned_group_tables(L // G, G, V, F, w.e_std, syn.SEED_E)
+    setup_s = time.time() - t0
+    freq = syn.calibration_freq(V)
+    tables = GroupedTables(ctx, host, V, F, G, freq, w.cache_frac)
+    S = 64
+    try:
+        s = DecodeStack(ctx, W, tables, T, D, F, V)
+        ids = torch.from_numpy(np.stack([syn.zipf_ids(T, V, w.zipf_s, seed=syn.SEED_IDS + w.index + 7919 * k)
+                                         for k in range(S)])).cuda()
+        xs = bf16_randn((S, T, D), w.x_std, syn.SEED_ACT)
+        st = torch.cuda.Stream()
+        with torch.cuda.stream(st):
+            s.ids_buf.copy_(ids[0])
+            s.xs[0].copy_(xs[0])
+            s.run(st)
+        torch.cuda.synchronize()
+        assert stp.staple_get_error(ctx, st) == 0
+        s.capture(st)
+
+        def one(k):
+            s.ids_buf.copy_(ids[k % S])
+            s.xs[0].copy_(xs[k % S])
+            s.replay()
+
+        with torch.cuda.stream(st):
+            for k in range(8):
+                one(k)
+        torch.cuda.synchronize()
+        barrier(world)
+        ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with Clocks(local) as clk:
+            torch.cuda.synchronize()
+            c0 = time.time()
+            with torch.cuda.stream(st):
+                ev0.record(st)
+                for k in range(steps):
+                    one(k)
+                ev1.record(st)
+            torch.cuda.synchronize()
+            c1 = time.time()
+        assert stp.staple_get_error(ctx, st) == 0
+        ms = max_over_ranks(ev0.elapsed_time(ev1), world)
+        misses = [int(m.item()) for m in s.r.mc]
+        U = int(s.r.U.item())
+        s.release()
+    finally:
+        tables.close()
+    step_ms = ms / steps
+    wbytes = L * 3 * D * F * 2
+    return {"workload": w.name, "layers": L, "groups_of": G, "T": T, "d_model": D, "d_ff": F,
+            "steps": steps, "ms_per_step": step_ms, "tokens_per_s": job_value(T * steps, ms, world),
+            "U_last_step": U, "misses_last_step_per_group": misses,
+            "weight_bytes_per_step": wbytes, "weight_gbs": wbytes / (step_ms * 1e-3) / 1e9,
+            "table_bytes_host": L * V * F * 2, "setup_s": setup_s,
+            "graph": "one CUDA graph per step: dedup, 4 group gathers on side streams, 16 layers",
+            "clocks": clk.summary(c0, c1)}
+
+
+def run_stack_train(stp, ctx, w, steps, world, local):
+    """12 stacked 1B-shaped layers, training: one dedup per step, three group
+    gathers (side streams), forward, backward in reverse with every layer's dE
+    returned to host memory while the backward continues."""
+    import torch
+
+    from token_indexed_sparse_staple_b200.stack import GroupedTables, TrainStack
+    T, D, F, V, L, G = w.T, w.D, w.F, w.V, w.layers, w.group
+    t0 = time.time()
+    W = stack_weights(L, D, F, w.w_std)
+    host = pinned_group_tables(L // G, G, V, F, w.e_std, syn.SEED_E)
+    setup_s = time.time() - t0
+    freq = syn.calibration_freq(V)
+    tables = GroupedTables(ctx, host, V, F, G, freq, w.cache_frac)
+    S = 4
+    try:
+        s = TrainStack(ctx, W, tables, T, D, F, V)
+        ids = [torch.from_numpy(syn.zipf_ids(T, V, w.zipf_s, seed=syn.SEED_IDS + w.index + 7919 * k)).cuda()
+               for k in range(S)]
+        x0 = [bf16_randn((T, D), w.x_std, syn.SEED_ACT + 2 * k) for k in range(S)]
+        dyt = [bf16_randn((T, D), w.dy_std, syn.SEED_ACT + 2 * k + 1) for k in range(S)]
+        st = torch.cuda.Stream()
+        k = 0
+
+        def one():
+            nonlocal k
+            r = s.step(ids[k % S], x0[k % S], dyt[k % S], next_ids=ids[(k + 1) % S], stream=st)
+            k += 1
+            return r
+
+        with torch.cuda.stream(st):
+            for _ in range(2):
+                one()
+        torch.cuda.synchronize()
+        assert stp.staple_get_error(ctx, st) == 0
+        barrier(world)
+        ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with Clocks(local) as clk:
+            torch.cuda.synchronize()
+            c0 = time.time()
+            with torch.cuda.stream(st):
+                ev0.record(st)
+                for _ in range(steps):
+                    r = one()
+                ev1.record(st)
+            torch.cuda.synchronize()
+            c1 = time.time()
+        assert stp.staple_get_error(ctx, st) == 0
+        ms = max_over_ranks(ev0.elapsed_time(ev1), world)
+        U = int(r.U.item())
+        misses = [int(m.item()) for m in r.mc]
+    finally:
+        tables.close()
+    step_ms = ms / steps
+    flops = 18 * T * D * F * L
+    h2d = sum(misses) * G * F * 2          # zero-copy miss rows of all groups
+    d2h = L * (U * F * 4 + U * 4 + 4)      # dE rows, ids and U of every layer
+    pk = peaks()
+    tf = flops / (step_ms * 1e-3) / 1e12
+    return {"workload": w.name, "layers": L, "groups_of": G, "T": T, "d_model": D, "d_ff": F,
+            "steps": steps, "ms_per_step": step_ms, "tokens_per_s": job_value(T * steps, ms, world),
+            "U_last_step": U, "misses_last_step_per_group": misses,
+            "tflops": tf, "tensor_frac_sustained": tf / pk["bf16_tflops_sustained"],
+            "host_link": {"h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                          "h2d_gbs": h2d / (step_ms * 1e-3) / 1e9,
+                          "d2h_gbs": d2h / (step_ms * 1e-3) / 1e9},
+            "table_bytes_host": L * V * F * 2, "setup_s": setup_s,
+            "clocks": clk.summary(c0, c1)}
+
+
 def train_flops(w):
     return 18 * w.T * w.D * w.F   # 3 forward + 6 backward GEMMs of 2*T*D*F
 
@@ -558,6 +745,9 @@ def main():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=[DEFAULT_WORKLOAD])
     ap.add_argument("--train-steps", type=int, default=200)
     ap.add_argument("--no-train", action="store_true")
+    ap.add_argument("--no-stacks", action="store_true")
+    ap.add_argument("--stack-decode-steps", type=int, default=256)
+    ap.add_argument("--stack-train-steps", type=int, default=4)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     w = syn.WORKLOADS[args.workload]
@@ -639,6 +829,17 @@ def main():
             }
         except Exception as ex:  # the decode line must still print
             line["train_layer"] = {"error": repr(ex)}
+        release_pinned()
+    if not args.no_stacks:
+        for key, fn, name, n in (("stack_decode", run_stack_decode, "olmo2-7b-decode-16l",
+                                  args.stack_decode_steps),
+                                 ("stack_train", run_stack_train, "olmo2-1b-train-12l",
+                                  args.stack_train_steps)):
+            try:
+                line[key] = fn(stp, ctx, syn.WORKLOADS[name], n, world, local)
+            except Exception as ex:  # the headline line must still print
+                line[key] = {"error": repr(ex)}
+            release_pinned()
     if world == 1 and rank == 0 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline_decode(w)
     stp.staple_context_destroy(ctx)
