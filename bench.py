@@ -574,6 +574,15 @@ def run_stack_decode(stp, ctx, w, steps, world, local):
         misses = [int(m.item()) for m in s.r.mc]
         U = int(s.r.U.item())
         s.release()
+        # a few steps outside the graph with per-launch CUDA events
+        stp.staple_trace_enable(ctx, True)
+        with torch.cuda.stream(st):
+            for k in range(4):
+                s.ids_buf.copy_(ids[k])
+                s.run(st)
+        torch.cuda.synchronize()
+        kern = kernel_table(stp.staple_trace_read(ctx), 4)
+        stp.staple_trace_enable(ctx, False)
     finally:
         tables.close()
     step_ms = ms / steps
@@ -584,7 +593,7 @@ def run_stack_decode(stp, ctx, w, steps, world, local):
             "weight_bytes_per_step": wbytes, "weight_gbs": wbytes / (step_ms * 1e-3) / 1e9,
             "table_bytes_host": L * V * F * 2, "setup_s": setup_s,
             "graph": "one CUDA graph per step: dedup, 4 group gathers on side streams, 16 layers",
-            "clocks": clk.summary(c0, c1)}
+            "clocks": clk.summary(c0, c1), "kernels_4_traced_steps": kern}
 
 
 def run_stack_train(stp, ctx, w, steps, world, local):
@@ -638,6 +647,13 @@ def run_stack_train(stp, ctx, w, steps, world, local):
         ms = max_over_ranks(ev0.elapsed_time(ev1), world)
         U = int(r.U.item())
         misses = [int(m.item()) for m in r.mc]
+        # one more step with per-launch CUDA events: the kernel list
+        stp.staple_trace_enable(ctx, True)
+        with torch.cuda.stream(st):
+            one()
+        torch.cuda.synchronize()
+        kern = kernel_table(stp.staple_trace_read(ctx), 1)
+        stp.staple_trace_enable(ctx, False)
     finally:
         tables.close()
     step_ms = ms / steps
@@ -654,7 +670,7 @@ def run_stack_train(stp, ctx, w, steps, world, local):
                           "h2d_gbs": h2d / (step_ms * 1e-3) / 1e9,
                           "d2h_gbs": d2h / (step_ms * 1e-3) / 1e9},
             "table_bytes_host": L * V * F * 2, "setup_s": setup_s,
-            "clocks": clk.summary(c0, c1)}
+            "clocks": clk.summary(c0, c1), "kernels_one_traced_step": kern}
 
 
 def train_flops(w):

@@ -60,7 +60,8 @@ def _f64b(a):
     return syn.bf16_bits_to_f32(a).astype(np.float64)
 
 
-def test_train_stack_matches_oracle_per_layer(stp, ctx):
+@pytest.mark.parametrize("de_return", ["dma", "kernel"])
+def test_train_stack_matches_oracle_per_layer(stp, ctx, de_return):
     import torch
 
     from token_indexed_sparse_staple_b200.stack import TrainStack
@@ -69,7 +70,7 @@ def test_train_stack_matches_oracle_per_layer(stp, ctx):
     freq = syn.calibration_freq(V, n_tokens=1 << 18)
     W, tables = _build(stp, ctx, layers, groups, V, F, G, freq)
     try:
-        s = TrainStack(ctx, W, tables, T, D, F, V, keep_dy=True)
+        s = TrainStack(ctx, W, tables, T, D, F, V, keep_dy=True, de_return=de_return)
         for step in range(2):       # two steps: the second finds its head prefetched
             ids = syn.zipf_ids(T, V, 1.1, seed=50 + step)
             nxt = syn.zipf_ids(T, V, 1.1, seed=51 + step)

@@ -11,8 +11,13 @@ the computation runs in the library's kernels).
   prefetch streams while earlier layers compute, and a layer waits only for
   its own group (Decode row: synchronise when a group is first consumed).
 - Training: the backward pass runs the layers in reverse.  Each layer's U
-  table-gradient rows go back to host memory (staple_embed_grad_to_host) on a
-  copy stream while the next layer's backward runs.  The next step's dedup
+  table-gradient rows go back to host memory on a copy stream while the next
+  layer's backward runs.  By default the copy engine moves exactly U rows:
+  U reaches pinned host memory right after the dedup, long before the
+  backward needs it.  SM stores over the host link (staple_embed_grad_to_host,
+  which reads U on the device and so also works inside a captured graph)
+  would occupy every SM's store path with slow posted writes and stall the
+  concurrent GEMMs' epilogues.  The next step's dedup
   and first-group gather run during this step's backward (successive batches
   are pipelined: retrieval-path table, Prefill row).  No table optimizer runs
   here, so nothing the prefetch reads changes in between.
@@ -84,6 +89,8 @@ class Retrieval:
                      for _ in range(n_groups)]
         self.ready = [torch.cuda.Event() for _ in range(n_groups)]
         self.free = torch.cuda.Event()   # recorded after the last reader of this step
+        self.U_host = torch.zeros(1, dtype=torch.int32, pin_memory=True)
+        self.U_known = torch.cuda.Event()  # U_host holds this step's U
 
     def embed(self, layer: int):
         """The embed argument of layer `layer`: its G-slice of its group's rows,
@@ -94,8 +101,12 @@ class Retrieval:
 
 
 def issue_dedup(ctx, r: Retrieval, ids, V: int, stream):
+    import torch
     stp.staple_dedup(ctx, ids, r.T, V, r.unique, r.inverse, r.seg, r.sorted_pos, r.U,
                      stream=stream)
+    with torch.cuda.stream(stream):
+        r.U_host.copy_(r.U, non_blocking=True)   # 4 bytes; read by the host much later
+    r.U_known.record(stream)
 
 
 def issue_group(ctx, r: Retrieval, tables: GroupedTables, g: int, stream, side):
@@ -132,9 +143,13 @@ class TrainStack:
     every layer returned to host memory."""
 
     def __init__(self, ctx, weights: list, tables: GroupedTables, T: int, D: int, F: int, V: int,
-                 freeze_up: bool = False, keep_dy: bool = False):
+                 freeze_up: bool = False, keep_dy: bool = False, de_return: str = "dma"):
         """keep_dy keeps every layer's incoming gradient (L buffers instead of
-        two alternating ones), so each layer can be checked on its own inputs."""
+        two alternating ones), so each layer can be checked on its own inputs.
+        de_return: "dma" (copy engine, U known on the host) or "kernel"
+        (staple_embed_grad_to_host, U read on the device)."""
+        assert de_return in ("dma", "kernel")
+        self.de_return = de_return
         import torch
         self.ctx, self.W, self.tables = ctx, weights, tables
         self.T, self.D, self.F, self.V, self.G = T, D, F, V, tables.G
@@ -208,6 +223,9 @@ class TrainStack:
             self._prefetch_head(rn, next_ids)
             self._primed = (self.step_no + 1, next_ids)
         # backward, layers in reverse
+        if self.de_return == "dma":
+            r.U_known.synchronize()               # completed long ago: the dedup ran first
+            U = int(r.U_host[0])
         dy = dy_top
         for l in reversed(range(self.L)):
             w = self.W[l]
@@ -217,8 +235,15 @@ class TrainStack:
                                  r.sorted_pos, r.inverse, r.seg, r.U, b.dgh, b.dE[k], b.ws, b.wsb,
                                  stream=st)
             self.copy.wait_stream(st)
-            stp.staple_embed_grad_to_host(self.ctx, F, T, b.dE[k], r.unique, r.U, b.host_dE[l],
-                                          b.host_unique[l], b.host_U[l], stream=self.copy)
+            if self.de_return == "dma":
+                with torch.cuda.stream(self.copy):
+                    b.host_dE[l][:U].copy_(b.dE[k][:U], non_blocking=True)
+                    b.host_unique[l][:U].copy_(r.unique[:U], non_blocking=True)
+                b.host_U[l][0] = U
+            else:
+                stp.staple_embed_grad_to_host(self.ctx, F, T, b.dE[k], r.unique, r.U,
+                                              b.host_dE[l], b.host_unique[l], b.host_U[l],
+                                              stream=self.copy)
             b.dE_copied[k].record(self.copy)
             dx = b.dy[l % len(b.dy)]   # the gradient layer l passes down (layer l-1's dy)
             dwg, dwu, dwd = b.dW[l]
