@@ -499,6 +499,29 @@ def pinned_group_tables(n_groups, G, V, F, std, seed0, chunk_rows=4096):
     return out
 
 
+def measure_host_link(nbytes=1 << 30, reps=5):
+    """Copy-engine bandwidth between pinned host memory and HBM, each way
+    (best of `reps` copies of `nbytes`, CUDA events).  The host link's peak is
+    not in the measured-peaks file, so the bench measures it here."""
+    import torch
+    h = torch.empty(nbytes, dtype=torch.uint8, pin_memory=True)
+    d = torch.empty(nbytes, dtype=torch.uint8, device="cuda")
+    out = {}
+    for name, dst, src in (("h2d_gbs", d, h), ("d2h_gbs", h, d)):
+        best = float("inf")
+        for _ in range(reps):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            dst.copy_(src, non_blocking=True)
+            e1.record()
+            torch.cuda.synchronize()
+            best = min(best, e0.elapsed_time(e1))
+        out[name] = nbytes / (best * 1e-3) / 1e9
+    del h, d
+    out["bytes"] = nbytes
+    return out
+
+
 def release_pinned():
     """Return cached page-locked host blocks to the system (torch keeps freed
     pinned blocks for reuse)."""
@@ -831,6 +854,12 @@ def main():
             tf = None
             if top[0] in gemm_flops:
                 tf = gemm_flops[top[0]] * wt.T * wt.D * wt.F / (top[1]["avg_us"] * 1e-6) / 1e12
+            link = measure_host_link()
+            k4 = kern.get("k4_gather_misses")
+            if k4:
+                zc = tr["misses"] * wt.F * 2 / (k4["avg_us"] * 1e-6) / 1e9
+                link["k4_zero_copy_gbs"] = zc
+                link["k4_frac_of_h2d"] = zc / link["h2d_gbs"]
             line["train_layer"] = {
                 "workload": wt.name, "tokens_per_s": job_value(wt.T, st_ms, world),
                 "ms_per_step": st_ms, "dense_ms_per_step": de_ms,
@@ -841,7 +870,7 @@ def main():
                              "peak": pk["bf16_tflops_sustained"], "unit": "TFLOP/s",
                              "frac": None if tf is None else tf / pk["bf16_tflops_sustained"],
                              "peak_source": pk["source"] + " (cuBLAS bf16, sustained)"},
-                "clocks": tr["staple"]["clocks"], "kernels": kern,
+                "clocks": tr["staple"]["clocks"], "kernels": kern, "host_link": link,
             }
         except Exception as ex:  # the decode line must still print
             line["train_layer"] = {"error": repr(ex)}
