@@ -74,6 +74,7 @@ struct Params {
   int32_t Ud;          // down units (Dt * ud)
   int32_t maxp_d;      // partial slots per down tile
   int32_t rcap;        // partial slices per reduction batch (ring memory / slice)
+  int32_t stage_tmem;  // stage down-unit weights in spare tensor memory
   // activations / outputs
   uint16_t* z;
   uint16_t* g_save;
@@ -190,7 +191,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int ngs = (t1 - t0) * p.ug;
   const int nsteps = ngs + (d1 - d0);
   const uint32_t ncols = p.N <= 32 ? 32 : (p.N <= 64 ? 64 : (p.N <= 128 ? 128 : 256));
-  const uint32_t tmem_cols = 2 * ncols;
+  // Tensor memory: two accumulators of ncols columns, then (p.stage_tmem) as
+  // many down-unit weight slots as fit in the 512 columns; a slot holds one
+  // unit's 128 rows x sub*64 bf16 (two k values per column).
+  const uint32_t slot_cols = uint32_t(p.sub) * (BK / 2);
+  const int nslots = p.stage_tmem ? int((512 - 2 * ncols) / slot_cols) : 0;
+  const uint32_t tmem_cols = nslots > 0 ? 512 : 2 * ncols;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
@@ -242,10 +248,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int k0 = (u * p.sub + j) * BK;
             tma_load_2d_hint(&tm_wg, &fullA[s], a + j * A_BLOCK, k0, tile * 64, once);
             tma_load_2d_hint(&tm_wu, &fullA[s], a + j * A_BLOCK + A_BLOCK / 2, k0, tile * 64, once);
-          } else {
+          } else if (j == 0) {
+            // one 3-D copy brings all `sub` k blocks of the unit
             const int x = d0 + i - ngs, tile = x / p.ud, u = x % p.ud;
-            tma_load_2d_hint(&tm_wd, &fullA[s], a + j * A_BLOCK, (u * p.sub + j) * BK, tile * BM,
-                             once);
+            tma_load_3d_hint(&tm_wd, &fullA[s], a, 0, tile * BM, u * p.sub, once);
           }
         }
         if (++s == S) {
@@ -268,8 +274,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int u = i % p.ug;
         uint8_t* b = sB + s * b_stage;
         mbar_arrive_expect_tx(&fullB[s], b_stage);
-        for (int j = 0; j < p.sub; ++j)
-          tma_load_2d(&tm_x, &fullB[s], b + j * b_block, (u * p.sub + j) * BK, 0);
+        tma_load_3d(&tm_x, &fullB[s], b, 0, 0, u * p.sub);
         if (++s == SB) {
           s = 0;
           ph ^= 1;
@@ -299,8 +304,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int u = (d0 + i - ngs) % p.ud;
         uint8_t* b = sB + s * b_stage;
         mbar_arrive_expect_tx(&fullB[s], b_stage);
-        for (int j = 0; j < p.sub; ++j)
-          tma_load_2d(&tm_z, &fullB[s], b + j * b_block, (u * p.sub + j) * BK, 0);
+        tma_load_3d(&tm_z, &fullB[s], b, 0, 0, u * p.sub);
         if (++s == SB) {
           s = 0;
           ph ^= 1;
@@ -311,11 +315,39 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       // ---------------------------------------------------------------- MMA
       const uint32_t idesc = idesc_bf16_f32(BM, p.N, false, false);
+      const uint32_t slot0 = tmem_base + 2 * ncols;  // first tensor-memory staging column
+      const int n_stage = min(d1 - d0, nslots);
       int sa = 0, sb = 0;
       uint32_t pha = 0, phb = 0;
       int piece = 0;
       bool ok = true;
       for (int i0 = 0; i0 < nsteps && ok; ++piece) {
+        if (i0 == ngs && n_stage > 0) {
+          // The first n_stage down units' weights move to tensor memory as
+          // they land; each copy's commit frees its ring stage for the next
+          // unit's weights, so W_down streams while z is still being made.
+          for (int k = 0; k < n_stage; ++k) {
+            if (!mbar_wait(&fullA[sa], pha, abort_flag, p.err)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint32_t a_addr = smem_u32(sA + sa * a_stage);
+            const uint32_t dst = slot0 + uint32_t(k) * slot_cols;
+            for (int j = 0; j < p.sub; ++j) {
+#pragma unroll
+              for (int kk = 0; kk < BK / 16; ++kk)
+                tmem_cp_128x256b(dst + uint32_t(j * (BK / 16) + kk) * 8,
+                                 sw128_desc(a_addr + j * A_BLOCK + kk * 32, 16, 1024));
+            }
+            umma_commit(&emptyA[sa]);
+            if (++sa == S) {
+              sa = 0;
+              pha ^= 1;
+            }
+          }
+          if (!ok) break;
+        }
         int nunits;
         if (i0 < ngs) {
           nunits = p.ug;
@@ -328,27 +360,51 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         const uint32_t dacc = tmem_base + uint32_t(buf) * ncols;
         for (int i = 0; i < nunits; ++i) {
-          if (!mbar_wait(&fullA[sa], pha, abort_flag, p.err) ||
+          const int du = i0 + i - ngs;  // down unit index (negative for gate/up)
+          const bool staged = du >= 0 && du < n_stage;
+          if ((!staged && !mbar_wait(&fullA[sa], pha, abort_flag, p.err)) ||
               !mbar_wait(&fullB[sb], phb, abort_flag, p.err)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint32_t a_addr = smem_u32(sA + sa * a_stage);
-          const uint32_t b_addr = smem_u32(sB + sb * b_stage);
-          for (int j = 0; j < p.sub; ++j) {
+          // Descriptors are built once per unit; a k step of 32 bytes adds 2
+          // to the start-address field (shared addresses stay below 2^18, so
+          // the field never carries).  At decode sizes each MMA is small and
+          // the issuing thread's own instructions set the pace.
+          const uint64_t bd = sw128_desc(smem_u32(sB + sb * b_stage), 16, 1024);
+          const uint32_t acc0 = i != 0 ? 1u : 0u;
+          if (staged) {
+            const uint32_t a_t = slot0 + uint32_t(du) * slot_cols;
 #pragma unroll
-            for (int k = 0; k < BK / 16; ++k)
-              umma_bf16(dacc, sw128_desc(a_addr + j * A_BLOCK + k * 32, 16, 1024),
-                        sw128_desc(b_addr + j * b_block + k * 32, 16, 1024), idesc,
-                        (i | j | k) != 0 ? 1u : 0u);
+            for (int j = 0; j < 2; ++j) {
+              if (j < p.sub) {
+#pragma unroll
+                for (int k = 0; k < BK / 16; ++k)
+                  umma_bf16_ta(dacc, a_t + uint32_t(j * (BK / 16) + k) * 8,
+                               bd + uint64_t((j * b_block + k * 32) >> 4), idesc,
+                               (j | k) != 0 ? 1u : acc0);
+              }
+            }
+          } else {
+            const uint64_t ad = sw128_desc(smem_u32(sA + sa * a_stage), 16, 1024);
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+              if (j < p.sub) {
+#pragma unroll
+                for (int k = 0; k < BK / 16; ++k)
+                  umma_bf16(dacc, ad + uint64_t((j * A_BLOCK + k * 32) >> 4),
+                            bd + uint64_t((j * b_block + k * 32) >> 4), idesc,
+                            (j | k) != 0 ? 1u : acc0);
+              }
+            }
+            umma_commit(&emptyA[sa]);
+            if (++sa == S) {
+              sa = 0;
+              pha ^= 1;
+            }
           }
-          umma_commit(&emptyA[sa]);
           umma_commit(&emptyB[sb]);
-          if (++sa == S) {
-            sa = 0;
-            pha ^= 1;
-          }
           if (++sb == SB) {
             sb = 0;
             phb ^= 1;

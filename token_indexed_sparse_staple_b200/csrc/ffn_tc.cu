@@ -66,6 +66,23 @@ bool make_map_f32(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// K-major bf16 operand [rows][k] seen as 3-D: (k within a 64-wide block,
+// row, block).  A box of `depth` blocks lands in shared memory as `depth`
+// consecutive [box_rows][64] 128-byte-swizzled tiles, so one copy fetches
+// what `depth` 2-D copies would.
+bool kmajor_blocks(CUtensorMap* m, const void* base, int rows, int k, int64_t ld, int box_rows,
+                   int depth) {
+  auto enc = encoder();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {uint64_t(tc::BK), uint64_t(rows), uint64_t(k / tc::BK)};
+  cuuint64_t strides[2] = {uint64_t(ld) * 2, uint64_t(tc::BK) * 2};
+  cuuint32_t box[3] = {uint32_t(tc::BK), uint32_t(box_rows), uint32_t(depth)};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
+             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // K-major operand [rows][k]: box 64 (k) x 128 (rows).
 bool kmajor(CUtensorMap* m, const void* base, int rows, int k, int64_t ld) {
   return make_map(m, base, uint64_t(k), uint64_t(rows), uint64_t(ld), tc::BK, 128);
@@ -165,8 +182,8 @@ staple_status tc_decode_fwd(const DeviceInfo& di, int T, int D, int F, const voi
   void* part = static_cast<uint8_t*>(ws) + pl.counter_bytes;
   CUtensorMap mg, mu, md, mx, mz, mp;
   if (!kmajor_rows(&mg, wg, F, D, D, 64) || !kmajor_rows(&mu, wu, F, D, D, 64) ||
-      !kmajor_rows(&md, wd, D, F, F, fused::BM) || !kmajor_rows(&mx, x, T, D, D, pl.N) ||
-      !kmajor_rows(&mz, z, T, F, F, pl.N) ||
+      !kmajor_blocks(&md, wd, D, F, F, fused::BM, pl.sub) ||
+      !kmajor_blocks(&mx, x, T, D, D, pl.N, pl.sub) || !kmajor_blocks(&mz, z, T, F, F, pl.N, pl.sub) ||
       // partial slots [Dt * maxp_d * N][128] fp32; a box is one piece's
       // 16-row slice for all N tokens
       !make_map_f32(&mp, part, fused::BM, uint64_t(pl.Dt) * pl.maxp_d * pl.N, fused::BM,
@@ -187,6 +204,7 @@ staple_status tc_decode_fwd(const DeviceInfo& di, int T, int D, int F, const voi
   p.Ud = pl.Ud;
   p.maxp_d = pl.maxp_d;
   p.rcap = fused::reduce_slices(pl.N, pl.sub);
+  p.stage_tmem = 1;
   p.z = static_cast<uint16_t*>(z);
   p.g_save = static_cast<uint16_t*>(g_save);
   p.h_save = static_cast<uint16_t*>(h_save);
