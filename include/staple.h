@@ -257,6 +257,23 @@ staple_status staple_embed_bwd(staple_context* ctx, staple_dtype dtype, int32_t 
                                const int32_t* U_dev, void* dgh, float* dE, void* workspace,
                                size_t workspace_bytes, staple_stream stream);
 
+/* The table-gradient half of staple_embed_bwd on its own: dE from a dh that
+ * staple_embed_bwd (called with dE == NULL) left in dgh, so that the
+ * reduction can run on another stream, next to the rest of the backward pass.
+ *   dh          device, T rows of F values (dtype), row pitch ld elements
+ *               (the dh half of dgh: dgh + F elements, ld = 2F)
+ *   sorted_pos, inverse, seg_off, U_dev   from staple_dedup for the same ids
+ *   dE          out, fp32 [>= U][F]; rows >= U untouched
+ *   workspace   as for staple_embed_bwd (staple_workspace_bytes(T, D, F)
+ *               bytes; its head is left untouched).  Two calls that overlap
+ *               on the GPU need two workspaces.
+ * Same result, bit for bit, as the reduction inside staple_embed_bwd. */
+staple_status staple_embed_grad(staple_context* ctx, staple_dtype dtype, int32_t T, int32_t D,
+                                int32_t F, const void* dh, int64_t ld, const int32_t* sorted_pos,
+                                const int32_t* inverse, const int32_t* seg_off,
+                                const int32_t* U_dev, float* dE, void* workspace,
+                                size_t workspace_bytes, staple_stream stream);
+
 /* Return one layer's table gradient to host memory, where the tables and
  * their optimizer live (the pages keep the tables in host DRAM and
  * materialise only the U active rows of a batch: AI Radio episode, paper

@@ -211,3 +211,41 @@ def test_olmo2_1b_decode_layer_full_size(stp, ctx):
     E_rows = syn.bf16_bits_to_f32(inp.table[inp.ids]).astype(np.float64)
     ref = oracle.ffn_forward(x, np.arange(w.T), wg, wu, wd, E_rows)
     compare(got, ref, TOL["bf16"], FWD)
+
+
+def test_split_table_gradient_matches_fused(stp, ctx):
+    """staple_embed_bwd with dE == NULL, then staple_embed_grad on another
+    stream, gives the dE of the fused call bit for bit."""
+    import torch
+    T, D, F, V = 3000, 128, 512, 5000
+    g = torch.Generator(device="cuda")
+    g.manual_seed(21)
+
+    def rnd(*shape, std=1.0):
+        return (torch.randn(shape, generator=g, device="cuda") * std).to(torch.bfloat16)
+
+    ids = torch.from_numpy(syn.zipf_ids(T, V, 1.1, seed=21)).cuda()
+    i32 = dict(dtype=torch.int32, device="cuda")
+    unique, inverse, sorted_pos = (torch.empty(T, **i32) for _ in range(3))
+    seg, U = torch.empty(T + 1, **i32), torch.empty(1, **i32)
+    stp.staple_dedup(ctx, ids, T, V, unique, inverse, seg, sorted_pos, U)
+    dy, gs, hs, wd = rnd(T, D), rnd(T, F), rnd(T, F), rnd(D, F, std=0.05)
+    wsb = stp.staple_workspace_bytes(T, D, F)
+    ws = torch.zeros(wsb, dtype=torch.uint8, device="cuda")
+    dgh = torch.empty((T, 2 * F), dtype=torch.bfloat16, device="cuda")
+    ref = torch.zeros((T, F), dtype=torch.float32, device="cuda")
+    stp.staple_embed_bwd(ctx, stp.STAPLE_BF16, T, D, F, dy, gs, hs, wd, sorted_pos, inverse, seg, U,
+                         dgh, ref, ws, wsb)
+    dgh2 = torch.empty_like(dgh)
+    got = torch.zeros_like(ref)
+    stp.staple_embed_bwd(ctx, stp.STAPLE_BF16, T, D, F, dy, gs, hs, wd, sorted_pos, inverse, seg, U,
+                         dgh2, None, ws, wsb)
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    stp.staple_embed_grad(ctx, stp.STAPLE_BF16, T, D, F, dgh2.data_ptr() + F * 2, 2 * F,
+                          sorted_pos, inverse, seg, U, got, ws, wsb, stream=side)
+    torch.cuda.synchronize()
+    assert stp.staple_get_error(ctx) == 0
+    assert torch.equal(dgh, dgh2)
+    u = int(U.item())
+    assert torch.equal(got[:u], ref[:u])

@@ -201,6 +201,14 @@ def staple_embed_bwd(ctx, dtype, T, D, F, dy, g_save, h_save, w_down, sorted_pos
         "staple_embed_bwd")
 
 
+def staple_embed_grad(ctx, dtype, T, D, F, dh, ld, sorted_pos, inverse, seg_off, U_dev, dE,
+                      workspace, workspace_bytes, stream=None):
+    """The table-gradient reduction alone (see include/staple.h)."""
+    _ok(lib().staple_embed_grad(ctx, dtype, T, D, F, _p(dh), ld, _p(sorted_pos), _p(inverse),
+                                _p(seg_off), _p(U_dev), _p(dE), _p(workspace), workspace_bytes,
+                                _stream(stream)), "staple_embed_grad")
+
+
 def staple_embed_grad_to_host(ctx, F, capacity, dE, unique, U_dev, host_dE, host_unique, host_U,
                               stream=None):
     """Rows [0, U) of dE and the U ids to page-locked, mapped host buffers

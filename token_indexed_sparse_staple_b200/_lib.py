@@ -56,6 +56,8 @@ SIGNATURES = {
     "staple_ffn_bwd": (c_status, [vp, C.c_int, i32, i32, i32, vp, vp, vp, vp, vp, vp, vp, vp,
                                   vp, vp, vp, sz, vp]),
     "staple_embed_grad_to_host": (c_status, [vp, i32, i32, vp, vp, vp, vp, vp, vp, vp]),
+    "staple_embed_grad": (c_status, [vp, C.c_int, i32, i32, i32, vp, i64, vp, vp, vp, vp, vp, vp,
+                                     sz, vp]),
     "staple_embed_grad_static": (c_status, [C.c_int, i32, i32, vp, i64, vp, vp, vp, vp, vp]),
 }
 

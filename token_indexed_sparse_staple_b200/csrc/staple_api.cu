@@ -458,6 +458,29 @@ staple_status staple_embed_bwd(staple_context* ctx, staple_dtype dtype, int32_t 
                                 st);
 }
 
+staple_status staple_embed_grad(staple_context* ctx, staple_dtype dtype, int32_t T, int32_t D,
+                                int32_t F, const void* dh, int64_t ld, const int32_t* sorted_pos,
+                                const int32_t* inverse, const int32_t* seg_off,
+                                const int32_t* U_dev, float* dE, void* workspace,
+                                size_t workspace_bytes, staple_stream stream) {
+  if (!ctx) return STAPLE_EINVAL;
+  STP_TRY(check_dims(dtype, T, D, F));
+  if (T == 0) return STAPLE_OK;
+  if (!dh || ld < F || !sorted_pos || !inverse || !seg_off || !U_dev || !dE || !aligned16(dE) ||
+      !aligned16(dh) || (ld * int64_t(esize(dtype))) % 16)
+    return STAPLE_EINVAL;
+  const size_t head = stp::decode_counter_bytes(D, F);  // left untouched
+  if (!workspace || workspace_bytes < head + stp::seg_reduce_workspace(T, F) ||
+      !aligned16(workspace))
+    return STAPLE_EINVAL;
+  STP_TRY(set_device(ctx));
+  stp::TraceScope trace_scope(ctx->tracer);
+  return stp::launch_seg_reduce(dtype == STAPLE_BF16, dh, ld, sorted_pos, inverse, seg_off, U_dev,
+                                T, F, dE,
+                                reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + head),
+                                cs(stream));
+}
+
 staple_status staple_embed_grad_to_host(staple_context* ctx, int32_t F, int32_t capacity,
                                         const float* dE, const int32_t* unique,
                                         const int32_t* U_dev, float* host_dE,
