@@ -92,19 +92,25 @@ __device__ __forceinline__ void store_bf16x32(uint16_t* dst, const float* v) {
   }
 }
 
-__device__ __forceinline__ void load_bf16x32(const uint16_t* src, float* v) {
+// 32 bf16 values as four 16-byte words: the loads are issued here and only
+// waited for where the words are first used, so a chunk's loads can be in
+// flight while the previous chunk is computed.
+__device__ __forceinline__ void load_raw32(const uint16_t* src, uint4 (&w)[4]) {
   const uint4* s = reinterpret_cast<const uint4*>(src);
 #pragma unroll
+  for (int i = 0; i < 4; ++i) w[i] = __ldg(s + i);
+}
+__device__ __forceinline__ void unpack32(const uint4 (&w)[4], float* v) {
+#pragma unroll
   for (int i = 0; i < 4; ++i) {
-    const uint4 w = __ldg(s + i);
-    v[8 * i + 0] = bf_lo(w.x);
-    v[8 * i + 1] = bf_hi(w.x);
-    v[8 * i + 2] = bf_lo(w.y);
-    v[8 * i + 3] = bf_hi(w.y);
-    v[8 * i + 4] = bf_lo(w.z);
-    v[8 * i + 5] = bf_hi(w.z);
-    v[8 * i + 6] = bf_lo(w.w);
-    v[8 * i + 7] = bf_hi(w.w);
+    v[8 * i + 0] = bf_lo(w[i].x);
+    v[8 * i + 1] = bf_hi(w[i].x);
+    v[8 * i + 2] = bf_lo(w[i].y);
+    v[8 * i + 3] = bf_hi(w[i].y);
+    v[8 * i + 4] = bf_lo(w[i].z);
+    v[8 * i + 5] = bf_hi(w[i].z);
+    v[8 * i + 6] = bf_lo(w[i].w);
+    v[8 * i + 7] = bf_hi(w[i].w);
   }
 }
 
@@ -147,22 +153,24 @@ __device__ __forceinline__ void epilogue_tile(const Params& p, uint32_t tacc, in
       }
     }
     const int f0 = nb * (BN / 2);
+    // the E row's chunk c+1 is loaded while chunk c is computed
+    uint4 ew[4] = {};
+    if (erow && row_ok && f0 < p.N) load_raw32(erow + f0, ew);
 #pragma unroll 1
     for (int c = 0; c < BN / 64; ++c) {
+      uint4 ec[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) ec[i] = ew[i];
+      const int f = f0 + c * 32;
+      if (erow && row_ok && c + 1 < BN / 64 && f + 32 < p.N) load_raw32(erow + f + 32, ew);
       uint32_t rg[32], ru[32];
       tmem_ld32(tacc + c * 32, rg);
       tmem_ld32(tacc + BN / 2 + c * 32, ru);
       tmem_ld_wait(rg);
       reg_fence(ru);
-      const int f = f0 + c * 32;
       if (row_ok && f < p.N) {
         float e[32];
-        if (erow) {
-          load_bf16x32(erow + f, e);
-        } else {
-#pragma unroll
-          for (int i = 0; i < 32; ++i) e[i] = 0.0f;
-        }
+        unpack32(ec, e);   // zeros when the layer has no table
         float g[32], h[32], z[32];
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
@@ -177,17 +185,34 @@ __device__ __forceinline__ void epilogue_tile(const Params& p, uint32_t tacc, in
       }
     }
   } else {  // EPI_DZ: accumulator = dz for features [nb*256, nb*256 + 256)
+    // g and h of chunk c+1 are loaded while chunk c is computed
+    const int64_t row_off = int64_t(m) * p.ldf + nb * BN;
+    uint4 gw[4], hw[4];
+    if (row_ok && nb * BN < p.N) {
+      load_raw32(p.g_in + row_off, gw);
+      load_raw32(p.h_in + row_off, hw);
+    }
 #pragma unroll 1
     for (int c = 0; c < BN / 32; ++c) {
+      const int f = nb * BN + c * 32;
+      uint4 gc[4], hc[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        gc[i] = gw[i];
+        hc[i] = hw[i];
+      }
+      if (row_ok && c + 1 < BN / 32 && f + 32 < p.N) {
+        load_raw32(p.g_in + row_off + (c + 1) * 32, gw);
+        load_raw32(p.h_in + row_off + (c + 1) * 32, hw);
+      }
       uint32_t r[32];
       tmem_ld32(tacc + c * 32, r);
       tmem_ld_wait(r);
-      const int f = nb * BN + c * 32;
       if (row_ok && f < p.N) {
         const int64_t off = int64_t(m) * p.ldf + f;
         float g[32], h[32], dg[32], dh[32];
-        load_bf16x32(p.g_in + off, g);
-        load_bf16x32(p.h_in + off, h);
+        unpack32(gc, g);
+        unpack32(hc, h);
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
           const float dz = __uint_as_float(r[i]);
