@@ -168,10 +168,10 @@ class Clocks:
 # to the captured value; otherwise the roofline's traffic is null.
 CAPTURED_TRAFFIC = {
     "k5k6_decode_fused": {
-        "bytes": 104_795_008,   # mean of two launches: 104,419,840 and 105,170,176
+        "bytes": 104_721_408,   # mean of two launches: 104,783,872 and 104,658,944
         "sources": ["token_indexed_sparse_staple_b200/csrc/decode_fused.cuh",
                     "token_indexed_sparse_staple_b200/csrc/common.cuh"],
-        "sha256": "ec425cc20cbff1a5e5b33be8d745bdb6ebf5816610cdc65a3906bc5acb7c4d0e",
+        "sha256": "01df376535cba85dbc3dad45f100bc7d9d57c38a0cb88ba34030a39c14b15db6",
         "profile": "profiles/decode_fused_olmo2_1b_T64.md",
     },
 }
