@@ -171,7 +171,7 @@ CAPTURED_TRAFFIC = {
         "bytes": 104_721_408,   # mean of two launches: 104,783,872 and 104,658,944
         "sources": ["token_indexed_sparse_staple_b200/csrc/decode_fused.cuh",
                     "token_indexed_sparse_staple_b200/csrc/common.cuh"],
-        "sha256": "01df376535cba85dbc3dad45f100bc7d9d57c38a0cb88ba34030a39c14b15db6",
+        "sha256": "17197f137ce9eb2a844d325527441d831dcc9a9b7022cff282f4428deceb022b",
         "profile": "profiles/decode_fused_olmo2_1b_T64.md",
     },
 }

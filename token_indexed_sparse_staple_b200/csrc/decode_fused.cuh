@@ -14,18 +14,22 @@
 //    ring is deep (HBM latency), the activation ring shallow (it hits L2).
 //  * Phase 1, gate/up: whole tiles are spread over the blocks.  A block
 //    finishes a tile straight from tensor memory, 16 tokens at a time: g and
-//    u rows go to shared memory, then all 128 epilogue threads compute
-//    h = u + E[id_t][f] (E rows prefetched into shared memory during the main
-//    loop), z = SiLU(g) h (g and h saved when asked) over consecutive
-//    features, and the tile's ready flag goes up.  (A compact loop: the
-//    epilogue runs while every SM's memory queues are full, where a large
-//    unrolled body stalls on instruction fetch.)
+//    u rows go to shared memory, then each of the 128 epilogue threads
+//    computes 8 consecutive features of one token, h = u + E[id_t][f] (E rows
+//    prefetched into shared memory during the main loop) and z = SiLU(g) h
+//    (g and h saved when asked), written 16 bytes at a time; then the
+//    tile's ready flag goes up.
 //  * Phase 2, down: the down units (tile x `sub` k blocks) are split evenly
 //    over the blocks (stream-K), so every SM streams the same share of
-//    W_down.  The activation loads wait (bounded spin, all flags of the
-//    block polled at once by one warp) on the ready flags of the gate/up
-//    tiles that produced the block's z columns; weight loads do not wait.  Each block's piece of a tile leaves an fp32 partial
-//    in the workspace (L2-resident) and bumps the tile's counter.
+//    W_down.  The first units' weights are copied from the ring into the
+//    tensor-memory columns the accumulators leave free as soon as they land,
+//    which frees the ring for the next units: W_down streams while the
+//    gate/up phase is still finishing.  The activation loads wait (bounded
+//    spin, all flags of the block polled at once by one warp) on the ready
+//    flags of the gate/up tiles that produced the block's z columns; weight
+//    loads do not wait.  Each block's piece of a tile leaves an fp32 partial
+//    [N][128] in the workspace (L2-resident; a warp writes 128 contiguous
+//    bytes per token) and bumps the tile's counter.
 //  * The down sums are spread over all blocks: once a block has finished its
 //    own pieces, its epilogue warps take 16-row chunks from an atomic work
 //    queue, wait (bounded) until the chunk's tile is complete, bring every
