@@ -92,9 +92,27 @@ bool mnmajor(CUtensorMap* m, const void* base, int k, int mn, int64_t ld) {
   return make_map(m, base, uint64_t(mn), uint64_t(k), uint64_t(ld), 64, tc::BK);
 }
 
+// Output map for the staged epilogue stores: bf16 [rows][cols] with leading
+// dimension ld, box 32 x 32, 64-byte swizzle (the layout write_row_sw64
+// stages).
+bool out_map(CUtensorMap* m, const void* base, int rows, int cols, int64_t ld) {
+  auto enc = encoder();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {uint64_t(cols), uint64_t(rows)};
+  cuuint64_t strides[1] = {uint64_t(ld) * 2};
+  cuuint32_t box[2] = {32, 32};
+  cuuint32_t estr[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// o: the three output maps of a staged epilogue (EPI_GATEUP: z, g, h;
+// EPI_DZ: dg, dh), NULL for the other epilogues.
 template <bool A_MN, bool B_MN, int BSRC, int EPI>
 staple_status launch(const char* name, const DeviceInfo& di, const CUtensorMap& a,
-                     const CUtensorMap& b0, const CUtensorMap& b1, tc::Params p, cudaStream_t st) {
+                     const CUtensorMap& b0, const CUtensorMap& b1, tc::Params p, cudaStream_t st,
+                     const CUtensorMap* o = nullptr) {
   p.k_blocks = (p.K + tc::BK - 1) / tc::BK;
   const int ntiles = p.tiles_m * p.tiles_n;
   if (ntiles == 0) return STAPLE_OK;
@@ -106,12 +124,16 @@ staple_status launch(const char* name, const DeviceInfo& di, const CUtensorMap& 
   const uint64_t bit = uint64_t(1) << (di.device & 63);
   if (!(attr_done.load() & bit)) {
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             tc::kSmemBytes) != cudaSuccess)
+                             tc::smem_bytes<EPI>()) != cudaSuccess)
       return STAPLE_ECUDA;
     attr_done.fetch_or(bit);
   }
   const int grid = std::min(ntiles, di.num_sms);
-  STP_LAUNCH(name, st, kern<<<grid, tc::kThreads, tc::kSmemBytes, st>>>(a, b0, b1, p));
+  const CUtensorMap& o0 = o ? o[0] : a;
+  const CUtensorMap& o1 = o ? o[1] : a;
+  const CUtensorMap& o2 = o ? o[2] : a;
+  STP_LAUNCH(name, st,
+             kern<<<grid, tc::kThreads, tc::smem_bytes<EPI>(), st>>>(a, b0, b1, o0, o1, o2, p));
   return cudaGetLastError() == cudaSuccess ? STAPLE_OK : STAPLE_ECUDA;
 }
 
@@ -275,7 +297,12 @@ staple_status tc_ffn_fwd(const DeviceInfo& di, int T, int D, int F, const void* 
       p.e_rows = e->n_rows;
     }
     p.err = err;
-    staple_status s = launch<false, false, tc::B_NHALF, tc::EPI_GATEUP>("k5_gateup", di, mx, mg, mu, p, st);
+    CUtensorMap mo[3];
+    if (!out_map(&mo[0], z, T, F, F) || !out_map(&mo[1], g_save ? g_save : z, T, F, F) ||
+        !out_map(&mo[2], h_save ? h_save : z, T, F, F))
+      return STAPLE_ECUDA;
+    staple_status s =
+        launch<false, false, tc::B_NHALF, tc::EPI_GATEUP>("k5_gateup", di, mx, mg, mu, p, st, mo);
     if (s != STAPLE_OK) return s;
   }
   tc::Params q{};
@@ -308,7 +335,13 @@ staple_status tc_dz(const DeviceInfo& di, int T, int D, int F, const void* dy, c
   p.h_in = static_cast<const uint16_t*>(h_save);
   p.dgh = static_cast<uint16_t*>(dgh);
   p.err = err;
-  return launch<false, true, tc::B_ONE, tc::EPI_DZ>("k7_dz", di, mdy, mwd, mwd, p, st);
+  // dg = columns [0, F) of dgh, dh = [F, 2F): two maps of F columns, row pitch 2F
+  CUtensorMap mo[3];
+  if (!out_map(&mo[0], dgh, T, F, 2 * int64_t(F)) ||
+      !out_map(&mo[1], static_cast<uint16_t*>(dgh) + F, T, F, 2 * int64_t(F)))
+    return STAPLE_ECUDA;
+  mo[2] = mo[1];
+  return launch<false, true, tc::B_ONE, tc::EPI_DZ>("k7_dz", di, mdy, mwd, mwd, p, st, mo);
 }
 
 staple_status tc_ffn_bwd(const DeviceInfo& di, int T, int D, int F, const void* dy,

@@ -39,6 +39,16 @@ constexpr int kSmemBytes = STAGES * STAGE_BYTES + 1024 /*align*/ + 256 /*barrier
 enum BSrc { B_ONE = 0, B_NHALF = 1, B_KSPLIT = 2 };
 enum Epi { EPI_BF16 = 0, EPI_F32 = 1, EPI_GATEUP = 2, EPI_DZ = 3 };
 
+// The heavy epilogues stage every 32-row x 32-column output block of a warp
+// in shared memory (64-byte swizzle) and write it with one TMA store: a
+// thread holds one accumulator row, so its own stores would each touch a
+// different row.  2 KB per block: z, g, h for EPI_GATEUP; dg, dh for EPI_DZ.
+constexpr int kOutBox = 32 * 32 * 2;
+template <int EPI>
+constexpr int out_blocks() { return EPI == EPI_GATEUP ? 3 : (EPI == EPI_DZ ? 2 : 0); }
+template <int EPI>
+constexpr int smem_bytes() { return kSmemBytes + 4 * out_blocks<EPI>() * kOutBox; }
+
 struct Params {
   int32_t M, N, K;            // output rows, output columns (features for GATEUP / DZ), K
   int32_t tiles_m, tiles_n, k_blocks;
@@ -114,9 +124,51 @@ __device__ __forceinline__ void unpack32(const uint4 (&w)[4], float* v) {
   }
 }
 
+// Row r (32 bf16 values) of a 32 x 32 block in the 64-byte-swizzled layout
+// the TMA store reads: 16-byte chunk k of row r sits at chunk k ^ ((r/2) % 4).
+__device__ __forceinline__ void write_row_sw64(uint8_t* box, int r, const float* v) {
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    uint4 w;
+    w.x = pack_bf2(v[8 * k + 0], v[8 * k + 1]);
+    w.y = pack_bf2(v[8 * k + 2], v[8 * k + 3]);
+    w.z = pack_bf2(v[8 * k + 4], v[8 * k + 5]);
+    w.w = pack_bf2(v[8 * k + 6], v[8 * k + 7]);
+    *reinterpret_cast<uint4*>(box + r * 64 + ((k ^ ((r >> 1) & 3)) << 4)) = w;
+  }
+}
+
+// Tensor maps the staged output blocks are stored through (box 32 x 32).
+struct OutMaps {
+  const CUtensorMap* m[3];
+};
+
+// Lane 0 waits until the warp's previous block stores have read the staging
+// buffer; then the whole warp may write it again.
+__device__ __forceinline__ void stage_begin(int lane) {
+  if (lane == 0) bulk_wait_read0();
+  __syncwarp();
+}
+// Make the staged rows visible to TMA, then lane 0 stores the n blocks.
+__device__ __forceinline__ void stage_store(int lane, uint8_t* stg, const OutMaps& om,
+                                            const bool (&use)[3], int col, int row0) {
+  fence_async_smem();
+  __syncwarp();
+  if (lane == 0) {
+#pragma unroll
+    for (int b = 0; b < 3; ++b)
+      if (use[b]) tma_store_2d(om.m[b], stg + b * kOutBox, col, row0);
+    bulk_commit();
+  }
+}
+
+// m = this thread's accumulator row; lane = m % 32; stg = the warp's staging
+// blocks (EPI_GATEUP, EPI_DZ).
 template <int EPI>
-__device__ __forceinline__ void epilogue_tile(const Params& p, uint32_t tacc, int m, int nb) {
+__device__ __forceinline__ void epilogue_tile(const Params& p, uint32_t tacc, int m, int nb,
+                                              int lane, uint8_t* stg, const OutMaps& om) {
   const bool row_ok = m < p.M;
+  const int m0w = m - lane;   // the warp's first row
   if constexpr (EPI == EPI_BF16 || EPI == EPI_F32) {
 #pragma unroll 1
     for (int c = 0; c < BN / 32; ++c) {
@@ -168,7 +220,8 @@ __device__ __forceinline__ void epilogue_tile(const Params& p, uint32_t tacc, in
       tmem_ld32(tacc + BN / 2 + c * 32, ru);
       tmem_ld_wait(rg);
       reg_fence(ru);
-      if (row_ok && f < p.N) {
+      if (f < p.N) {   // the same for the whole warp
+        // rows past M are staged too; the TMA store leaves them out
         float e[32];
         unpack32(ec, e);   // zeros when the layer has no table
         float g[32], h[32], z[32];
@@ -178,16 +231,18 @@ __device__ __forceinline__ void epilogue_tile(const Params& p, uint32_t tacc, in
           h[i] = __uint_as_float(ru[i]) + e[i];
           z[i] = g[i] * sigmoid_f(g[i]) * h[i];
         }
-        const int64_t off = int64_t(m) * p.ldf + f;
-        store_bf16x32(p.z + off, z);
-        if (p.g_save) store_bf16x32(p.g_save + off, g);
-        if (p.h_save) store_bf16x32(p.h_save + off, h);
+        const bool use[3] = {true, p.g_save != nullptr, p.h_save != nullptr};
+        stage_begin(lane);
+        write_row_sw64(stg, lane, z);
+        if (use[1]) write_row_sw64(stg + kOutBox, lane, g);
+        if (use[2]) write_row_sw64(stg + 2 * kOutBox, lane, h);
+        stage_store(lane, stg, om, use, f, m0w);
       }
     }
   } else {  // EPI_DZ: accumulator = dz for features [nb*256, nb*256 + 256)
     // g and h of chunk c+1 are loaded while chunk c is computed
     const int64_t row_off = int64_t(m) * p.ldf + nb * BN;
-    uint4 gw[4], hw[4];
+    uint4 gw[4] = {}, hw[4] = {};
     if (row_ok && nb * BN < p.N) {
       load_raw32(p.g_in + row_off, gw);
       load_raw32(p.h_in + row_off, hw);
@@ -208,10 +263,9 @@ __device__ __forceinline__ void epilogue_tile(const Params& p, uint32_t tacc, in
       uint32_t r[32];
       tmem_ld32(tacc + c * 32, r);
       tmem_ld_wait(r);
-      if (row_ok && f < p.N) {
-        const int64_t off = int64_t(m) * p.ldf + f;
+      if (f < p.N) {   // the same for the whole warp
         float g[32], h[32], dg[32], dh[32];
-        unpack32(gc, g);
+        unpack32(gc, g);   // zeros for rows past M (staged, never stored)
         unpack32(hc, h);
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
@@ -220,9 +274,11 @@ __device__ __forceinline__ void epilogue_tile(const Params& p, uint32_t tacc, in
           dh[i] = dz * g[i] * s;
           dg[i] = dz * h[i] * (s * (1.0f + g[i] * (1.0f - s)));
         }
-        uint16_t* row = p.dgh + int64_t(m) * (2 * p.ldf);
-        store_bf16x32(row + f, dg);
-        store_bf16x32(row + p.ldf + f, dh);
+        const bool use[3] = {true, true, false};
+        stage_begin(lane);
+        write_row_sw64(stg, lane, dg);
+        write_row_sw64(stg + kOutBox, lane, dh);
+        stage_store(lane, stg, om, use, f, m0w);
       }
     }
   }
@@ -234,12 +290,15 @@ __device__ __forceinline__ void epilogue_tile(const Params& p, uint32_t tacc, in
 template <bool A_MN, bool B_MN, int BSRC, int EPI>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB0,
-                const __grid_constant__ CUtensorMap tmB1, const Params p) {
+                const __grid_constant__ CUtensorMap tmB1, const __grid_constant__ CUtensorMap tmO0,
+                const __grid_constant__ CUtensorMap tmO1, const __grid_constant__ CUtensorMap tmO2,
+                const Params p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align_smem_1024(smem_raw);
   uint8_t* sA = smem;
   uint8_t* sB = smem + STAGES * A_STAGE;
-  uint64_t* full = reinterpret_cast<uint64_t*>(sB + STAGES * B_STAGE);
+  uint8_t* s_out = sB + STAGES * B_STAGE;  // [4 warps][out_blocks][32][32] bf16, swizzled
+  uint64_t* full = reinterpret_cast<uint64_t*>(s_out + 4 * out_blocks<EPI>() * kOutBox);
   uint64_t* empty = full + STAGES;
   uint64_t* tfull = empty + STAGES;
   uint64_t* tempty = tfull + 2;
@@ -385,6 +444,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     // -------------------------------------------------------------- epilogue
     const int q = warp & 3;
     const int row = q * 32 + lane;
+    uint8_t* stg = s_out + q * out_blocks<EPI>() * kOutBox;
+    const OutMaps om{{&tmO0, &tmO1, &tmO2}};
     int iter = 0;
     for (int t = blockIdx.x; t < ntiles; t += gridDim.x, ++iter) {
       const int buf = iter & 1;
@@ -395,11 +456,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!__all_sync(0xffffffffu, ok)) break;
       tc_fence_after();
       const uint32_t tacc = tmem_base + (uint32_t(q * 32) << 16) + uint32_t(buf * BN);
-      epilogue_tile<EPI>(p, tacc, mb * BM + row, nb);
+      epilogue_tile<EPI>(p, tacc, mb * BM + row, nb, lane, stg, om);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&tempty[buf]);
     }
+    // the block's last staged stores must finish before its shared memory goes
+    if (out_blocks<EPI>() > 0 && lane == 0) bulk_wait0();
   }
 
   tc_fence_before();
