@@ -108,6 +108,21 @@ __host__ __device__ inline int owner(int x, int U, int grid) {
   return c;
 }
 
+// A block finishes its gate/up tiles one after the other, so a tile's ready
+// flag rises later the further it sits in its block's range.  The lateness of
+// down unit x is the largest such position among the tiles that make the z
+// columns x reads (0 when each is its block's first tile).
+__device__ inline int unit_lateness(int x, const Params& p, int grid) {
+  const int u = x % p.ud;
+  int late = 0;
+  for (int j = 0; j < p.sub; ++j) {
+    const int t = u * p.sub + j;  // gate/up tile: 64 features = one 64-wide k block of z
+    if (t >= p.G) break;
+    late = max(late, t - range_start(owner(t, p.G, grid), p.G, grid));
+  }
+  return late;
+}
+
 __device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void grid_dep_launch() {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
@@ -181,6 +196,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   // barrier, so every epilogue warp takes the same path through bar.sync
   int* s_epi_fail = s_flag + 1;
   uint64_t* rbar = reinterpret_cast<uint64_t*>(tail + 320);  // partial slices landed
+  // Down-step order (blocks with at most kMaxOrder down units): within each
+  // piece, the units whose z is ready first (lateness 0) come first.  The
+  // weight loader, the activation loader and the MMA thread all follow it.
+  constexpr int kMaxOrder = 64;
+  uint8_t* s_late = tail + 384;   // [kMaxOrder] lateness (capped) of unit d0 + k
+  uint8_t* s_order = tail + 448;  // [kMaxOrder] down step k -> unit d0 + s_order[k]
   int32_t* s_ids = reinterpret_cast<int32_t*>(tail + 512);            // [kMaxN]
   float* s_x = reinterpret_cast<float*>(s_ids + kMaxN);               // [128][kXStride]
   uint16_t* s_e = reinterpret_cast<uint16_t*>(s_x + 128 * kXStride);  // [N][64]
@@ -194,6 +215,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int d0 = range_start(blockIdx.x, p.Ud, grid), d1 = range_start(blockIdx.x + 1, p.Ud, grid);
   const int ngs = (t1 - t0) * p.ug;
   const int nsteps = ngs + (d1 - d0);
+  const int nd = d1 - d0;
+  const bool reorder = nd <= kMaxOrder;
   const uint32_t ncols = p.N <= 32 ? 32 : (p.N <= 64 ? 64 : (p.N <= 128 ? 128 : 256));
   // Tensor memory: two accumulators of ncols columns, then (p.stage_tmem) as
   // many down-unit weight slots as fit in the 512 columns; a slot holds one
@@ -230,10 +253,27 @@ __global__ void __launch_bounds__(kThreads, 1)
     tmem_alloc(tmem_slot, tmem_cols);
     tmem_relinquish();
   }
+  if (warp == 2 && reorder && nd > 0) {
+    for (int k = lane; k < nd; k += 32)
+      s_late[k] = uint8_t(min(255, unit_lateness(d0 + k, p, grid)));
+    __syncwarp();
+    if (lane == 0) {
+      int pos = 0;
+      for (int xb = d0; xb < d1;) {
+        const int xe = min(d1, (xb / p.ud + 1) * p.ud);  // one piece: one down tile
+        for (int pass = 0; pass < 2; ++pass)
+          for (int x = xb; x < xe; ++x)
+            if ((s_late[x - d0] == 0) == (pass == 0)) s_order[pos++] = uint8_t(x - d0);
+        xb = xe;
+      }
+    }
+  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  // the unit of the block's k-th down step
+  auto unit = [&](int k) { return d0 + (reorder ? int(s_order[k]) : k); };
   grid_dep_launch();
 
   if (warp == 0) {
@@ -254,7 +294,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             tma_load_2d_hint(&tm_wu, &fullA[s], a + j * A_BLOCK + A_BLOCK / 2, k0, tile * 64, once);
           } else if (j == 0) {
             // one 3-D copy brings all `sub` k blocks of the unit
-            const int x = d0 + i - ngs, tile = x / p.ud, u = x % p.ud;
+            const int x = unit(i - ngs), tile = x / p.ud, u = x % p.ud;
             tma_load_3d_hint(&tm_wd, &fullA[s], a, 0, tile * BM, u * p.sub, once);
           }
         }
@@ -286,33 +326,48 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
     ok = __shfl_sync(0xffffffffu, ok, 0);
-    // z for the down steps.  Every gate/up tile that feeds one of this
-    // block's down units must have raised its ready flag.  The whole warp
-    // polls those flags at once: checked one unit at a time, each check is
-    // an L2 round trip on the issue path of every unit.
-    if (ok && d1 > d0) {
+    // z for the down steps, in two rounds: first the units of lateness 0,
+    // then the rest.  Before a round the whole warp polls every ready flag
+    // the round needs at once (checked one unit at a time, each check would
+    // put an L2 round trip on the issue path of every unit); lane 0 then
+    // issues the round's z loads in step order.
+    auto poll = [&](bool late_round) {
       bool mine = true;
-      for (int x = d0 + lane; x < d1 && mine; x += 32) {
-        // unit x reads z columns [f_lo, f_hi), made by tiles f_lo/64 .. (f_hi-1)/64
-        const int f_lo = (x % p.ud) * p.sub * BK;
+      for (int k = lane; k < nd && mine; k += 32) {
+        if (reorder && ((s_late[k] != 0) != late_round)) continue;
+        // unit d0 + k reads z columns [f_lo, f_hi), made by tiles f_lo/64 .. (f_hi-1)/64
+        const int f_lo = ((d0 + k) % p.ud) * p.sub * BK;
         const int f_hi = min(p.F, f_lo + p.sub * BK);
         for (int t = f_lo / 64; t <= (f_hi - 1) / 64 && mine; ++t)
           mine = spin_until(&p.ready[t], 1u, abort_flag, p.err);
       }
-      ok = __all_sync(0xffffffffu, mine);
-    }
-    if (lane == 0 && ok) {
+      return __all_sync(0xffffffffu, mine);
+    };
+    int k = 0;  // next down step to issue (lane 0)
+    auto issue = [&](bool stop_at_late) {
       fence_async_global();
-      for (int i = ngs; i < nsteps; ++i) {
-        if (!mbar_wait(&emptyB[s], ph ^ 1, abort_flag, p.err)) break;
-        const int u = (d0 + i - ngs) % p.ud;
+      for (; k < nd; ++k) {
+        const int x = unit(k);
+        if (stop_at_late && reorder && s_late[x - d0] != 0) break;
+        if (!mbar_wait(&emptyB[s], ph ^ 1, abort_flag, p.err)) return false;
         uint8_t* b = sB + s * b_stage;
         mbar_arrive_expect_tx(&fullB[s], b_stage);
-        tma_load_3d(&tm_z, &fullB[s], b, 0, 0, u * p.sub);
+        tma_load_3d(&tm_z, &fullB[s], b, 0, 0, (x % p.ud) * p.sub);
         if (++s == SB) {
           s = 0;
           ph ^= 1;
         }
+      }
+      return true;
+    };
+    if (ok && nd > 0) {
+      ok = poll(false);
+      if (lane == 0 && ok) ok = issue(true);
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      const int k1 = __shfl_sync(0xffffffffu, k, 0);
+      if (ok && k1 < nd) {
+        ok = poll(true);
+        if (lane == 0 && ok) issue(false);
       }
     }
   } else if (warp == 1) {
