@@ -522,6 +522,31 @@ def measure_host_link(nbytes=1 << 30, reps=5):
     return out
 
 
+def measure_host_adamw(stp, w, U=4529, steps=3):
+    """The host AdamW (staple_adamw_rows) on U distinct rows of one layer's
+    bf16 table with fp32 moments, all in host memory as the pages keep them:
+    per element it reads and writes the weight (2 + 2 bytes) and both moments
+    (8 + 8) and reads the fp32 gradient (4).  All host threads."""
+    rng = np.random.default_rng(5)
+    table = np.zeros((w.V, w.F), np.uint16)            # touched rows only are paged in
+    m = np.zeros((w.V, w.F), np.float32)
+    v = np.zeros((w.V, w.F), np.float32)
+    ids = np.sort(rng.choice(w.V, U, replace=False)).astype(np.int32)
+    grad = (rng.standard_normal((U, w.F)) * 0.01).astype(np.float32)
+    stp.staple_adamw_rows(table, w.F, stp.STAPLE_BF16, w.F, ids, U, grad, w.F, m, v, w.F,
+                          lr=1e-3, beta1=0.9, beta2=0.999, eps=1e-8, weight_decay=0.0, step=1)
+    t0 = time.perf_counter()
+    for s in range(steps):
+        stp.staple_adamw_rows(table, w.F, stp.STAPLE_BF16, w.F, ids, U, grad, w.F, m, v, w.F,
+                              lr=1e-3, beta1=0.9, beta2=0.999, eps=1e-8, weight_decay=0.0,
+                              step=s + 2)
+    dt = (time.perf_counter() - t0) / steps
+    nbytes = U * w.F * 24
+    return {"rows": U, "F": w.F, "ms_per_step": dt * 1e3, "rows_per_s": U / dt,
+            "gbs": nbytes / dt / 1e9, "threads": os.cpu_count(),
+            "bytes_per_step": nbytes, "note": "host memory traffic of one layer's update"}
+
+
 def release_pinned():
     """Return cached page-locked host blocks to the system (torch keeps freed
     pinned blocks for reuse)."""
@@ -855,6 +880,7 @@ def main():
             if top[0] in gemm_flops:
                 tf = gemm_flops[top[0]] * wt.T * wt.D * wt.F / (top[1]["avg_us"] * 1e-6) / 1e12
             link = measure_host_link()
+            adamw = measure_host_adamw(stp, wt)
             k4 = kern.get("k4_gather_misses")
             if k4:
                 zc = tr["misses"] * wt.F * 2 / (k4["avg_us"] * 1e-6) / 1e9
@@ -871,6 +897,7 @@ def main():
                              "frac": None if tf is None else tf / pk["bf16_tflops_sustained"],
                              "peak_source": pk["source"] + " (cuBLAS bf16, sustained)"},
                 "clocks": tr["staple"]["clocks"], "kernels": kern, "host_link": link,
+                "host_adamw": adamw,
             }
         except Exception as ex:  # the decode line must still print
             line["train_layer"] = {"error": repr(ex)}

@@ -194,6 +194,20 @@ staple_status staple_gather_unique_rows(staple_context* ctx, const staple_cache*
                                         int32_t* miss_list, int32_t* miss_count, void* rows,
                                         staple_stream stream, staple_stream side);
 
+/* Cache write-back after the table rows changed on the host (an optimizer
+ * step on the host tables, where the pages keep them together with their
+ * AdamW moments: Table 4's caption, ai4snews summary): the cached copies of
+ * the listed distinct ids are read again from the table, so the cache keeps
+ * serving the current rows.
+ *   unique, slot, U_dev   device, from staple_gather_unique_rows (slot[j] =
+ *                         the cache slot of unique[j], -1 when not cached)
+ * Every grouped layer of a row is copied.  EINVAL if the cache was not built
+ * from this table's row shape. */
+staple_status staple_cache_refresh(staple_context* ctx, staple_cache* cache,
+                                   const staple_table* table, const int32_t* unique,
+                                   const int32_t* slot, const int32_t* U_dev,
+                                   staple_stream stream);
+
 /* staple_dedup followed by staple_gather_unique_rows (ids -> unique/inverse,
  * hit/miss map, U rows). */
 staple_status staple_gather_rows(staple_context* ctx, const staple_cache* cache,
@@ -308,6 +322,37 @@ staple_status staple_ffn_bwd(staple_context* ctx, staple_dtype dtype, int32_t T,
                              const void* dgh, const void* w_gate, const void* w_up, void* dx,
                              float* dw_gate, float* dw_up, float* dw_down, void* workspace,
                              size_t workspace_bytes, staple_stream stream);
+
+/* ------------------------------------------------ host optimizer (AdamW) */
+
+typedef struct staple_adamw {
+  float lr;
+  float beta1;
+  float beta2;
+  float eps;
+  float weight_decay;   /* decoupled: w -= lr * weight_decay * w */
+  int32_t step;         /* t >= 1: bias corrections 1 - beta^t */
+} staple_adamw;
+
+/* AdamW on the U table rows a step touched, on the host, where the tables
+ * and their fp32 moments live (the pages offload the tables with their AdamW
+ * moments to host DRAM: Table 4's caption; ai4snews summary).  For each
+ * j < U, row r = ids[j]:
+ *   m[r] = b1 m[r] + (1 - b1) g_j,   v[r] = b2 v[r] + (1 - b2) g_j^2
+ *   w[r] -= lr (m[r] / (1 - b1^t) / (sqrt(v[r] / (1 - b2^t)) + eps) + weight_decay w[r])
+ * computed in fp32 (Loshchilov & Hutter, decoupled weight decay); a bf16
+ * table is rounded to nearest, ties to even.
+ *   table      host, rows of F values (dtype), row pitch table_pitch elements
+ *              (a grouped table's layer: base + layer * F, pitch groups * F)
+ *   ids        host int32 [U], distinct (e.g. staple_embed_grad_to_host's ids)
+ *   grad       host fp32 [U][grad_pitch]: row j is the gradient of row ids[j]
+ *   m, v       host fp32 [V][moment_pitch], indexed by row id
+ *   threads    host threads to use (<= 0: all hardware threads)
+ * Plain host code (no device, no context); returns when done. */
+staple_status staple_adamw_rows(void* table, int64_t table_pitch, staple_dtype dtype, int32_t F,
+                                const int32_t* ids, int32_t U, const float* grad,
+                                int64_t grad_pitch, float* m, float* v, int64_t moment_pitch,
+                                const staple_adamw* hp, int32_t threads);
 
 /* ------------------------------------------- allocation-free table gradient */
 

@@ -18,7 +18,7 @@ import numpy as np
 __all__ = [
     "silu", "silu_grad", "dedup", "hot_set", "probe", "gather_rows",
     "ffn_forward", "ffn_backward", "forward_rows", "embed_grad_rows",
-    "weight_grad_entries", "dx_rows", "cache_rows_for", "paper_shapes",
+    "weight_grad_entries", "dx_rows", "cache_rows_for", "paper_shapes", "adamw_rows",
 ]
 
 
@@ -238,6 +238,40 @@ def dx_rows(rows, dy, x, ids, w_gate, w_up, w_down, table=None) -> np.ndarray:
     bw = ffn_backward(np.asarray(dy)[rows], np.asarray(x)[rows], np.asarray(ids)[rows],
                       w_gate, w_up, w_down, fw)
     return bw["dx"]
+
+
+# --------------------------------------------------------------------------
+# Host optimizer step on the touched rows ([TLA] Table 4 caption: the tables
+# are offloaded with their AdamW moments; [AIS] Interpretation: the table is
+# the trained parameter, per-row gradients)
+# --------------------------------------------------------------------------
+
+def adamw_rows(table, ids, grad, m, v, lr, beta1, beta2, eps, weight_decay, step):
+    """One AdamW step on the rows `ids` of a table, the others untouched.
+
+    The pages train the tables with AdamW, fp32 moments in host memory, but
+    print no update formula or hyperparameters.  Reading: the standard AdamW
+    with decoupled weight decay (Loshchilov & Hutter, "Decoupled Weight Decay
+    Regularization"), applied only to the rows that got a gradient:
+
+        m = b1 m + (1 - b1) g,    v = b2 v + (1 - b2) g^2
+        m_hat = m / (1 - b1^t),   v_hat = v / (1 - b2^t)
+        w = w - lr (m_hat / (sqrt(v_hat) + eps) + weight_decay w)
+
+    table, m, v: [V][F]; ids: [U] distinct; grad: [U][F].  Returns new fp64
+    copies (table, m, v); the oracle rounds nothing.
+    """
+    w = np.array(table, dtype=np.float64)
+    m = np.array(m, dtype=np.float64)
+    v = np.array(v, dtype=np.float64)
+    ids = np.asarray(ids, dtype=np.int64)
+    g = np.asarray(grad, dtype=np.float64)
+    m[ids] = beta1 * m[ids] + (1.0 - beta1) * g
+    v[ids] = beta2 * v[ids] + (1.0 - beta2) * g * g
+    m_hat = m[ids] / (1.0 - beta1 ** step)
+    v_hat = v[ids] / (1.0 - beta2 ** step)
+    w[ids] = w[ids] - lr * (m_hat / (np.sqrt(v_hat) + eps) + weight_decay * w[ids])
+    return w, m, v
 
 
 # --------------------------------------------------------------------------

@@ -160,3 +160,63 @@ def test_register_pageable_host_table(stp, ctx):
         assert int(mc.item()) == 3
     finally:
         stp.staple_table_unregister(table)
+
+
+def test_cache_refresh_after_host_adamw(stp, ctx):
+    """After the host AdamW updates a batch's rows, staple_cache_refresh
+    re-reads the cached ones: cached copies of the batch's hot ids equal the
+    updated table rows, the other cached rows are untouched, and a new gather
+    returns the updated table bit for bit (hits from the cache, misses from the
+    host).  Two grouped layers per host row; the optimizer updates layer 1."""
+    import torch
+    V, F, G, T = 4000, 128, 2, 2500
+    parts = [syn.bf16_normal((V, F), 0.05, 500 + g)[0] for g in range(G)]
+    E = np.ascontiguousarray(np.stack(parts, axis=1).reshape(V, G * F))
+    host = torch.from_numpy(E.view(np.int16)).pin_memory()
+    table = stp.staple_table_register(ctx, host, E.nbytes, V, F, G, stp.STAPLE_BF16,
+                                      stp.STAPLE_TABLE_HOST_PINNED)
+    freq = syn.calibration_freq(V, n_tokens=1 << 18)
+    cache = stp.staple_cache_build(ctx, table, freq, 0.05)
+    try:
+        hot = stp.staple_cache_hot_ids(cache)
+        K = hot.size
+        ids = syn.zipf_ids(T, V, 1.1, seed=77)
+        d_ids = torch.from_numpy(ids).cuda()
+        unique, inverse, sorted_pos, slot, miss = (empty(T, "i32") for _ in range(5))
+        seg, U, mc = empty(T + 1, "i32"), empty(1, "i32"), empty(1, "i32")
+        rows = torch.zeros((T, G * F), dtype=torch.bfloat16, device="cuda")
+        stp.staple_gather_rows(ctx, cache, table, d_ids, T, unique, inverse, seg, sorted_pos, U,
+                               slot, miss, mc, rows)
+        torch.cuda.synchronize()
+        u = int(U.item())
+        uniq = unique.cpu().numpy()[:u].copy()
+        cache_before = read_device(stp.staple_cache_rows(cache), K * G * F * 2).view(np.uint16)
+        cache_before = cache_before.reshape(K, G * F).copy()
+        # host AdamW on layer 1 of the batch's rows (the pinned buffer itself)
+        rng = np.random.default_rng(78)
+        grad = (rng.standard_normal((u, F)) * 0.1).astype(np.float32)
+        m = np.zeros((V, F), np.float32)
+        v = np.zeros((V, F), np.float32)
+        stp.staple_adamw_rows(host.data_ptr() + F * 2, G * F, stp.STAPLE_BF16, F, uniq, u, grad, F,
+                              m, v, F, lr=1e-2, beta1=0.9, beta2=0.999, eps=1e-8,
+                              weight_decay=0.0, step=1, threads=4)
+        updated = host.numpy().view(np.uint16).reshape(V, G * F).copy()
+        assert not np.array_equal(updated[uniq], E[uniq])          # the rows did change
+        stp.staple_cache_refresh(ctx, cache, table, unique, slot, U)
+        torch.cuda.synchronize()
+        assert stp.staple_get_error(ctx) == 0
+        cache_after = read_device(stp.staple_cache_rows(cache), K * G * F * 2).view(np.uint16)
+        cache_after = cache_after.reshape(K, G * F)
+        in_batch = np.isin(hot, uniq)
+        assert in_batch.any() and (~in_batch).any()
+        np.testing.assert_array_equal(cache_after[in_batch], updated[hot[in_batch]])
+        np.testing.assert_array_equal(cache_after[~in_batch], cache_before[~in_batch])
+        # a new gather sees the updated rows, hits and misses alike
+        rows2 = torch.zeros_like(rows)
+        stp.staple_gather_rows(ctx, cache, table, d_ids, T, unique, inverse, seg, sorted_pos, U,
+                               slot, miss, mc, rows2)
+        torch.cuda.synchronize()
+        np.testing.assert_array_equal(bits(rows2)[:u], updated[uniq])
+    finally:
+        stp.staple_cache_free(cache)
+        stp.staple_table_unregister(table)

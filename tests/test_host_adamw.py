@@ -1,0 +1,92 @@
+"""The library's host AdamW (staple_adamw_rows) against the oracle's fp64
+AdamW, on the CPU: no GPU is involved.
+
+fp32 tables: table and moments within 1e-6 relative to the oracle after
+several steps.  bf16 tables: the library updates in fp32 and rounds to bf16,
+the oracle in fp64; each value may differ from the oracle's value rounded to
+bf16 by at most one bf16 step.  The moments (fp32 in both cases) stay within
+1e-6.  Rows that got no gradient must not change, bit for bit.  Tables use a
+grouped layout (one layer's slice of a [V][G][F] array)."""
+from __future__ import annotations
+
+import numpy as np
+import pytest
+
+import oracle
+import synthetic as syn
+
+HP = dict(lr=3e-3, beta1=0.9, beta2=0.999, eps=1e-8, weight_decay=0.01)
+# the library receives the hyperparameters as fp32; the oracle gets the same
+# values (0.999 is 0.99900001287 in fp32, so 1 - beta2 differs by 1.3e-5
+# from the decimal)
+HP32 = {k: float(np.float32(x)) for k, x in HP.items()}
+
+
+@pytest.fixture(scope="module")
+def stp():
+    import token_indexed_sparse_staple_b200 as m
+    return m
+
+
+def _run(stp, dtype, threads, steps=3, V=700, F=96, G=3, layer=1, U=150, seed=41):
+    rng = np.random.default_rng(seed)
+    if dtype == "bf16":
+        full = syn.bf16_normal((V, G * F), 0.05, seed)[0]          # [V][G*F] bf16 bits
+        w_ref = syn.bf16_bits_to_f32(full[:, layer * F:(layer + 1) * F]).astype(np.float64)
+        sdt = stp.STAPLE_BF16
+    else:
+        full = (rng.standard_normal((V, G * F)) * 0.05).astype(np.float32)
+        w_ref = full[:, layer * F:(layer + 1) * F].astype(np.float64)
+        sdt = stp.STAPLE_F32
+    before = full.copy()
+    m = np.zeros((V, F), np.float32)
+    v = np.zeros((V, F), np.float32)
+    m_ref, v_ref = np.zeros((V, F)), np.zeros((V, F))
+    touched = np.zeros(V, bool)
+    for step in range(1, steps + 1):
+        ids = np.sort(rng.choice(V, U, replace=False)).astype(np.int32)
+        touched[ids] = True
+        g = (rng.standard_normal((U, F)) * 0.1).astype(np.float32)
+        base = full.ctypes.data + layer * F * full.itemsize
+        stp.staple_adamw_rows(base, G * F, sdt, F, ids, U, g, F, m, v, F, step=step,
+                              threads=threads, **HP)
+        w_new, m_ref, v_ref = oracle.adamw_rows(w_ref, ids, g.astype(np.float64), m_ref, v_ref,
+                                                step=step, **HP32)
+        got = full[:, layer * F:(layer + 1) * F]
+        if dtype == "bf16":
+            # one bf16 step (8 significant bits) at the oracle's value
+            got_f = syn.bf16_bits_to_f32(got).astype(np.float64)
+            step_size = np.exp2(np.floor(np.log2(np.maximum(np.abs(w_new), 1e-30))) - 7)
+            off = np.abs(got_f - w_new) / step_size
+            assert off.max() <= 1.0, f"step {step}: bf16 table off by {off.max():.2f} steps"
+            w_ref = got_f                 # the next step starts from the stored table
+        else:
+            np.testing.assert_allclose(got.astype(np.float64), w_new, rtol=1e-6,
+                                       atol=1e-6 * np.abs(w_new).max())
+            w_ref = got.astype(np.float64)
+        np.testing.assert_allclose(m, m_ref, rtol=1e-5, atol=1e-6 * np.abs(m_ref).max())
+        np.testing.assert_allclose(v, v_ref, rtol=1e-5, atol=1e-6 * np.abs(v_ref).max())
+        m_ref, v_ref = m.astype(np.float64), v.astype(np.float64)
+    # untouched rows, and the other layers of every row, are bit for bit unchanged
+    other = np.ones(G * F, bool)
+    other[layer * F:(layer + 1) * F] = False
+    np.testing.assert_array_equal(full[:, other], before[:, other])
+    np.testing.assert_array_equal(full[~touched], before[~touched])
+    assert not np.any(m[~touched]) and not np.any(v[~touched])
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("threads", [1, 4])
+def test_host_adamw_matches_oracle(stp, dtype, threads):
+    _run(stp, dtype, threads)
+
+
+def test_host_adamw_rejects_bad_arguments(stp):
+    import ctypes as C
+    hp = stp.staple_adamw(1e-3, 0.9, 0.999, 1e-8, 0.0, 0)     # step 0 is not a step
+    buf = np.zeros(16, np.float32)
+    ids = np.zeros(1, np.int32)
+    st = stp.lib().staple_adamw_rows(buf.ctypes.data, 4, stp.STAPLE_F32, 4, ids.ctypes.data, 1,
+                                     buf.ctypes.data, 4, buf.ctypes.data, buf.ctypes.data, 4,
+                                     C.byref(hp), 1)
+    assert st == stp.STAPLE_EINVAL

@@ -374,3 +374,62 @@ def test_planted_backward_mistakes_are_caught(kind, monkeypatch):
     monkeypatch.setattr(oracle, "ffn_backward", _mutant_backward(kind))
     with pytest.raises(AssertionError):
         test_backward_matches_brute_force(0)
+
+
+# --------------------------------------------------------------------------
+# Host AdamW on the touched rows
+# --------------------------------------------------------------------------
+
+_HP = dict(lr=1e-2, beta1=0.9, beta2=0.99, eps=1e-8, weight_decay=0.1)
+
+
+def test_adamw_dense_matches_torch_adamw():
+    """All rows touched every step: the oracle is torch.optim.AdamW (fp64)."""
+    import torch
+    rng = np.random.default_rng(31)
+    V, F = 6, 5
+    w0 = rng.standard_normal((V, F))
+    p = torch.nn.Parameter(torch.tensor(w0, dtype=torch.float64))
+    opt = torch.optim.AdamW([p], lr=_HP["lr"], betas=(_HP["beta1"], _HP["beta2"]),
+                            eps=_HP["eps"], weight_decay=_HP["weight_decay"])
+    w, m, v = w0.copy(), np.zeros((V, F)), np.zeros((V, F))
+    ids = np.arange(V)
+    for step in range(1, 4):
+        g = rng.standard_normal((V, F))
+        p.grad = torch.tensor(g, dtype=torch.float64)
+        opt.step()
+        w, m, v = oracle.adamw_rows(w, ids, g, m, v, step=step, **_HP)
+        np.testing.assert_allclose(w, p.detach().numpy(), rtol=1e-12, atol=1e-14)
+
+
+def test_adamw_first_step_closed_form_and_untouched_rows():
+    """From zero moments, step 1 moves w by lr (g / (|g| + eps) + wd w); rows
+    without a gradient keep their value and moments."""
+    rng = np.random.default_rng(32)
+    V, F = 10, 7
+    w0 = rng.standard_normal((V, F))
+    m0, v0 = np.zeros((V, F)), np.zeros((V, F))
+    m0[1], v0[1] = 0.5, 0.25                      # an untouched row with state
+    ids = np.array([3, 7, 0])
+    g = rng.standard_normal((3, F))
+    w, m, v = oracle.adamw_rows(w0, ids, g, m0, v0, step=1, **_HP)
+    expect = w0[ids] - _HP["lr"] * (g / (np.abs(g) + _HP["eps"]) + _HP["weight_decay"] * w0[ids])
+    np.testing.assert_allclose(w[ids], expect, rtol=1e-12)
+    rest = np.setdiff1d(np.arange(V), ids)
+    np.testing.assert_array_equal(w[rest], w0[rest])
+    np.testing.assert_array_equal(m[rest], m0[rest])
+    np.testing.assert_array_equal(v[rest], v0[rest])
+
+
+def test_planted_adamw_mistake_is_caught(monkeypatch):
+    """Without the bias corrections the closed form above fails."""
+    def no_bias_correction(table, ids, grad, m, v, lr, beta1, beta2, eps, weight_decay, step):
+        w, m, v = np.array(table, float), np.array(m, float), np.array(v, float)
+        g = np.asarray(grad, float)
+        m[ids] = beta1 * m[ids] + (1 - beta1) * g
+        v[ids] = beta2 * v[ids] + (1 - beta2) * g * g
+        w[ids] = w[ids] - lr * (m[ids] / (np.sqrt(v[ids]) + eps) + weight_decay * w[ids])
+        return w, m, v
+    monkeypatch.setattr(oracle, "adamw_rows", no_bias_correction)
+    with pytest.raises(AssertionError):
+        test_adamw_first_step_closed_form_and_untouched_rows()

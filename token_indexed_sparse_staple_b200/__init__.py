@@ -15,7 +15,7 @@ import ctypes as C
 import numpy as np
 
 from . import _lib
-from ._lib import staple_embed
+from ._lib import staple_adamw, staple_embed
 
 STAPLE_OK = 0
 STAPLE_EINVAL, STAPLE_EIDRANGE, STAPLE_ECUDA, STAPLE_ENOMEM = -1, -2, -3, -4
@@ -25,7 +25,7 @@ STAPLE_EMBED_NONE, STAPLE_EMBED_TABLE, STAPLE_EMBED_ROWS = 0, 1, 2
 STAPLE_TABLE_DEVICE, STAPLE_TABLE_HOST_PINNED, STAPLE_TABLE_HOST_REGISTER = 1, 2, 4
 
 __all__ = [n for n in _lib.SIGNATURES] + [
-    "StapleError", "staple_embed", "make_embed", "lib",
+    "StapleError", "staple_embed", "staple_adamw", "make_embed", "lib",
 ]
 
 
@@ -231,3 +231,20 @@ def staple_embed_grad_static(dtype, T, F, dh, ld, sorted_pos, inverse, seg_off, 
     _ok(lib().staple_embed_grad_static(dtype, T, F, _p(dh), ld, _p(sorted_pos), _p(inverse),
                                        _p(seg_off), _p(dE), _stream(stream)),
         "staple_embed_grad_static")
+
+
+def staple_cache_refresh(ctx, cache, table, unique, slot, U_dev, stream=None):
+    """Re-read the cached copies of the listed distinct ids from the table
+    (after a host-side update; see include/staple.h)."""
+    _ok(lib().staple_cache_refresh(ctx, cache, table, _p(unique), _p(slot), _p(U_dev),
+                                   _stream(stream)), "staple_cache_refresh")
+
+
+def staple_adamw_rows(table, table_pitch, dtype, F, ids, U, grad, grad_pitch, m, v, moment_pitch,
+                      lr, beta1, beta2, eps, weight_decay, step, threads=0):
+    """Host AdamW on the U table rows listed in ids (all host buffers: numpy
+    arrays, pinned tensors or raw addresses; see include/staple.h)."""
+    hp = staple_adamw(lr, beta1, beta2, eps, weight_decay, step)
+    _ok(lib().staple_adamw_rows(_p(table), table_pitch, dtype, F, _p(ids), U, _p(grad), grad_pitch,
+                                _p(m), _p(v), moment_pitch, C.byref(hp), threads),
+        "staple_adamw_rows")

@@ -28,6 +28,11 @@ class staple_embed(C.Structure):
                 ("index", vp), ("n_rows", i64)]
 
 
+class staple_adamw(C.Structure):
+    _fields_ = [("lr", C.c_float), ("beta1", C.c_float), ("beta2", C.c_float), ("eps", C.c_float),
+                ("weight_decay", C.c_float), ("step", i32)]
+
+
 # name -> (restype, argtypes); mirrors include/staple.h
 SIGNATURES = {
     "staple_abi_version": (C.c_int, []),
@@ -56,6 +61,9 @@ SIGNATURES = {
     "staple_ffn_bwd": (c_status, [vp, C.c_int, i32, i32, i32, vp, vp, vp, vp, vp, vp, vp, vp,
                                   vp, vp, vp, sz, vp]),
     "staple_embed_grad_to_host": (c_status, [vp, i32, i32, vp, vp, vp, vp, vp, vp, vp]),
+    "staple_cache_refresh": (c_status, [vp, vp, vp, vp, vp, vp, vp]),
+    "staple_adamw_rows": (c_status, [vp, i64, C.c_int, i32, vp, i32, vp, i64, vp, vp, i64,
+                                     P(staple_adamw), i32]),
     "staple_embed_grad": (c_status, [vp, C.c_int, i32, i32, i32, vp, i64, vp, vp, vp, vp, vp, vp,
                                      sz, vp]),
     "staple_embed_grad_static": (c_status, [C.c_int, i32, i32, vp, i64, vp, vp, vp, vp, vp]),

@@ -275,7 +275,7 @@ __global__ void __launch_bounds__(1024)
 // flight per thread.  K3 copies hit rows from the cache; K4 reads miss rows
 // from the table (mapped host memory, or HBM for a device table).
 // ---------------------------------------------------------------------------
-enum GatherMode { G_HITS = 0, G_MISSES = 1, G_LIST = 2 };
+enum GatherMode { G_HITS = 0, G_MISSES = 1, G_LIST = 2, G_REFRESH = 3 };
 
 template <int MODE>
 __global__ void __launch_bounds__(256)
@@ -298,6 +298,10 @@ __global__ void __launch_bounds__(256)
     } else if (MODE == G_MISSES) { // rows[j] = table[unique[j]], j from the miss list
       j = miss_list[i];
       srow = ids[j];
+    } else if (MODE == G_REFRESH) { // cache[slot[j]] = table[ids[j]] for cached ids
+      if (slot[i] < 0) continue;
+      j = slot[i];
+      srow = ids[i];
     } else {                       // rows[i] = table[ids[i]]
       j = i;
       srow = ids[i];
@@ -342,6 +346,20 @@ staple_status launch_gather_misses(const void* table_dev, int64_t table_pitch_by
              gather_kernel<G_MISSES><<<num_sms, 256, 0, st>>>(
                  static_cast<const uint8_t*>(table_dev), table_pitch_bytes, unique, miss_count,
                  nullptr, miss_list, static_cast<uint8_t*>(rows), row_bytes));
+  return cudaGetLastError() == cudaSuccess ? STAPLE_OK : STAPLE_ECUDA;
+}
+
+// Cache write-back after a table update: the cached copies of the listed
+// distinct ids (slot from the probe, -1 when not cached) are read again from
+// the table.
+staple_status launch_cache_refresh(const void* table_dev, int64_t table_pitch_bytes,
+                                   int64_t row_bytes, const int32_t* unique, const int32_t* slot,
+                                   const int32_t* U_dev, void* cache_rows, int num_sms,
+                                   cudaStream_t st) {
+  STP_LAUNCH("k14_cache_refresh", st,
+             gather_kernel<G_REFRESH><<<num_sms, 256, 0, st>>>(
+                 static_cast<const uint8_t*>(table_dev), table_pitch_bytes, unique, U_dev, slot,
+                 nullptr, static_cast<uint8_t*>(cache_rows), row_bytes));
   return cudaGetLastError() == cudaSuccess ? STAPLE_OK : STAPLE_ECUDA;
 }
 

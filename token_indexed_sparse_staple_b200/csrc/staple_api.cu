@@ -374,6 +374,21 @@ staple_status staple_gather_unique_rows(staple_context* ctx, const staple_cache*
   return STAPLE_OK;
 }
 
+staple_status staple_cache_refresh(staple_context* ctx, staple_cache* cache,
+                                   const staple_table* table, const int32_t* unique,
+                                   const int32_t* slot, const int32_t* U_dev,
+                                   staple_stream stream) {
+  if (!ctx || !cache || !table || !unique || !slot || !U_dev) return STAPLE_EINVAL;
+  if (cache->device != ctx->di.device ||
+      cache->row_bytes != int64_t(table->groups) * table->F * int64_t(esize(table->dtype)))
+    return STAPLE_EINVAL;
+  if (cache->K == 0) return STAPLE_OK;
+  STP_TRY(set_device(ctx));
+  stp::TraceScope trace_scope(ctx->tracer);
+  return stp::launch_cache_refresh(table->dev, cache->row_bytes, cache->row_bytes, unique, slot,
+                                   U_dev, cache->rows, ctx->di.num_sms, cs(stream));
+}
+
 staple_status staple_gather_rows(staple_context* ctx, const staple_cache* cache,
                                  const staple_table* table, const int32_t* ids, int32_t T,
                                  int32_t* unique, int32_t* inverse, int32_t* seg_off,
