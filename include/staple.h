@@ -194,6 +194,30 @@ staple_status staple_gather_unique_rows(staple_context* ctx, const staple_cache*
                                         int32_t* miss_list, int32_t* miss_count, void* rows,
                                         staple_stream stream, staple_stream side);
 
+/* staple_gather_unique_rows with the misses taken the bulk way, the pages'
+ * prefill path (retrieval-path table, Prefill row): the miss rows are packed
+ * on the host into a page-locked staging buffer and copied to the device in
+ * bulk by the copy engine (chunk by chunk, each chunk's copy starting as soon
+ * as it is packed), then placed into rows by a scatter kernel.  No SM reads
+ * host memory.  The calling thread waits for the probe (the host needs the
+ * miss list), packs with `threads` host threads (<= 0: all), and returns once
+ * the copies and the scatter are queued on `stream`; call it from a helper
+ * thread to overlap it with other work.  Not while `stream` is captured.
+ *   staging_host  page-locked, >= T * groups * F elements
+ *   staging_dev   device, >= T * groups * F elements, 16-byte aligned
+ *   list_host     page-locked int32 [1 + 2T] (miss count, miss list, ids)
+ *   chunk_rows    rows per bulk copy (>= 1)
+ * The buffers may be reused by the next call on the same stream.  The table
+ * must be in host memory (HOST_PINNED or HOST_REGISTER).  Same results as
+ * staple_gather_unique_rows, bit for bit. */
+staple_status staple_gather_unique_rows_bulk(staple_context* ctx, const staple_cache* cache,
+                                             const staple_table* table, const int32_t* unique,
+                                             const int32_t* U_dev, int32_t T, int32_t* slot,
+                                             int32_t* miss_list, int32_t* miss_count, void* rows,
+                                             void* staging_host, void* staging_dev,
+                                             int32_t* list_host, int32_t chunk_rows,
+                                             int32_t threads, staple_stream stream);
+
 /* Cache write-back after the table rows changed on the host (an optimizer
  * step on the host tables, where the pages keep them together with their
  * AdamW moments: Table 4's caption, ai4snews summary): the cached copies of

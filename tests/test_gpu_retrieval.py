@@ -220,3 +220,61 @@ def test_cache_refresh_after_host_adamw(stp, ctx):
     finally:
         stp.staple_cache_free(cache)
         stp.staple_table_unregister(table)
+
+
+@pytest.mark.parametrize("frac,groups,chunk,threads", [(0.05, 1, 256, 4), (0.0, 1, 7, 1),
+                                                       (0.05, 4, 1, 0), (1.0, 2, 64, 2)])
+def test_bulk_miss_path_equals_zero_copy(stp, ctx, frac, groups, chunk, threads):
+    """The prefill path (misses packed on the host, bulk copy, scatter) gives
+    the same rows, hit/miss map and miss list as the zero-copy gather, bit for
+    bit, and both equal the oracle's rows; two calls in a row on one stream
+    reuse the staging buffers."""
+    import torch
+    V, F, T = 3000, 128, 2000
+    w = syn.Workload("bulk", T=T, D=64, F=F, V=V, layers=groups, dtype="bf16", w_std=0.02,
+                     e_std=0.05, x_std=1.0, dy_std=1.0, table="host", cache_frac=frac,
+                     group=groups, training=False)
+    E = _table(w, groups=groups)
+    host = torch.from_numpy(E.view(np.int16)).pin_memory()
+    table = stp.staple_table_register(ctx, host, E.nbytes, V, F, groups, stp.STAPLE_BF16,
+                                      stp.STAPLE_TABLE_HOST_PINNED)
+    cache = stp.staple_cache_build(ctx, table, syn.calibration_freq(V, n_tokens=1 << 18), frac)
+    try:
+        st = torch.cuda.Stream()
+        staging_h = torch.empty((T, groups * F), dtype=torch.bfloat16).pin_memory()
+        staging_d = torch.empty((T, groups * F), dtype=torch.bfloat16, device="cuda")
+        list_h = torch.empty(1 + 2 * T, dtype=torch.int32).pin_memory()
+        for rep in range(2):
+            ids = syn.zipf_ids(T, V, 1.1, seed=90 + rep)
+            d_ids = torch.from_numpy(ids).cuda()
+            unique, inverse, sorted_pos = (empty(T, "i32") for _ in range(3))
+            seg, U = empty(T + 1, "i32"), empty(1, "i32")
+            stp.staple_dedup(ctx, d_ids, T, V, unique, inverse, seg, sorted_pos, U, stream=st)
+            out = {}
+            for path in ("zero_copy", "bulk"):
+                slot, miss = empty(T, "i32"), empty(T, "i32")
+                mc = empty(1, "i32")
+                rows = torch.zeros((T, groups * F), dtype=torch.bfloat16, device="cuda")
+                if path == "bulk":
+                    stp.staple_gather_unique_rows_bulk(ctx, cache, table, unique, U, T, slot, miss,
+                                                       mc, rows, staging_h, staging_d, list_h,
+                                                       chunk_rows=chunk, threads=threads, stream=st)
+                else:
+                    stp.staple_gather_unique_rows(ctx, cache, table, unique, U, T, slot, miss, mc,
+                                                  rows, stream=st, side=st)
+                st.synchronize()
+                u = int(U.item())
+                out[path] = (bits(rows)[:u], slot.cpu().numpy()[:u], int(mc.item()),
+                             miss.cpu().numpy()[:int(mc.item())])
+            assert stp.staple_get_error(ctx, st) == 0
+            zr, zs, zc, zm = out["zero_copy"]
+            br, bs, bc, bm = out["bulk"]
+            np.testing.assert_array_equal(br, zr)
+            np.testing.assert_array_equal(bs, zs)
+            assert bc == zc
+            np.testing.assert_array_equal(bm, zm)
+            u_ref = oracle.dedup(ids)[0]
+            np.testing.assert_array_equal(br, oracle.gather_rows(E, u_ref))
+    finally:
+        stp.staple_cache_free(cache)
+        stp.staple_table_unregister(table)

@@ -248,3 +248,16 @@ def staple_adamw_rows(table, table_pitch, dtype, F, ids, U, grad, grad_pitch, m,
     _ok(lib().staple_adamw_rows(_p(table), table_pitch, dtype, F, _p(ids), U, _p(grad), grad_pitch,
                                 _p(m), _p(v), moment_pitch, C.byref(hp), threads),
         "staple_adamw_rows")
+
+
+def staple_gather_unique_rows_bulk(ctx, cache, table, unique, U_dev, T, slot, miss_list,
+                                   miss_count, rows, staging_host, staging_dev, list_host,
+                                   chunk_rows=256, threads=0, stream=None):
+    """Rows of the batch's distinct ids with the misses packed on the host and
+    copied in bulk (the prefill path; see include/staple.h).  Blocks the
+    calling thread until the probe is done and the rows are packed."""
+    _ok(lib().staple_gather_unique_rows_bulk(ctx, cache, table, _p(unique), _p(U_dev), T, _p(slot),
+                                             _p(miss_list), _p(miss_count), _p(rows),
+                                             _p(staging_host), _p(staging_dev), _p(list_host),
+                                             chunk_rows, threads, _stream(stream)),
+        "staple_gather_unique_rows_bulk")

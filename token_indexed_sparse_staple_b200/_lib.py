@@ -62,6 +62,8 @@ SIGNATURES = {
                                   vp, vp, vp, sz, vp]),
     "staple_embed_grad_to_host": (c_status, [vp, i32, i32, vp, vp, vp, vp, vp, vp, vp]),
     "staple_cache_refresh": (c_status, [vp, vp, vp, vp, vp, vp, vp]),
+    "staple_gather_unique_rows_bulk": (c_status, [vp, vp, vp, vp, vp, i32, vp, vp, vp, vp, vp, vp,
+                                                  vp, i32, i32, vp]),
     "staple_adamw_rows": (c_status, [vp, i64, C.c_int, i32, vp, i32, vp, i64, vp, vp, i64,
                                      P(staple_adamw), i32]),
     "staple_embed_grad": (c_status, [vp, C.c_int, i32, i32, i32, vp, i64, vp, vp, vp, vp, vp, vp,

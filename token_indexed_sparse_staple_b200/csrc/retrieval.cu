@@ -275,7 +275,7 @@ __global__ void __launch_bounds__(1024)
 // flight per thread.  K3 copies hit rows from the cache; K4 reads miss rows
 // from the table (mapped host memory, or HBM for a device table).
 // ---------------------------------------------------------------------------
-enum GatherMode { G_HITS = 0, G_MISSES = 1, G_LIST = 2, G_REFRESH = 3 };
+enum GatherMode { G_HITS = 0, G_MISSES = 1, G_LIST = 2, G_REFRESH = 3, G_SCATTER = 4 };
 
 template <int MODE>
 __global__ void __launch_bounds__(256)
@@ -298,6 +298,9 @@ __global__ void __launch_bounds__(256)
     } else if (MODE == G_MISSES) { // rows[j] = table[unique[j]], j from the miss list
       j = miss_list[i];
       srow = ids[j];
+    } else if (MODE == G_SCATTER) { // rows[miss_list[i]] = staging[i]
+      j = miss_list[i];
+      srow = i;
     } else if (MODE == G_REFRESH) { // cache[slot[j]] = table[ids[j]] for cached ids
       if (slot[i] < 0) continue;
       j = slot[i];
@@ -346,6 +349,18 @@ staple_status launch_gather_misses(const void* table_dev, int64_t table_pitch_by
              gather_kernel<G_MISSES><<<num_sms, 256, 0, st>>>(
                  static_cast<const uint8_t*>(table_dev), table_pitch_bytes, unique, miss_count,
                  nullptr, miss_list, static_cast<uint8_t*>(rows), row_bytes));
+  return cudaGetLastError() == cudaSuccess ? STAPLE_OK : STAPLE_ECUDA;
+}
+
+// Miss rows that arrived packed in miss order (bulk path): staging row i goes
+// to rows[miss_list[i]].
+staple_status launch_scatter_misses(const void* staging, int64_t row_bytes,
+                                    const int32_t* miss_list, const int32_t* miss_count,
+                                    void* rows, int num_sms, cudaStream_t st) {
+  STP_LAUNCH("k4b_scatter_misses", st,
+             gather_kernel<G_SCATTER><<<num_sms * 2, 256, 0, st>>>(
+                 static_cast<const uint8_t*>(staging), row_bytes, nullptr, miss_count, nullptr,
+                 miss_list, static_cast<uint8_t*>(rows), row_bytes));
   return cudaGetLastError() == cudaSuccess ? STAPLE_OK : STAPLE_ECUDA;
 }
 

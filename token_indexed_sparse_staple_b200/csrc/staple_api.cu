@@ -3,8 +3,10 @@
 // stream orchestration around the kernels.  Every compute step runs in the
 // CUDA kernels of the other translation units.
 #include <cuda_runtime.h>
+#include <thread>
 
 #include <algorithm>
+#include <atomic>
 #include <cmath>
 #include <cstring>
 #include <new>
@@ -372,6 +374,81 @@ staple_status staple_gather_unique_rows(staple_context* ctx, const staple_cache*
     STP_CUDA(cudaStreamWaitEvent(st, ctx->ev_side, 0));
   }
   return STAPLE_OK;
+}
+
+staple_status staple_gather_unique_rows_bulk(staple_context* ctx, const staple_cache* cache,
+                                             const staple_table* table, const int32_t* unique,
+                                             const int32_t* U_dev, int32_t T, int32_t* slot,
+                                             int32_t* miss_list, int32_t* miss_count, void* rows,
+                                             void* staging_host, void* staging_dev,
+                                             int32_t* list_host, int32_t chunk_rows,
+                                             int32_t threads, staple_stream stream) {
+  if (!ctx || !table || !U_dev || !slot || !miss_list || !miss_count || T < 0) return STAPLE_EINVAL;
+  if (T > 0 && (!unique || !rows || !staging_host || !staging_dev || !list_host)) return STAPLE_EINVAL;
+  if (!aligned16(rows) || !aligned16(staging_dev) || chunk_rows < 1) return STAPLE_EINVAL;
+  if (!(table->flags & (STAPLE_TABLE_HOST_PINNED | STAPLE_TABLE_HOST_REGISTER))) return STAPLE_EINVAL;
+  const int64_t row_bytes = int64_t(table->groups) * table->F * int64_t(esize(table->dtype));
+  if (cache && cache->row_bytes != row_bytes) return STAPLE_EINVAL;
+  STP_TRY(set_device(ctx));
+  cudaStream_t st = cs(stream);
+  cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+  STP_CUDA(cudaStreamIsCapturing(st, &cap));
+  if (cap != cudaStreamCaptureStatusNone) return STAPLE_EINVAL;  // the host must wait below
+  stp::TraceScope trace_scope(ctx->tracer);
+  if (T == 0) return STAPLE_OK;
+  STP_TRY(stp::launch_probe(unique, U_dev, cache && cache->K > 0 ? cache->hkeys : nullptr,
+                            cache ? cache->hvals : nullptr,
+                            cache ? uint32_t(cache->cap - 1) : 0u, slot, miss_list, miss_count,
+                            st));
+  // the miss ids to the host: count, miss list, unique ids (list_host: [1 + 2T])
+  STP_CUDA(cudaMemcpyAsync(list_host, miss_count, sizeof(int32_t), cudaMemcpyDeviceToHost, st));
+  STP_CUDA(cudaMemcpyAsync(list_host + 1, miss_list, size_t(T) * sizeof(int32_t),
+                           cudaMemcpyDeviceToHost, st));
+  STP_CUDA(cudaMemcpyAsync(list_host + 1 + T, unique, size_t(T) * sizeof(int32_t),
+                           cudaMemcpyDeviceToHost, st));
+  STP_CUDA(cudaEventRecord(ctx->ev_main, st));
+  if (cache && cache->K > 0)
+    STP_TRY(stp::launch_gather_hits(cache->rows, row_bytes, U_dev, slot, rows, ctx->di.num_sms, st));
+  STP_CUDA(cudaEventSynchronize(ctx->ev_main));
+  // pack the miss rows from the host table in miss order, chunk by chunk;
+  // each chunk's copy to the device starts as soon as it is packed
+  const int32_t n = std::min(list_host[0], T);
+  const int32_t* ml = list_host + 1;
+  const int32_t* uq = list_host + 1 + T;
+  const uint8_t* src = static_cast<const uint8_t*>(table->base);
+  uint8_t* hs = static_cast<uint8_t*>(staging_host);
+  uint8_t* ds = static_cast<uint8_t*>(staging_dev);
+  const int32_t nchunks = (n + chunk_rows - 1) / chunk_rows;
+  int nt = threads > 0 ? threads : int(std::thread::hardware_concurrency());
+  nt = std::max(1, std::min(nt, nchunks));
+  // one pool per call: workers claim chunks and mark each one packed; this
+  // thread issues the chunks' copies in order as they become ready
+  std::atomic<int32_t> next{0};
+  std::vector<std::atomic<int>> packed(size_t(std::max(nchunks, 1)));
+  for (auto& a : packed) a.store(0, std::memory_order_relaxed);
+  auto worker = [&]() {
+    for (int32_t c; (c = next.fetch_add(1)) < nchunks;) {
+      const int32_t c1 = std::min(n, (c + 1) * chunk_rows);
+      for (int32_t i = c * chunk_rows; i < c1; ++i)
+        std::memcpy(hs + int64_t(i) * row_bytes, src + int64_t(uq[ml[i]]) * row_bytes,
+                    size_t(row_bytes));
+      packed[size_t(c)].store(1, std::memory_order_release);
+    }
+  };
+  std::vector<std::thread> pool;
+  for (int t = 0; t < nt; ++t) pool.emplace_back(worker);
+  cudaError_t ce = cudaSuccess;
+  for (int32_t c = 0; c < nchunks; ++c) {
+    while (!packed[size_t(c)].load(std::memory_order_acquire)) std::this_thread::yield();
+    const int32_t c0 = c * chunk_rows, c1 = std::min(n, c0 + chunk_rows);
+    if (ce == cudaSuccess)
+      ce = cudaMemcpyAsync(ds + int64_t(c0) * row_bytes, hs + int64_t(c0) * row_bytes,
+                           size_t(c1 - c0) * size_t(row_bytes), cudaMemcpyHostToDevice, st);
+  }
+  for (auto& th : pool) th.join();
+  if (ce != cudaSuccess) return STAPLE_ECUDA;
+  return stp::launch_scatter_misses(staging_dev, row_bytes, miss_list, miss_count, rows,
+                                    ctx->di.num_sms, st);
 }
 
 staple_status staple_cache_refresh(staple_context* ctx, staple_cache* cache,
