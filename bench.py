@@ -168,10 +168,10 @@ class Clocks:
 # to the captured value; otherwise the roofline's traffic is null.
 CAPTURED_TRAFFIC = {
     "k5k6_decode_fused": {
-        "bytes": 104_721_408,   # mean of two launches: 104,783,872 and 104,658,944
+        "bytes": 105_380_736,   # mean of two launches: 104,985,088 and 105,776,384
         "sources": ["token_indexed_sparse_staple_b200/csrc/decode_fused.cuh",
                     "token_indexed_sparse_staple_b200/csrc/common.cuh"],
-        "sha256": "17197f137ce9eb2a844d325527441d831dcc9a9b7022cff282f4428deceb022b",
+        "sha256": "4647dd800c2c0b6da6c48f346d879fd031482b13f079970f888337c404a604b3",
         "profile": "profiles/decode_fused_olmo2_1b_T64.md",
     },
 }

@@ -175,8 +175,9 @@ def test_trace_records_every_kernel(stp, ctx):
 
 @pytest.mark.parametrize("T", [1, 17, 64, 200, 256])
 def test_bf16_decode_sizes_match_oracle(stp, ctx, T):
-    """T <= 256 runs the weight-streaming kernels (weights on the MMA's M side,
-    split-K down projection with a last-block reduction)."""
+    """T <= 256 runs the fused weight-streaming kernel (weights on the MMA's M
+    side, stream-K down projection whose fp32 partials are summed in piece
+    order)."""
     w = _bf16_workload(T, 256, 576, 4000)
     inp = syn.make_layer_inputs(w, with_dy=False)
     got = run_layer(stp, ctx, inp, w.D, w.F, w.V, embed="table", training=False)
@@ -193,8 +194,9 @@ def test_bf16_decode_saves_g_and_h(stp, ctx):
 
 @pytest.mark.parametrize("D,F", [(2048, 1024), (1024, 8192), (4096, 11008)])
 def test_bf16_decode_cluster_split_shapes(stp, ctx, D, F):
-    """Down projections whose K is split over 2..8 blocks of a cluster, and
-    the 7B shape (d_ff 11008 = 172 k blocks of 64)."""
+    """Down tiles whose K is split over a few to many blocks, and the 7B shape
+    (d_ff 11008 = 172 gate/up tiles over at most 148 blocks, so some blocks
+    make two)."""
     w = _bf16_workload(64, D, F, 2000)
     inp = syn.make_layer_inputs(w, with_dy=False)
     got = run_layer(stp, ctx, inp, w.D, w.F, w.V, embed="table", training=False)

@@ -97,12 +97,16 @@ struct Params {
   int32_t* err;
 };
 
-__host__ __device__ inline int range_start(int c, int U, int grid) {
-  return int((int64_t(c) * U) / grid);
+// floor(a * b / d) for non-negative a, b and positive d; 32-bit division
+// whenever the product fits (a 64-bit division is a long software sequence).
+__host__ __device__ inline int muldiv(int a, int b, int d) {
+  const uint64_t prod = uint64_t(a) * uint64_t(b);
+  return prod <= 0xffffffffull ? int(uint32_t(prod) / uint32_t(d)) : int(prod / uint64_t(d));
 }
+__host__ __device__ inline int range_start(int c, int U, int grid) { return muldiv(c, U, grid); }
 // The block whose range holds unit x.
 __host__ __device__ inline int owner(int x, int U, int grid) {
-  int c = int((int64_t(x) * grid) / U);
+  int c = muldiv(x, grid, U);
   while (c + 1 < grid && range_start(c + 1, U, grid) <= x) ++c;
   while (c > 0 && range_start(c, U, grid) > x) --c;
   return c;
@@ -196,6 +200,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   // barrier, so every epilogue warp takes the same path through bar.sync
   int* s_epi_fail = s_flag + 1;
   uint64_t* rbar = reinterpret_cast<uint64_t*>(tail + 320);  // partial slices landed
+  uint64_t* obar = reinterpret_cast<uint64_t*>(tail + 328);  // down-step order written
   // Down-step order (blocks with at most kMaxOrder down units): within each
   // piece, the units whose z is ready first (lateness 0) come first.  The
   // weight loader, the activation loader and the MMA thread all follow it.
@@ -239,6 +244,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&tempty[b], 4);
     }
     mbar_init(rbar, 1);
+    mbar_init(obar, 1);
     *abort_flag = 0;
     *s_epi_fail = 0;
     fence_barrier_init();
@@ -253,7 +259,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     tmem_alloc(tmem_slot, tmem_cols);
     tmem_relinquish();
   }
-  if (warp == 2 && reorder && nd > 0) {
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  // the unit of the block's k-th down step
+  auto unit = [&](int k) { return d0 + (reorder ? int(s_order[k]) : k); };
+  // The step order is worked out by an epilogue warp (idle until the first
+  // gate/up tile is done), off the path of the first weight loads; the
+  // loaders wait for it on obar before their first down step.
+  const bool ordered = reorder && nd > 0;
+  if (warp == 3 && ordered) {
     for (int k = lane; k < nd; k += 32)
       s_late[k] = uint8_t(min(255, unit_lateness(d0 + k, p, grid)));
     __syncwarp();
@@ -267,13 +283,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         xb = xe;
       }
     }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(obar);
   }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem_base = *tmem_slot;
-  // the unit of the block's k-th down step
-  auto unit = [&](int k) { return d0 + (reorder ? int(s_order[k]) : k); };
   grid_dep_launch();
 
   if (warp == 0) {
@@ -283,6 +295,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       int s = 0;
       uint32_t ph = 0;
       for (int i = 0; i < nsteps; ++i) {
+        if (i == ngs && ordered && !mbar_wait(obar, 0, abort_flag, p.err)) break;
         if (!mbar_wait(&emptyA[s], ph ^ 1, abort_flag, p.err)) break;
         mbar_arrive_expect_tx(&fullA[s], a_stage);
         uint8_t* a = sA + s * a_stage;
@@ -360,6 +373,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       return true;
     };
+    if (ok && ordered) ok = __all_sync(0xffffffffu, mbar_wait(obar, 0, abort_flag, p.err));
     if (ok && nd > 0) {
       ok = poll(false);
       if (lane == 0 && ok) ok = issue(true);
