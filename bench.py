@@ -168,10 +168,10 @@ class Clocks:
 # to the captured value; otherwise the roofline's traffic is null.
 CAPTURED_TRAFFIC = {
     "k5k6_decode_fused": {
-        "bytes": 105_380_736,   # mean of two launches: 104,985,088 and 105,776,384
+        "bytes": 104_836_480,   # mean of two launches: 104,961,536 and 104,711,424
         "sources": ["token_indexed_sparse_staple_b200/csrc/decode_fused.cuh",
                     "token_indexed_sparse_staple_b200/csrc/common.cuh"],
-        "sha256": "4647dd800c2c0b6da6c48f346d879fd031482b13f079970f888337c404a604b3",
+        "sha256": "e5a5d0c3a590bbed8fc807c3b305e3b19dfef2477a792dcda8bb92b3dd0c630a",
         "profile": "profiles/decode_fused_olmo2_1b_T64.md",
     },
 }

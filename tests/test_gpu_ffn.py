@@ -193,7 +193,7 @@ def test_bf16_decode_saves_g_and_h(stp, ctx):
 
 
 @pytest.mark.parametrize("D,F", [(2048, 1024), (1024, 8192), (4096, 11008)])
-def test_bf16_decode_cluster_split_shapes(stp, ctx, D, F):
+def test_bf16_decode_split_k_shapes(stp, ctx, D, F):
     """Down tiles whose K is split over a few to many blocks, and the 7B shape
     (d_ff 11008 = 172 gate/up tiles over at most 148 blocks, so some blocks
     make two)."""

@@ -97,16 +97,12 @@ struct Params {
   int32_t* err;
 };
 
-// floor(a * b / d) for non-negative a, b and positive d; 32-bit division
-// whenever the product fits (a 64-bit division is a long software sequence).
-__host__ __device__ inline int muldiv(int a, int b, int d) {
-  const uint64_t prod = uint64_t(a) * uint64_t(b);
-  return prod <= 0xffffffffull ? int(uint32_t(prod) / uint32_t(d)) : int(prod / uint64_t(d));
+__host__ __device__ inline int range_start(int c, int U, int grid) {
+  return int((int64_t(c) * U) / grid);
 }
-__host__ __device__ inline int range_start(int c, int U, int grid) { return muldiv(c, U, grid); }
 // The block whose range holds unit x.
 __host__ __device__ inline int owner(int x, int U, int grid) {
-  int c = muldiv(x, grid, U);
+  int c = int((int64_t(x) * grid) / U);
   while (c + 1 < grid && range_start(c + 1, U, grid) <= x) ++c;
   while (c > 0 && range_start(c, U, grid) > x) --c;
   return c;
@@ -170,6 +166,12 @@ __device__ __forceinline__ bool spin_until(const uint32_t* a, uint32_t want, vol
   return true;
 }
 
+// kOrder: blocks order their down steps by lateness.  Only useful when
+// some block makes two or more gate/up tiles (more tiles than blocks); with
+// kOrder false that code is compiled out, which keeps the kernel body small
+// (the gate/up epilogue runs while the memory queues are full, where extra
+// code shows up as instruction-fetch stalls).
+template <bool kOrder>
 __global__ void __launch_bounds__(kThreads, 1)
     decode_fused_kernel(const __grid_constant__ CUtensorMap tm_wg,
                         const __grid_constant__ CUtensorMap tm_wu,
@@ -221,7 +223,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int ngs = (t1 - t0) * p.ug;
   const int nsteps = ngs + (d1 - d0);
   const int nd = d1 - d0;
-  const bool reorder = nd <= kMaxOrder;
+  // With no more gate/up tiles than blocks, every tile is its block's first,
+  // every lateness is 0 and the order is the identity: skip it.
+  const bool reorder = kOrder && nd <= kMaxOrder && p.G > grid;
   const uint32_t ncols = p.N <= 32 ? 32 : (p.N <= 64 ? 64 : (p.N <= 128 ? 128 : 256));
   // Tensor memory: two accumulators of ncols columns, then (p.stage_tmem) as
   // many down-unit weight slots as fit in the 512 columns; a slot holds one
@@ -377,11 +381,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (ok && nd > 0) {
       ok = poll(false);
       if (lane == 0 && ok) ok = issue(true);
-      ok = __shfl_sync(0xffffffffu, ok, 0);
-      const int k1 = __shfl_sync(0xffffffffu, k, 0);
-      if (ok && k1 < nd) {
-        ok = poll(true);
-        if (lane == 0 && ok) issue(false);
+      if (kOrder) {
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        const int k1 = __shfl_sync(0xffffffffu, k, 0);
+        if (ok && k1 < nd) {
+          ok = poll(true);
+          if (lane == 0 && ok) issue(false);
+        }
       }
     }
   } else if (warp == 1) {

@@ -245,14 +245,16 @@ staple_status tc_decode_fwd(const DeviceInfo& di, int T, int D, int F, const voi
   p.part = static_cast<float*>(part);
   p.err = err;
 
-  auto kern = fused::decode_fused_kernel;
-  static std::atomic<uint64_t> attr_done{0};
+  // down-step ordering only where some block makes two or more gate/up tiles
+  const int order = pl.G > pl.grid ? 1 : 0;
+  auto kern = order ? fused::decode_fused_kernel<true> : fused::decode_fused_kernel<false>;
+  static std::atomic<uint64_t> attr_done[2];
   const uint64_t bit = uint64_t(1) << (di.device & 63);
-  if (!(attr_done.load() & bit)) {
+  if (!(attr_done[order].load() & bit)) {
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024) !=
         cudaSuccess)
       return STAPLE_ECUDA;
-    attr_done.fetch_or(bit);
+    attr_done[order].fetch_or(bit);
   }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(pl.grid);
