@@ -90,3 +90,40 @@ def test_host_adamw_rejects_bad_arguments(stp):
                                      buf.ctypes.data, 4, buf.ctypes.data, buf.ctypes.data, 4,
                                      C.byref(hp), 1)
     assert st == stp.STAPLE_EINVAL
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_host_adamw_paths_agree_bit_for_bit(stp, dtype, monkeypatch):
+    """The vector paths (AVX-512, AVX2, where the CPU has them) perform the
+    scalar path's IEEE operations in the same order, so all give the same
+    bits.  F = 100 leaves ragged tails after 16- and 8-lane blocks, and one
+    NaN gradient takes a bf16 value through the NaN branch of the rounding."""
+    V, F, U = 300, 100, 120
+    rng = np.random.default_rng(5)
+    if dtype == "bf16":
+        table0 = syn.bf16_normal((V, F), 0.05, 77)[0]
+        sdt = stp.STAPLE_BF16
+    else:
+        table0 = (rng.standard_normal((V, F)) * 0.05).astype(np.float32)
+        sdt = stp.STAPLE_F32
+    grads = [(rng.standard_normal((U, F)) * 0.1).astype(np.float32) for _ in range(2)]
+    grads[1][3, 17] = np.nan
+    ids = [np.sort(rng.choice(V, U, replace=False)).astype(np.int32) for _ in range(2)]
+    out = {}
+    for isa in ("scalar", "avx2", "avx512"):
+        monkeypatch.setenv("STAPLE_ADAMW_ISA", isa)
+        table = table0.copy()
+        m = np.zeros((V, F), np.float32)
+        v = np.zeros((V, F), np.float32)
+        for step in (1, 2):
+            stp.staple_adamw_rows(table.ctypes.data, F, sdt, F, ids[step - 1], U, grads[step - 1],
+                                  F, m, v, F, step=step, threads=3, **HP)
+        out[isa] = (table.view(np.uint8), m.view(np.uint32), v.view(np.uint32))
+    for isa in ("avx2", "avx512"):
+        for a, b in zip(out[isa], out["scalar"]):
+            np.testing.assert_array_equal(a, b, err_msg=isa)
+    # the NaN reached the table, as a NaN
+    r = ids[1][3]
+    got = out["scalar"][0].view(np.uint16 if dtype == "bf16" else np.float32)[r, 17]
+    val = syn.bf16_bits_to_f32(np.array([got]))[0] if dtype == "bf16" else got
+    assert np.isnan(val)

@@ -1,4 +1,5 @@
-"""Build libstaple.so (the C-ABI library) in-tree for sm_100a with nvcc.
+"""Build libstaple.so (the C-ABI library) in-tree: the CUDA sources for sm_100a
+with nvcc, the plain host C++ sources (*.cpp) with the host compiler.
 
     python -m token_indexed_sparse_staple_b200.build [--verbose-ptxas]
 
@@ -23,6 +24,10 @@ LIB = os.path.join(PKG, "libstaple.so")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 CFLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "-Xcompiler", "-O2",
           "--expt-relaxed-constexpr", "-I", os.path.join(ROOT, "include")]
+# host-only sources: no floating-point contraction, so that scalar and vector
+# paths perform the same IEEE operations
+HOST_CFLAGS = ["-O3", "-std=c++17", "-fPIC", "-ffp-contract=off", "-Wall",
+               "-I", os.path.join(ROOT, "include")]
 
 
 def nvcc() -> str:
@@ -32,8 +37,15 @@ def nvcc() -> str:
     raise RuntimeError("nvcc not found")
 
 
+def cxx() -> str:
+    for cand in (os.environ.get("CXX"), shutil.which("g++"), shutil.which("c++")):
+        if cand and shutil.which(cand):
+            return cand
+    raise RuntimeError("no host C++ compiler found")
+
+
 def sources() -> list[str]:
-    return sorted(os.path.join(CSRC, f) for f in os.listdir(CSRC) if f.endswith(".cu"))
+    return sorted(os.path.join(CSRC, f) for f in os.listdir(CSRC) if f.endswith((".cu", ".cpp")))
 
 
 def _newer(target: str, deps: list[str]) -> bool:
@@ -51,12 +63,15 @@ def build(verbose_ptxas: bool = False, force: bool = False) -> str:
     objs = []
     jobs = []
     for src in sources():
-        obj = os.path.join(BUILD, os.path.basename(src)[:-3] + ".o")
+        obj = os.path.join(BUILD, os.path.splitext(os.path.basename(src))[0] + ".o")
         objs.append(obj)
         if force or verbose_ptxas or not _newer(obj, [src] + headers):
-            cmd = [cc, *ARCH, *CFLAGS, "-c", src, "-o", obj]
-            if verbose_ptxas:
-                cmd += ["-Xptxas", "-v"]
+            if src.endswith(".cpp"):
+                cmd = [cxx(), *HOST_CFLAGS, "-c", src, "-o", obj]
+            else:
+                cmd = [cc, *ARCH, *CFLAGS, "-c", src, "-o", obj]
+                if verbose_ptxas:
+                    cmd += ["-Xptxas", "-v"]
             jobs.append(cmd)
 
     def run(cmd):
@@ -71,7 +86,7 @@ def build(verbose_ptxas: bool = False, force: bool = False) -> str:
             if r.returncode != 0:
                 failed.append(cmd[-3])
     if failed:
-        raise RuntimeError("nvcc failed for: " + ", ".join(failed))
+        raise RuntimeError("compile failed for: " + ", ".join(failed))
     if force or jobs or not _newer(LIB, objs):
         cmd = [cc, *ARCH, "-shared", "-o", LIB, *objs, "-lcudart_static", "-ldl", "-lrt", "-lpthread"]
         r = subprocess.run(cmd, capture_output=True, text=True)
