@@ -470,21 +470,28 @@ def run_train(stp, ctx, w, steps, warmup, world, local):
         staging_h = torch.empty((T, F), dtype=torch.bfloat16).pin_memory()
         staging_d = torch.empty((T, F), dtype=torch.bfloat16, device="cuda")
         list_h = torch.empty(1 + 2 * T, dtype=torch.int32).pin_memory()
-        times = []
-        for _ in range(6):
-            torch.cuda.synchronize()
-            t0 = time.perf_counter()
-            stp.staple_gather_unique_rows_bulk(ctx, cache, tab, r.unique, r.U, T, r.slot, r.miss,
-                                               r.mc, r.rows, staging_h, staging_d, list_h,
-                                               chunk_rows=256, threads=0, stream=stream)
-            stream.synchronize()
-            times.append(time.perf_counter() - t0)
+        by_chunk = {}
+        for chunk in (64, 128, 256, 512):
+            times = []
+            for _ in range(6):
+                torch.cuda.synchronize()
+                t0 = time.perf_counter()
+                stp.staple_gather_unique_rows_bulk(ctx, cache, tab, r.unique, r.U, T, r.slot,
+                                                   r.miss, r.mc, r.rows, staging_h, staging_d,
+                                                   list_h, chunk_rows=chunk, threads=0,
+                                                   stream=stream)
+                stream.synchronize()
+                times.append(time.perf_counter() - t0)
+            by_chunk[chunk] = statistics.median(times[1:])
         assert stp.staple_get_error(ctx, stream) == 0
-        t_bulk = statistics.median(times[1:])
+        best = min(by_chunk, key=by_chunk.get)
+        t_bulk = by_chunk[best]
         nb = int(r.mc.item()) * F * 2
         out["bulk_misses"] = {"ms": t_bulk * 1e3, "miss_bytes": nb, "gbs": nb / t_bulk / 1e9,
-                              "how": "probe + hits + host pack (all threads) + bulk H2D in "
-                                     "256-row chunks + scatter, wall time, median of 5"}
+                              "chunk_rows": best,
+                              "ms_by_chunk_rows": {c: round(t * 1e3, 3) for c, t in by_chunk.items()},
+                              "how": "probe + hits + host pack (all threads) + bulk H2D chunk by "
+                                     "chunk + scatter, wall time, median of 5 per chunk size"}
     finally:
         stp.staple_cache_free(cache)
         stp.staple_table_unregister(tab)
