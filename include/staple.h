@@ -209,7 +209,9 @@ staple_status staple_gather_unique_rows(staple_context* ctx, const staple_cache*
  *   chunk_rows    rows per bulk copy (>= 1)
  * The buffers may be reused by the next call on the same stream.  The table
  * must be in host memory (HOST_PINNED or HOST_REGISTER).  Same results as
- * staple_gather_unique_rows, bit for bit. */
+ * staple_gather_unique_rows, bit for bit.  A miss whose id lies outside
+ * [0, V) is not read: its row is zero-filled and the call returns
+ * STAPLE_EIDRANGE (after queuing the rest). */
 staple_status staple_gather_unique_rows_bulk(staple_context* ctx, const staple_cache* cache,
                                              const staple_table* table, const int32_t* unique,
                                              const int32_t* U_dev, int32_t T, int32_t* slot,

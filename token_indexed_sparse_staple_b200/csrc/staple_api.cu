@@ -412,7 +412,7 @@ staple_status staple_gather_unique_rows_bulk(staple_context* ctx, const staple_c
   STP_CUDA(cudaEventSynchronize(ctx->ev_main));
   // pack the miss rows from the host table in miss order, chunk by chunk;
   // each chunk's copy to the device starts as soon as it is packed
-  const int32_t n = std::min(list_host[0], T);
+  const int32_t n = std::max(0, std::min(list_host[0], T));
   const int32_t* ml = list_host + 1;
   const int32_t* uq = list_host + 1 + T;
   const uint8_t* src = static_cast<const uint8_t*>(table->base);
@@ -424,14 +424,25 @@ staple_status staple_gather_unique_rows_bulk(staple_context* ctx, const staple_c
   // one pool per call: workers claim chunks and mark each one packed; this
   // thread issues the chunks' copies in order as they become ready
   std::atomic<int32_t> next{0};
+  std::atomic<bool> bad_id{false};
   std::vector<std::atomic<int>> packed(size_t(std::max(nchunks, 1)));
   for (auto& a : packed) a.store(0, std::memory_order_relaxed);
   auto worker = [&]() {
     for (int32_t c; (c = next.fetch_add(1)) < nchunks;) {
       const int32_t c1 = std::min(n, (c + 1) * chunk_rows);
-      for (int32_t i = c * chunk_rows; i < c1; ++i)
-        std::memcpy(hs + int64_t(i) * row_bytes, src + int64_t(uq[ml[i]]) * row_bytes,
-                    size_t(row_bytes));
+      for (int32_t i = c * chunk_rows; i < c1; ++i) {
+        // the host reads its own memory here: an id outside the table (the
+        // dedup reports it, it does not clamp) must not steer the read
+        const int32_t pos = ml[i];
+        const int64_t id = pos >= 0 && pos < T ? int64_t(uq[pos]) : -1;
+        uint8_t* dst = hs + int64_t(i) * row_bytes;
+        if (id < 0 || id >= table->V) {
+          std::memset(dst, 0, size_t(row_bytes));
+          bad_id.store(true, std::memory_order_relaxed);
+          continue;
+        }
+        std::memcpy(dst, src + id * row_bytes, size_t(row_bytes));
+      }
       packed[size_t(c)].store(1, std::memory_order_release);
     }
   };
@@ -447,8 +458,9 @@ staple_status staple_gather_unique_rows_bulk(staple_context* ctx, const staple_c
   }
   for (auto& th : pool) th.join();
   if (ce != cudaSuccess) return STAPLE_ECUDA;
-  return stp::launch_scatter_misses(staging_dev, row_bytes, miss_list, miss_count, rows,
-                                    ctx->di.num_sms, st);
+  STP_TRY(stp::launch_scatter_misses(staging_dev, row_bytes, miss_list, miss_count, rows,
+                                     ctx->di.num_sms, st));
+  return bad_id.load() ? STAPLE_EIDRANGE : STAPLE_OK;
 }
 
 staple_status staple_cache_refresh(staple_context* ctx, staple_cache* cache,
