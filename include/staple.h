@@ -370,7 +370,8 @@ typedef struct staple_adamw {
  * table is rounded to nearest, ties to even.
  *   table      host, rows of F values (dtype), row pitch table_pitch elements
  *              (a grouped table's layer: base + layer * F, pitch groups * F)
- *   ids        host int32 [U], distinct (e.g. staple_embed_grad_to_host's ids)
+ *   ids        host int32 [U], distinct, each in [0, V) (e.g. staple_embed_grad_to_host's
+ *              ids); a negative id returns STAPLE_EINVAL before anything changes
  *   grad       host fp32 [U][grad_pitch]: row j is the gradient of row ids[j]
  *   m, v       host fp32 [V][moment_pitch], indexed by row id
  *   threads    host threads to use (<= 0: all hardware threads)

@@ -127,3 +127,17 @@ def test_host_adamw_paths_agree_bit_for_bit(stp, dtype, monkeypatch):
     got = out["scalar"][0].view(np.uint16 if dtype == "bf16" else np.float32)[r, 17]
     val = syn.bf16_bits_to_f32(np.array([got]))[0] if dtype == "bf16" else got
     assert np.isnan(val)
+
+
+def test_host_adamw_rejects_negative_ids_before_updating(stp):
+    F, V, U = 16, 8, 3
+    table = np.ones((V, F), np.float32)
+    m = np.zeros((V, F), np.float32)
+    v = np.zeros((V, F), np.float32)
+    g = np.ones((U, F), np.float32)
+    ids = np.array([1, -2, 5], np.int32)
+    with pytest.raises(stp.StapleError) as ex:
+        stp.staple_adamw_rows(table.ctypes.data, F, stp.STAPLE_F32, F, ids, U, g, F, m, v, F,
+                              step=1, threads=1, **HP)
+    assert ex.value.status == stp.STAPLE_EINVAL
+    assert np.all(table == 1.0) and not np.any(m) and not np.any(v)

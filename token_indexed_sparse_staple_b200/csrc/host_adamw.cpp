@@ -231,6 +231,9 @@ extern "C" staple_status staple_adamw_rows(void* table, int64_t table_pitch, sta
       grad_pitch < F || moment_pitch < F || hp->step < 1 ||
       (dtype != STAPLE_BF16 && dtype != STAPLE_F32))
     return STAPLE_EINVAL;
+  // ids index host memory directly: reject a negative one before any update
+  for (int32_t r = 0; r < U; ++r)
+    if (ids[r] < 0) return STAPLE_EINVAL;
   Job j;
   j.table = static_cast<uint8_t*>(table);
   j.table_pitch = table_pitch;
