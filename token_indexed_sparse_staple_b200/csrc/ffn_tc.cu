@@ -176,6 +176,13 @@ DecodePlan plan_decode(int T, int D, int F, int num_sms) {
   // every block needs at least one down unit (so the blocks covering a down
   // tile are consecutive and each writes its partial slot)
   pl.grid = std::max(1, std::min(std::min(num_sms, kMaxDecodeGrid), pl.Ud));
+  // With more gate/up tiles than blocks, use the fewest blocks that take the
+  // same largest number of tiles each, so that no block makes more tiles
+  // than the others (172 tiles: 86 blocks of two instead of 148 of one or two).
+  if (pl.G > pl.grid) {
+    const int per = cdiv(pl.G, pl.grid);
+    pl.grid = std::max(1, std::min(pl.grid, cdiv(pl.G, per)));
+  }
   pl.maxp_d = piece_bound(pl.ud, pl.Ud);
   pl.counter_bytes = decode_counter_bytes(D, F);
   pl.part_bytes = size_t(pl.Dt * pl.maxp_d) * pl.N * fused::BM * sizeof(float);
