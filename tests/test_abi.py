@@ -71,3 +71,29 @@ def test_null_arguments_are_rejected_before_any_launch(lib):
     assert lib.staple_ffn_fwd(None, 0, 1, 64, 64, None, None, None, None, None, None, None,
                               None, None, None, 0, None) == stp.STAPLE_EINVAL
     assert lib.staple_dedup(None, None, 0, 10, None, None, None, None, None, None) == stp.STAPLE_EINVAL
+
+
+def test_null_arguments_of_the_later_calls_are_rejected(lib):
+    """The calls added after the layer calls validate their arguments before
+    touching a device or host buffer: NULL handles and pointers return
+    STAPLE_EINVAL (no GPU is needed to check that)."""
+    E = stp.STAPLE_EINVAL
+    bf = stp.STAPLE_BF16
+    assert lib.staple_gather_unique_rows(None, None, None, None, None, 4, None, None, None, None,
+                                         None, None) == E
+    assert lib.staple_gather_unique_rows_bulk(None, None, None, None, None, 4, None, None, None,
+                                              None, None, None, None, 256, 0, None) == E
+    assert lib.staple_cache_refresh(None, None, None, None, None, None, None) == E
+    assert lib.staple_embed_bwd(None, bf, 4, 64, 64, None, None, None, None, None, None, None,
+                                None, None, None, None, 0, None) == E
+    assert lib.staple_ffn_bwd(None, bf, 4, 64, 64, None, None, None, None, None, None, None, None,
+                              None, None, None, 0, None) == E
+    assert lib.staple_embed_grad(None, bf, 4, 64, 64, None, 128, None, None, None, None, None,
+                                 None, 0, None) == E
+    assert lib.staple_embed_grad_to_host(None, 64, 4, None, None, None, None, None, None,
+                                         None) == E
+    assert lib.staple_embed_grad_static(bf, 4, 64, None, 64, None, None, None, None, None) == E
+    hp = stp.staple_adamw(1e-3, 0.9, 0.999, 1e-8, 0.0, 1)
+    import ctypes as C
+    assert lib.staple_adamw_rows(None, 4, stp.STAPLE_F32, 4, None, 1, None, 4, None, None, 4,
+                                 C.byref(hp), 1) == E
