@@ -284,6 +284,14 @@ def test_gather_is_a_bit_copy():
     np.testing.assert_array_equal(rows, bits[[0, 7, 39]])
     grouped = oracle.gather_rows(bits, uniq, row_offset=8, width=8)
     np.testing.assert_array_equal(grouped, bits[[0, 7, 39], 8:16])
+    # the cache image: slot k holds the row of the k-th hot id, element by element
+    freq = np.array([3, 9, 1, 9, 0, 4] + [0] * 34, dtype=np.int64)
+    hot, _ = oracle.hot_set(freq, 0.1)                  # 4 slots: ids 1, 3, 5, 0
+    cache = oracle.cache_rows_for(bits, hot)
+    assert list(hot) == [1, 3, 5, 0]
+    for k, i in enumerate([1, 3, 5, 0]):
+        for f in range(bits.shape[1]):
+            assert cache[k, f] == bits[i, f]
 
 
 # --------------------------------------------------------------------------
