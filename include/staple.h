@@ -52,7 +52,10 @@ typedef enum staple_status {
   STAPLE_EINVAL = -1,       /* bad argument: null pointer, size, alignment, flags */
   STAPLE_EIDRANGE = -2,     /* (device-detected) a token id was outside [0, V) */
   STAPLE_ECUDA = -3,        /* a CUDA runtime call failed */
-  STAPLE_ENOMEM = -4,       /* device or pinned-host allocation failed */
+  STAPLE_ENOMEM = -4,       /* device or pinned-host allocation failed.  For tests,
+                               STAPLE_FAIL_ALLOC=<site> in the environment fails
+                               that allocation ("context_err", "cache_rows",
+                               "cache_hash", "cache_hot", or "all") */
   STAPLE_ETIMEOUT = -5,     /* (device-detected) a bounded kernel wait ran out */
   STAPLE_EUNSUPPORTED = -6, /* valid request this build does not implement */
   STAPLE_ENODEV = -7        /* no usable sm_100 device */

@@ -278,3 +278,33 @@ def test_bulk_miss_path_equals_zero_copy(stp, ctx, frac, groups, chunk, threads)
     finally:
         stp.staple_cache_free(cache)
         stp.staple_table_unregister(table)
+
+
+def test_injected_allocation_failures_return_enomem(stp, ctx, monkeypatch):
+    """Fault injection on the host: STAPLE_FAIL_ALLOC names an allocation
+    site, and that allocation fails as if the device were out of memory.  The
+    call returns STAPLE_ENOMEM, frees what it had allocated, and works again
+    once the variable is gone."""
+    V, F = 64, 64
+    table = dev(syn.bf16_normal((V, F), 0.01, 3)[0], "bf16")
+    th = stp.staple_table_register(ctx, table, V * F * 2, V, F, 1, stp.STAPLE_BF16,
+                                   stp.STAPLE_TABLE_DEVICE)
+    freq = np.arange(V, dtype=np.int64)
+    try:
+        for site in ("cache_rows", "cache_hash", "cache_hot", "all"):
+            monkeypatch.setenv("STAPLE_FAIL_ALLOC", site)
+            with pytest.raises(stp.StapleError) as ex:
+                stp.staple_cache_build(ctx, th, freq, 0.25)
+            assert ex.value.status == stp.STAPLE_ENOMEM, site
+        monkeypatch.setenv("STAPLE_FAIL_ALLOC", "context_err")
+        with pytest.raises(stp.StapleError) as ex:
+            stp.staple_context_create(0)
+        assert ex.value.status == stp.STAPLE_ENOMEM
+        monkeypatch.delenv("STAPLE_FAIL_ALLOC")
+        cache = stp.staple_cache_build(ctx, th, freq, 0.25)
+        np.testing.assert_array_equal(stp.staple_cache_hot_ids(cache),
+                                      oracle.hot_set(freq, 0.25)[0])
+        stp.staple_cache_free(cache)
+        assert stp.staple_get_error(ctx) == 0
+    finally:
+        stp.staple_table_unregister(th)

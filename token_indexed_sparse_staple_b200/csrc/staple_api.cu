@@ -8,6 +8,7 @@
 #include <algorithm>
 #include <atomic>
 #include <cmath>
+#include <cstdlib>
 #include <cstring>
 #include <new>
 #include <vector>
@@ -112,6 +113,21 @@ const char* staple_status_string(staple_status s) {
   return "STAPLE_UNKNOWN";
 }
 
+// Every device allocation the library makes goes through here (none happens
+// in a per-step call).  Fault injection for tests, on the host: with
+// STAPLE_FAIL_ALLOC set to an allocation's site name ("context_err",
+// "cache_rows", "cache_hash", "cache_hot") or to "all", that allocation
+// fails as if the device were out of memory.
+static cudaError_t lib_malloc(void** p, size_t bytes, const char* site) {
+  if (const char* e = std::getenv("STAPLE_FAIL_ALLOC")) {
+    if (!std::strcmp(e, site) || !std::strcmp(e, "all")) {
+      *p = nullptr;
+      return cudaErrorMemoryAllocation;
+    }
+  }
+  return cudaMalloc(p, bytes);
+}
+
 staple_status staple_context_create(int device, staple_context** out) {
   if (!out) return STAPLE_EINVAL;
   *out = nullptr;
@@ -125,7 +141,9 @@ staple_status staple_context_create(int device, staple_context** out) {
   if (!c) return STAPLE_ENOMEM;
   c->di.device = device;
   c->di.num_sms = prop.multiProcessorCount;
-  if (cudaMalloc(&c->d_err, sizeof(int32_t)) != cudaSuccess) {
+  if (lib_malloc(reinterpret_cast<void**>(&c->d_err), sizeof(int32_t), "context_err") !=
+      cudaSuccess) {
+    cudaGetLastError();
     delete c;
     return STAPLE_ENOMEM;
   }
@@ -262,10 +280,14 @@ staple_status staple_cache_build(staple_context* ctx, const staple_table* table,
   c->row_bytes = int64_t(table->groups) * table->F * int64_t(esize(table->dtype));
   c->hot.assign(order.begin(), order.begin() + K);
   cudaStream_t st = cs(stream);
-  bool ok = cudaMalloc(&c->rows, size_t(std::max<int64_t>(K, 1)) * c->row_bytes) == cudaSuccess &&
-            cudaMalloc(&c->hkeys, size_t(cap) * 4) == cudaSuccess &&
-            cudaMalloc(&c->hvals, size_t(cap) * 4) == cudaSuccess &&
-            cudaMalloc(&c->hot_dev, size_t(K + 1) * 4) == cudaSuccess;
+  bool ok = lib_malloc(reinterpret_cast<void**>(&c->rows),
+                       size_t(std::max<int64_t>(K, 1)) * c->row_bytes, "cache_rows") == cudaSuccess &&
+            lib_malloc(reinterpret_cast<void**>(&c->hkeys), size_t(cap) * 4, "cache_hash") ==
+                cudaSuccess &&
+            lib_malloc(reinterpret_cast<void**>(&c->hvals), size_t(cap) * 4, "cache_hash") ==
+                cudaSuccess &&
+            lib_malloc(reinterpret_cast<void**>(&c->hot_dev), size_t(K + 1) * 4, "cache_hot") ==
+                cudaSuccess;
   if (!ok) {
     cudaGetLastError();
     staple_cache_free(c);
