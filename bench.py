@@ -239,39 +239,43 @@ def decode_setup(stp, w, local):
     st["y_host"] = torch.empty((S, T, D), dtype=torch.bfloat16).pin_memory()
     st["emb"] = [stp.make_embed(stp.STAPLE_EMBED_TABLE, st["table"], F, st["ids"][s], V)
                  for s in range(S)]
+    st["emb_none"] = stp.make_embed(stp.STAPLE_EMBED_NONE)
     st["wsb"] = stp.staple_workspace_bytes(T, D, F)
     st["ws"] = torch.zeros(st["wsb"], dtype=torch.uint8, device="cuda")
     return st
 
 
-def decode_step(stp, ctx, w, st, s, stream):
+def decode_step(stp, ctx, w, st, s, stream, dense=False):
     r = s % st["R"]
     b = s % st["S"]
-    stp.staple_ffn_fwd(ctx, stp.STAPLE_BF16, w.T, w.D, w.F, st["x"][b], st["emb"][b], st["wg"][r],
+    emb = st["emb_none"] if dense else st["emb"][b]
+    stp.staple_ffn_fwd(ctx, stp.STAPLE_BF16, w.T, w.D, w.F, st["x"][b], emb, st["wg"][r],
                        st["wu"][r], st["wd"][r], st["z"], st["y"], None, None, st["ws"], st["wsb"],
                        stream=stream)
 
 
-def run_decode(stp, ctx, w, args, world, local):
+def capture_steps(step, n, stream):
+    """One CUDA graph of n consecutive steps (step(s) for s in [0, n))."""
     import torch
-    st = decode_setup(stp, w, local)
-    stream = torch.cuda.Stream()
-    G = st["R"] * st["S"] // 4   # steps per captured graph (cycles weights 16x)
-    with torch.cuda.stream(stream):
-        for s in range(max(args.warmup, 3)):
-            decode_step(stp, ctx, w, st, s, stream)
-    torch.cuda.synchronize()
-    assert stp.staple_get_error(ctx, stream) == 0
-    # capture G steps once; replay to cover the K timed steps (untraced)
-    graph = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(graph, stream=stream):
-        for s in range(G):
-            decode_step(stp, ctx, w, st, s, stream)
-    reps = max(1, (args.steps + G - 1) // G)
-    K = reps * G
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        for s in range(n):
+            step(s)
+    return g
+
+
+def time_graph_steps(step, K, G, stream, warmup, world, local):
+    """Exactly K steps: a captured graph of G steps replayed K // G times, then
+    a graph of the K % G remaining steps.  Untraced; CUDA events on the
+    launching stream, max over ranks.  Returns (ms_max, ms_local, clocks)."""
+    import torch
+    full = capture_steps(step, G, stream) if K >= G else None
+    rem = capture_steps(step, K % G, stream) if K % G else None
     with torch.cuda.stream(stream):       # replay() launches on the current stream
-        for _ in range(max(1, args.warmup // G)):
-            graph.replay()
+        for _ in range(max(1, warmup // G)):
+            for g in (full, rem):
+                if g is not None:
+                    g.replay()
     torch.cuda.synchronize()
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier(world)
@@ -280,23 +284,47 @@ def run_decode(stp, ctx, w, args, world, local):
         t0 = time.time()
         with torch.cuda.stream(stream):
             ev0.record(stream)
-            for _ in range(reps):
-                graph.replay()
+            for _ in range(K // G):
+                full.replay()
+            if rem is not None:
+                rem.replay()
             ev1.record(stream)
         torch.cuda.synchronize()
         t1 = time.time()
     ms = ev0.elapsed_time(ev1)
-    assert stp.staple_get_error(ctx, stream) == 0
-    ms_max = max_over_ranks(ms, world)
-    del graph
+    del full, rem
+    return max_over_ranks(ms, world), ms, clk.summary(t0, t1)
+
+
+def run_decode(stp, ctx, w, args, world, local):
+    import torch
+    st = decode_setup(stp, w, local)
+    stream = torch.cuda.Stream()
+    G = st["R"] * st["S"] // 4   # steps per captured graph (cycles weights 16x)
+    K = max(1, args.steps)
+    out = {}
+    for mode in ("staple", "dense"):
+        dense = mode == "dense"
+
+        def step(s, dense=dense):
+            decode_step(stp, ctx, w, st, s, stream, dense)
+
+        with torch.cuda.stream(stream):
+            for s in range(max(args.warmup, 3)):
+                step(s)
+        torch.cuda.synchronize()
+        assert stp.staple_get_error(ctx, stream) == 0
+        ms_max, ms, clocks = time_graph_steps(step, K, G, stream, args.warmup, world, local)
+        assert stp.staple_get_error(ctx, stream) == 0
+        out[mode] = {"ms": ms_max, "ms_local": ms, "clocks": clocks}
+    res = {"K": K, "ms": out["staple"]["ms"], "ms_local": out["staple"]["ms_local"],
+           "clocks": out["staple"]["clocks"], "dense_ms": out["dense"]["ms"],
+           "dense_clocks": out["dense"]["clocks"]}
     # the same steps again with per-kernel CUDA events recorded around every
     # launch: the kernel list and shares (events between launches stop the
     # programmatic overlap of consecutive launches, so these steps are slower)
     stp.staple_trace_enable(ctx, True)
-    tgraph = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(tgraph, stream=stream):
-        for s in range(G):
-            decode_step(stp, ctx, w, st, s, stream)
+    tgraph = capture_steps(lambda s: decode_step(stp, ctx, w, st, s, stream), G, stream)
     with torch.cuda.stream(stream):
         for _ in range(4):
             tgraph.replay()
@@ -306,11 +334,13 @@ def run_decode(stp, ctx, w, args, world, local):
     assert stp.staple_get_error(ctx, stream) == 0
     del tgraph
     kern = kernel_table(trace, G)
-    res = {"K": K, "ms": ms_max, "ms_local": ms, "clocks": clk.summary(t0, t1), "kernels": kern,
-           "launches_per_step": sum(d["launches"] for d in kern.values()) / G}
+    res["kernels"] = kern
+    # a captured launch holds one pair of trace events, re-recorded by every
+    # replay: the records cover the G captured steps once
+    res["launches_per_step"] = sum(d["launches"] for d in kern.values()) / G
     # end to end through the public call with host buffers: H2D of x and ids
     # from pinned memory, the layer, D2H of y, every step
-    Ke = min(K, 4096)
+    Ke = K
     h2d = st["x"][0].numel() * 2 + st["ids"][0].numel() * 4
     d2h = st["y"].numel() * 2
     xd = torch.empty_like(st["x"][0])
@@ -667,6 +697,8 @@ def run_stack_decode(stp, ctx, w, steps, world, local):
             "steps": steps, "ms_per_step": step_ms, "tokens_per_s": job_value(T * steps, ms, world),
             "U_last_step": U, "misses_last_step_per_group": misses,
             "weight_bytes_per_step": wbytes, "weight_gbs": wbytes / (step_ms * 1e-3) / 1e9,
+            "weight_frac": wbytes / (step_ms * 1e-3) / 1e9 / peaks()["hbm_gbs"],
+            "sm_mhz": clk.summary(c0, c1).get("sm_mhz"),
             "table_bytes_host": L * V * F * 2, "setup_s": setup_s,
             "graph": "one CUDA graph per step: dedup, 4 group gathers on side streams, 16 layers",
             "clocks": clk.summary(c0, c1), "kernels_4_traced_steps": kern}
@@ -742,6 +774,7 @@ def run_stack_train(stp, ctx, w, steps, world, local):
             "steps": steps, "ms_per_step": step_ms, "tokens_per_s": job_value(T * steps, ms, world),
             "U_last_step": U, "misses_last_step_per_group": misses,
             "tflops": tf, "tensor_frac_sustained": tf / pk["bf16_tflops_sustained"],
+            "sm_mhz": clk.summary(c0, c1).get("sm_mhz"),
             "host_link": {"h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                           "h2d_gbs": h2d / (step_ms * 1e-3) / 1e9,
                           "d2h_gbs": d2h / (step_ms * 1e-3) / 1e9},
@@ -766,64 +799,97 @@ def blas_threads():
         return os.cpu_count() or 1
 
 
-def oracle_decode_inputs(w):
+def decode_config(w):
+    """The `config` of the decode workload, shared by both arms."""
+    return {"workload": w.name, "T": w.T, "d_model": w.D, "d_ff": w.F, "vocab": w.V,
+            "table": "device (1.64 GB in HBM)", "weights": "random N(0,0.02) bf16",
+            "l2": "inputs larger than L2: 4 rotating weight sets (403 MB) and 64 token batches",
+            "graph": "steps replayed from captured CUDA graphs of 64 steps (+ the remainder)"}
+
+
+def oracle_decode_batch(w):
+    """One decode batch for the oracle, fp64: x, the three weights and the T
+    tokens' gathered table rows (the oracle needs only those rows)."""
     inp = syn.make_layer_inputs(w, with_table=False)
-    rows = {}
-    for b in range(4):
-        ids = syn.zipf_ids(w.T, w.V, w.zipf_s, seed=syn.SEED_IDS + w.index + 7919 * b)
-        rows[b] = ids
+    x, wg, wu, wd = (inp.f64(k) for k in ("x", "w_gate", "w_up", "w_down"))
     E_rows = syn.bf16_normal((w.T, w.F), w.e_std, syn.SEED_E)[1].astype(np.float64)
-    return inp, E_rows
+    return x, wg, wu, wd, E_rows
+
+
+def oracle_decode_tokens(batch, n):
+    """The oracle's forward of the batch's first n tokens."""
+    import oracle
+    x, wg, wu, wd, E_rows = batch
+    oracle.ffn_forward(x[:n], np.arange(n), wg, wu, wd, E_rows[:n])
 
 
 def cpu_baseline_decode(w, seconds=12.0):
     """The oracle's forward on whole 64-token batches for ~seconds of CPU time."""
-    import oracle
-    inp, E_rows = oracle_decode_inputs(w)
-    x, wg, wu, wd = (inp.f64(k) for k in ("x", "w_gate", "w_up", "w_down"))
-    ids = np.arange(w.T)  # rows of E_rows: each token's own (already gathered) table row
+    batch = oracle_decode_batch(w)
     n = 0
     t0 = time.time()
     while time.time() - t0 < seconds or n == 0:
-        oracle.ffn_forward(x, ids, wg, wu, wd, E_rows)
+        oracle_decode_tokens(batch, w.T)
         n += 1
     dt = time.time() - t0
     return {"value": n * w.T / dt, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
             "sample": f"{n} full decode batches of {w.T} tokens (fp64 numpy oracle), {dt:.1f} s"}
 
 
-def reference_arm(w, args):
-    """--impl reference: the oracle as the reference implementation.  Each step
-    is one token's forward on a REF_SLICE-feature slice of d_ff (REF_SLICE/F of
-    a token's work); tokens/s counts those fractions."""
+def cpu_baseline_train(w, seconds=12.0, n=256):
+    """The oracle's forward and full backward (dx, dW_gate, dW_up, dW_down, dE)
+    on the first n tokens of the training microbatch, repeated for ~seconds.
+    The layer's cost grows linearly with its token count, so tokens/s over the
+    sample stands for the whole 16384-token microbatch (an extrapolation)."""
     import oracle
-    inp = syn.make_layer_inputs(w, T=1, with_table=False)
-    x, wg, wu, wd = (inp.f64(k) for k in ("x", "w_gate", "w_up", "w_down"))
-    E = syn.bf16_normal((1, w.F), w.e_std, syn.SEED_E)[1].astype(np.float64)
-    nsl = w.F // REF_SLICE
-
-    def step(s):
-        k = s % nsl
-        sl = slice(k * REF_SLICE, (k + 1) * REF_SLICE)
-        oracle.ffn_forward(x, [0], wg[sl], wu[sl], wd[:, sl], E[:, sl])
-
-    for s in range(args.warmup):
-        step(s)
+    inp = syn.make_layer_inputs(w, T=n, with_table=False, with_dy=True)
+    x, wg, wu, wd, dy = (inp.f64(k) for k in ("x", "w_gate", "w_up", "w_down", "dy"))
+    E_rows = syn.bf16_normal((n, w.F), w.e_std, syn.SEED_E)[1].astype(np.float64)
+    ids = np.arange(n)
+    reps = 0
     t0 = time.time()
-    for s in range(args.steps):
-        step(s)
+    while time.time() - t0 < seconds or reps == 0:
+        fw = oracle.ffn_forward(x, ids, wg, wu, wd, E_rows)
+        oracle.ffn_backward(dy, x, ids, wg, wu, wd, fw)
+        reps += 1
     dt = time.time() - t0
-    tokens = args.steps * REF_SLICE / w.F
-    v = tokens / dt
+    return {"value": reps * n / dt, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
+            "sample": f"{reps} x fwd+bwd of {n} of the {w.T} tokens (fp64 numpy oracle), "
+                      f"{dt:.1f} s; extrapolated to the microbatch (cost linear in tokens)"}
+
+
+def reference_arm(w, args, budget_s=60.0):
+    """--impl reference: the oracle on the decode workload (same config, metric
+    and step count as the CUDA arm).  A step is the oracle's forward of the
+    step's batch; when K whole batches would take more than budget_s, each
+    step is bounded to the batch's first n tokens (n from one timed batch),
+    and tokens/s counts the tokens actually computed."""
+    batch = oracle_decode_batch(w)
+    t0 = time.time()
+    oracle_decode_tokens(batch, w.T)
+    t_batch = max(time.time() - t0, 1e-6)
+    K, W = max(1, args.steps), max(0, args.warmup)
+    n = int(max(1, min(w.T, w.T * budget_s / ((K + W) * t_batch))))
+    for _ in range(W):
+        oracle_decode_tokens(batch, n)
+    t0 = time.time()
+    for _ in range(K):
+        oracle_decode_tokens(batch, n)
+    dt = time.time() - t0
+    v = K * n / dt
+    sample = (f"per step: the forward of {n} of the batch's {w.T} tokens "
+              f"({'the whole batch' if n == w.T else 'bounded sample'}), fp64 numpy oracle")
     return {"metric": METRIC, "value": v, "unit": "tokens/s", "n_gpus": args.gpus,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000 * dt / args.steps,
+            "steps": K, "warmup": W, "ms_per_step": 1000 * dt / K,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-            "data": "synthetic", "impl": "reference",
-            "config": {"workload": w.name, "T": w.T, "d_model": w.D, "d_ff": w.F, "vocab": w.V},
-            "cpu_baseline": {"value": v, "unit": "tokens/s", "kind": "oracle", "cores": blas_threads(),
-                             "sample": f"per step: 1 token x {REF_SLICE} of {w.F} d_ff features "
-                                       f"(1/{nsl} token), fp64 numpy oracle"},
+            "data": "synthetic", "impl": "reference", "config": decode_config(w),
+            "cpu_baseline": {"value": v, "unit": "tokens/s", "kind": "oracle",
+                             "cores": blas_threads(), "sample": sample},
             "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def r3(v):
+    return None if v is None else float(f"{v:.4g}")
 
 
 # --------------------------------------------------------------------------
@@ -841,6 +907,8 @@ def main():
     ap.add_argument("--stack-decode-steps", type=int, default=256)
     ap.add_argument("--stack-train-steps", type=int, default=4)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--detail", default=None,
+                    help="also write every per-kernel table and sub-measurement to this JSON file")
     args = ap.parse_args()
     w = syn.WORKLOADS[args.workload]
 
@@ -860,6 +928,7 @@ def main():
     torch.cuda.set_device(local)
     ctx = stp.staple_context_create(local)
     pk = peaks()
+    detail = {}
     dec = run_decode(stp, ctx, w, args, world, local)
     K = dec["K"]
     value = job_value(w.T * K, dec["ms"], world)
@@ -870,30 +939,37 @@ def main():
     launch_us = dec["ms_local"] * 1000.0 / K if one else kd.get("avg_us", float("nan"))
     ach = dec["alg_bytes"] / (launch_us * 1e-6) / 1e9
     traffic, traffic_src = captured_traffic(dec["roofline_kernel"])
+    dense_us = dec["dense_ms"] * 1000.0 / K
+    step_us = dec["ms"] * 1000.0 / K
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K,
         "warmup": args.warmup, "ms_per_step": dec["ms"] / K, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": w.name, "T": w.T, "d_model": w.D, "d_ff": w.F, "vocab": w.V,
-                   "table": "device (1.64 GB in HBM)", "weights": "random N(0,0.02) bf16",
-                   "l2": "inputs larger than L2: 4 rotating weight sets (403 MB) and 64 token batches",
-                   "graph": "steps replayed from one captured CUDA graph of 64 steps"},
-        "roofline": {"bound": "hbm", "kernel": dec["roofline_kernel"], "achieved": ach,
-                     "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": ach / pk["hbm_gbs"],
+        "config": decode_config(w),
+        "roofline": {"bound": "hbm", "kernel": dec["roofline_kernel"], "achieved": r3(ach),
+                     "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": r3(ach / pk["hbm_gbs"]),
                      "traffic": traffic, "traffic_source": traffic_src,
                      "peak_source": pk["source"] + " (copy bandwidth)",
-                     "alg_bytes_per_launch": dec["alg_bytes"], "note": dec["alg_note"],
-                     "launch_us": launch_us, "traced_launch_us": kd.get("avg_us"),
+                     "alg_bytes_per_launch": dec["alg_bytes"], "launch_us": r3(launch_us),
+                     "traced_launch_us": kd.get("avg_us"),
                      "duration": ("untraced timed step (one launch per step)" if one else
                                   "traced per-launch CUDA events")},
-        "e2e": {"value": job_value(w.T * dec["e2e"]["K"], dec["e2e"]["ms"], world),
+        "e2e": {"value": r3(job_value(w.T * dec["e2e"]["K"], dec["e2e"]["ms"], world)),
                 "unit": "tokens/s", "h2d_bytes_per_step": dec["e2e"]["h2d"],
                 "d2h_bytes_per_step": dec["e2e"]["d2h"], "steps": dec["e2e"]["K"],
-                "how": "per step: pinned H2D of x and ids, staple_ffn_fwd, D2H of y (Python loop)"},
+                "how": "per step: pinned H2D of x and ids, staple_ffn_fwd, D2H of y"},
         "gpu_launches": int(round(dec["launches_per_step"] * K)),
         "clocks": dec["clocks"],
-        "kernels": dec["kernels"],
+        "decode_dense": {"us_per_step": r3(dense_us), "us_per_step_staple": r3(step_us),
+                         "e_path_overhead": r3((step_us - dense_us) / dense_us),
+                         "how": "same kernel and steps with STAPLE_EMBED_NONE (no E rows)"},
     }
+    detail["decode_kernels"] = dec["kernels"]
+    detail["decode_dense_clocks"] = dec["dense_clocks"]
+    detail["roofline_note"] = dec["alg_note"]
+    if world == 1 and rank == 0 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline_decode(w)
+    train = None
     if not args.no_train:
         try:
             wt = syn.WORKLOADS["olmo2-1b-train-layer"]
@@ -914,41 +990,59 @@ def main():
                 zc = tr["misses"] * wt.F * 2 / (k4["avg_us"] * 1e-6) / 1e9
                 link["k4_zero_copy_gbs"] = zc
                 link["k4_frac_of_h2d"] = zc / link["h2d_gbs"]
-            line["train_layer"] = {
-                "workload": wt.name, "tokens_per_s": job_value(wt.T, st_ms, world),
-                "ms_per_step": st_ms, "dense_ms_per_step": de_ms,
-                "e_path_overhead": (st_ms - de_ms) / de_ms, "steps": args.train_steps,
-                "U": tr["U"], "misses": tr["misses"], "bulk_misses": tr.get("bulk_misses"),
-                "tflops": train_flops(wt) / (st_ms / 1000.0) / 1e12,
-                "roofline": {"bound": "tensor", "kernel": top[0], "achieved": tf,
+            layer_tf = train_flops(wt) / (st_ms / 1000.0) / 1e12
+            train = {
+                "workload": wt.name, "tokens_per_s": r3(job_value(wt.T, st_ms, world)),
+                "ms_per_step": r3(st_ms), "dense_ms_per_step": r3(de_ms),
+                "e_path_overhead": r3((st_ms - de_ms) / de_ms), "steps": args.train_steps,
+                "U": tr["U"], "misses": tr["misses"],
+                "tflops": r3(layer_tf),
+                "layer_frac_sustained": r3(layer_tf / pk["bf16_tflops_sustained"]),
+                "roofline": {"bound": "tensor", "kernel": top[0], "achieved": r3(tf),
                              "peak": pk["bf16_tflops_sustained"], "unit": "TFLOP/s",
-                             "frac": None if tf is None else tf / pk["bf16_tflops_sustained"],
+                             "frac": None if tf is None else r3(tf / pk["bf16_tflops_sustained"]),
                              "peak_source": pk["source"] + " (cuBLAS bf16, sustained)"},
-                "clocks": tr["staple"]["clocks"], "kernels": kern, "host_link": link,
-                "host_adamw": adamw,
+                "clocks": tr["staple"]["clocks"],
+                "dense_sm_mhz": tr["dense"]["clocks"].get("sm_mhz"),
             }
+            detail["train_layer"] = {"kernels": kern, "host_link": link, "host_adamw": adamw,
+                                     "bulk_misses": tr.get("bulk_misses"),
+                                     "dense_clocks": tr["dense"]["clocks"]}
         except Exception as ex:  # the decode line must still print
-            line["train_layer"] = {"error": repr(ex)}
+            train = {"error": repr(ex)}
         release_pinned()
+        if world == 1 and rank == 0 and not args.no_cpu_baseline and "error" not in train:
+            train["cpu_baseline"] = cpu_baseline_train(syn.WORKLOADS["olmo2-1b-train-layer"])
     if not args.no_stacks:
         for key, fn, name, n in (("stack_decode", run_stack_decode, "olmo2-7b-decode-16l",
                                   args.stack_decode_steps),
                                  ("stack_train", run_stack_train, "olmo2-1b-train-12l",
                                   args.stack_train_steps)):
             try:
-                line[key] = fn(stp, ctx, syn.WORKLOADS[name], n, world, local)
+                full = fn(stp, ctx, syn.WORKLOADS[name], n, world, local)
+                detail[key] = full
+                line[key] = {k: (r3(v) if isinstance(v, float) else v) for k, v in full.items()
+                             if k in STACK_KEYS}
             except Exception as ex:  # the headline line must still print
                 line[key] = {"error": repr(ex)}
             release_pinned()
-    if world == 1 and rank == 0 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline_decode(w)
+    if train is not None:
+        line["train_layer"] = train   # last, so that a tail of the output holds it
     stp.staple_context_destroy(ctx)
     if rank == 0:
+        if args.detail:
+            with open(args.detail, "w") as f:
+                json.dump({"line": line, "detail": detail}, f, indent=1)
         print(json.dumps(line), flush=True)
     if world > 1:
         import torch.distributed as dist
         barrier(world)
         dist.destroy_process_group()
+
+
+# keys of a stack's result that go into the printed line (the rest: --detail)
+STACK_KEYS = ("workload", "layers", "steps", "ms_per_step", "tokens_per_s", "weight_gbs",
+              "weight_frac", "tflops", "tensor_frac_sustained", "sm_mhz")
 
 
 if __name__ == "__main__":

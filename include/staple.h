@@ -91,6 +91,20 @@ staple_status staple_context_destroy(staple_context* ctx);
  * it.  The only call that waits for the device. */
 staple_status staple_get_error(staple_context* ctx, staple_stream stream, int32_t* device_error);
 
+/* Bound of every wait inside the library's kernels launched for this context
+ * from now on (an mbarrier wait for a copy or an MMA, a spin on a flag another
+ * block raises), in nanoseconds of the GPU's global timer; default 4 s.  A
+ * kernel whose wait runs out records STAPLE_ETIMEOUT in the device error word,
+ * stops its remaining work, lets the copies and MMAs it already issued finish,
+ * frees its tensor memory and returns, so the context stays usable; its
+ * outputs are then undefined.  After STAPLE_ETIMEOUT from a decode-sized call
+ * (see staple_ffn_fwd) zero the workspace's counter head again
+ * (staple_workspace_bytes) before the next such call.  This is the library's
+ * failure detection: no kernel waits without a bound.  EINVAL unless
+ * 1 <= limit_ns <= 60 s.  Host-only; takes effect for later launches (a
+ * captured CUDA graph keeps the limit it was captured with). */
+staple_status staple_set_wait_limit(staple_context* ctx, int64_t limit_ns);
+
 /* Per-kernel timing.  With tracing enabled, every kernel the library launches
  * for this context is bracketed by two CUDA events on its launch stream (a
  * record costs well under a microsecond of device time).  staple_trace_read
@@ -209,7 +223,8 @@ staple_status staple_gather_unique_rows(staple_context* ctx, const staple_cache*
  *   staging_host  page-locked, >= T * groups * F elements
  *   staging_dev   device, >= T * groups * F elements, 16-byte aligned
  *   list_host     page-locked int32 [1 + 2T] (miss count, miss list, ids)
- *   chunk_rows    rows per bulk copy (>= 1)
+ *   chunk_rows    rows per bulk copy (>= 1; a value above the miss count
+ *                 means one copy of all misses)
  * The buffers may be reused by the next call on the same stream.  The table
  * must be in host memory (HOST_PINNED or HOST_REGISTER).  Same results as
  * staple_gather_unique_rows, bit for bit.  A miss whose id lies outside
@@ -265,7 +280,12 @@ typedef struct staple_embed {
   int64_t n_rows;        /* rows addressable through index */
 } staple_embed;
 
-/* Forward pass of one layer.
+/* Forward pass of one layer: the pretrained SwiGLU FFN with the token-indexed
+ * row E[id] added to the up-projection's output, inside the SiLU gate
+ * (abstract: the embeddings join the FFN as a residual pathway; ai4snews
+ * summary, Interpretation: the zero-initialised table leaves the seed FFN's
+ * output unchanged, and the gate makes the added row context-dependent):
+ *     g = W_gate x,  h = W_up x + E[id],  z = SiLU(g) * h,  y = W_down z.
  *   x[T][D], w_gate[F][D], w_up[F][D], w_down[D][F]   inputs (dtype)
  *   z[T][F]     out: SiLU(g) * h, the down projection's input (kept for dW_down)
  *   y[T][D]     out: layer output
@@ -273,10 +293,13 @@ typedef struct staple_embed {
  *               both NULL for inference
  * bf16 needs D and F multiples of 64 and 16-byte aligned pointers;
  * T >= 0.  fp32 needs F a multiple of 8.
- * bf16 with 1 <= T <= 256 (decode sizes) runs one persistent kernel that
+ * bf16 with 1 <= T <= 256 (decode sizes; the pages serve at batch 64 on one
+ * B200: thelatestinai listing, Table 4) runs one persistent kernel that
  * streams both projections' weights across all SMs and needs the workspace
  * (staple_workspace_bytes, zero-filled once); larger T runs the tiled GEMMs
- * and ignores it. */
+ * and ignores it.  That kernel's blocks wait on one another, so its whole
+ * grid must be resident at once: STAPLE_EUNSUPPORTED when the device cannot
+ * hold it (the grid exceeds the SMs times the blocks per SM). */
 staple_status staple_ffn_fwd(staple_context* ctx, staple_dtype dtype, int32_t T, int32_t D,
                              int32_t F, const void* x, const staple_embed* embed,
                              const void* w_gate, const void* w_up, const void* w_down, void* z,
@@ -285,7 +308,11 @@ staple_status staple_ffn_fwd(staple_context* ctx, staple_dtype dtype, int32_t T,
 
 /* ----------------------------------------------------------- FFN backward */
 
-/* Table gradient of one layer (spec call: dY -> U gradient rows).
+/* Table gradient of one layer: dY -> one gradient row per distinct id of the
+ * batch (AI Radio episode, paper summary: during training only the U x d_ff
+ * rows of the batch's distinct ids exist on the GPU, as the trainable leaf,
+ * so each gets one accumulated gradient row; thelatestinai listing,
+ * retrieval-path table: the one dedup's inverse map serves every layer).
  * Computes dz = dY W_down, dh = dz * SiLU(g), dg = dz * h * SiLU'(g) into
  * dgh[T][2F] (dg in columns [0, F), dh in [F, 2F)), then
  *   dE[j][f] = sum of dh[i][f] over the tokens i of segment j (seg_off /
@@ -399,13 +426,16 @@ staple_status staple_adamw_rows(void* table, int64_t table_pitch, staple_dtype d
  *               (e.g. the dh half of staple_embed_bwd's dgh: base + F, ld = 2F)
  *   sorted_pos, inverse, seg_off   from staple_dedup for the same ids
  *   dE          out, fp32 [>= U][F]; rows >= U untouched
- * Runs on the current device, on `stream`.  The first call on a device looks
- * up the array's device address (cudaGetSymbolAddress); make that first call
- * before any stream capture.  Every call shares the one array, so calls that
- * overlap on the GPU race; nothing in it needs to start at zero.
- * Returns STAPLE_EINVAL for bad arguments and for a size beyond the array:
- * 2 * ceil(T / 64) * F * 4 bytes must not exceed 16 MiB (T <= 16384 at
- * F = 8192).  F must be a multiple of 8. */
+ * Runs on the current device, on `stream`.  The first call in each CUDA
+ * context of a device looks up the array's device address
+ * (cudaGetSymbolAddress) and keeps it for that context; make that first call
+ * before any stream capture (and again after a cudaDeviceReset, which starts
+ * a new context).  Every call shares the one array, so calls that overlap on
+ * the GPU race; nothing in it needs to start at zero.
+ * Returns STAPLE_EUNSUPPORTED, before any pointer is looked at, for a size
+ * beyond the array or beyond one dedup: T <= 32768 and
+ * 2 * ceil(T / 64) * F * 4 bytes <= 16 MiB (T <= 16384 at F = 8192), and
+ * STAPLE_EINVAL for other bad arguments.  F must be a multiple of 8. */
 staple_status staple_embed_grad_static(staple_dtype dtype, int32_t T, int32_t F, const void* dh,
                                        int64_t ld, const int32_t* sorted_pos,
                                        const int32_t* inverse, const int32_t* seg_off, float* dE,

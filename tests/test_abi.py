@@ -97,3 +97,25 @@ def test_null_arguments_of_the_later_calls_are_rejected(lib):
     import ctypes as C
     assert lib.staple_adamw_rows(None, 4, stp.STAPLE_F32, 4, None, 1, None, 4, None, None, 4,
                                  C.byref(hp), 1) == E
+
+
+def test_static_scratch_refuses_sizes_beyond_it(lib):
+    """staple_embed_grad_static checks its sizes before anything else, so the
+    refusal needs no GPU.  All pointers are NULL: without the size guard the
+    call would stop at the NULL check with STAPLE_EINVAL instead, so only the
+    guard can give STAPLE_EUNSUPPORTED (and no launch can follow)."""
+    U = stp.STAPLE_EUNSUPPORTED
+    bf = stp.STAPLE_BF16
+
+    def call(T, F):
+        return lib.staple_embed_grad_static(bf, T, F, None, F, None, None, None, None, None)
+
+    # 2 * ceil(T / 64) * F * 4 bytes against the 16 MiB array
+    assert call(16385, 8192) == U
+    assert call(16448, 8192) == U
+    assert call(8193, 16384) == U
+    # longer than one dedup (32768 tokens), though small F fits the array
+    assert call(32769, 8) == U
+    # at the limits the size passes and the NULL pointers are what is refused
+    assert call(16384, 8192) == stp.STAPLE_EINVAL
+    assert call(32768, 8) == stp.STAPLE_EINVAL

@@ -107,6 +107,22 @@ def test_bf16_zero_table_is_bitwise_dense(stp, ctx):
         np.testing.assert_array_equal(got[k] + 0.0, dense[k] + 0.0, err_msg=k)
 
 
+@pytest.mark.parametrize("T", [64, 300])
+def test_bf16_dense_run_matches_oracle(stp, ctx, T):
+    """The E path switched off (STAPLE_EMBED_NONE), the comparison run of the
+    "within 3%" claim (ai4snews summary, Interpretation), is the dense SwiGLU
+    FFN: the fused decode kernel (T = 64) and the tiled GEMMs (T = 300)
+    against the oracle with no table, forward and backward."""
+    w = _bf16_workload(T, 256, 576, 4000)
+    inp = syn.make_layer_inputs(w)
+    got = run_layer(stp, ctx, inp, w.D, w.F, w.V, embed="none")
+    x, wg, wu, wd = (inp.f64(k) for k in ("x", "w_gate", "w_up", "w_down"))
+    fw = oracle.ffn_forward(x, inp.ids, wg, wu, wd, None)
+    ref = {**fw, **oracle.ffn_backward(inp.f64("dy"), x, inp.ids, wg, wu, wd, fw)}
+    np.testing.assert_array_equal(got["unique"], ref["unique"])
+    compare(got, ref, TOL["bf16"], FWD + SAVED + BWD)
+
+
 def test_bf16_gathered_rows_equal_table_rows(stp, ctx):
     w = _bf16_workload(640, 256, 512, 3000)
     inp = syn.make_layer_inputs(w)

@@ -223,7 +223,10 @@ def test_cache_refresh_after_host_adamw(stp, ctx):
 
 
 @pytest.mark.parametrize("frac,groups,chunk,threads", [(0.05, 1, 256, 4), (0.0, 1, 7, 1),
-                                                       (0.05, 4, 1, 0), (1.0, 2, 64, 2)])
+                                                       (0.05, 4, 1, 0), (1.0, 2, 64, 2),
+                                                       # one chunk larger than the batch, and
+                                                       # the largest chunk size the call takes
+                                                       (0.05, 1, 5000, 2), (0.0, 1, 2**31 - 1, 0)])
 def test_bulk_miss_path_equals_zero_copy(stp, ctx, frac, groups, chunk, threads):
     """The prefill path (misses packed on the host, bulk copy, scatter) gives
     the same rows, hit/miss map and miss list as the zero-copy gather, bit for

@@ -6,7 +6,7 @@ owned by another allocator, or they must not call cudaMalloc because it
 synchronizes the device, or they only hold the buffers a host hands them): its
 scratch is built into the library.  Two calls in a row must both reproduce the
 dE of staple_embed_bwd for the same dh, and a size beyond the built-in scratch
-must be refused before anything runs.  This file is collected last so that a
+must be refused (STAPLE_EUNSUPPORTED) before anything runs.  This file is collected last so that a
 run stopping at the first failure has already run every other test."""
 import ctypes as C
 
@@ -75,9 +75,12 @@ def test_static_scratch_at_its_largest_size(stp, ctx):
     _case(stp, ctx, T=16384, D=64, F=8192, V=100352, seed=12)
 
 
-def test_static_scratch_refuses_larger_sizes(stp):
+def test_static_scratch_refuses_larger_sizes(stp, ctx):
+    """An oversize request is refused with STAPLE_EUNSUPPORTED before any
+    pointer is looked at or anything is launched (the NULL pointers would give
+    STAPLE_EINVAL otherwise), and the next call still works."""
     lib = stp.lib()
-    one = C.c_void_p(256)   # never dereferenced: the size check comes first
-    st = lib.staple_embed_grad_static(stp.STAPLE_BF16, 16385, 8192, one, 16384, one, one, one,
-                                      one, None)
-    assert st == stp.STAPLE_EINVAL
+    st = lib.staple_embed_grad_static(stp.STAPLE_BF16, 16448, 8192, None, 8192, None, None, None,
+                                      None, None)
+    assert st == stp.STAPLE_EUNSUPPORTED
+    _case(stp, ctx, T=700, D=64, F=256, V=3000, seed=13)

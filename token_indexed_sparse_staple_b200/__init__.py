@@ -95,6 +95,11 @@ def staple_get_error(ctx: int, stream=None) -> int:
     return e.value
 
 
+def staple_set_wait_limit(ctx: int, limit_ns: int) -> None:
+    """Bound of every kernel wait of later launches, in ns (see include/staple.h)."""
+    _ok(lib().staple_set_wait_limit(ctx, int(limit_ns)), "staple_set_wait_limit")
+
+
 def staple_trace_enable(ctx: int, enable: bool = True) -> None:
     _ok(lib().staple_trace_enable(ctx, int(bool(enable))), "staple_trace_enable")
 

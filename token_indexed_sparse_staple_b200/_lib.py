@@ -40,6 +40,7 @@ SIGNATURES = {
     "staple_context_create": (c_status, [C.c_int, P(vp)]),
     "staple_context_destroy": (c_status, [vp]),
     "staple_get_error": (c_status, [vp, vp, P(i32)]),
+    "staple_set_wait_limit": (c_status, [vp, i64]),
     "staple_trace_enable": (c_status, [vp, C.c_int]),
     "staple_trace_read": (c_status, [vp, vp, i32, P(i32)]),
     "staple_table_register": (c_status, [vp, vp, sz, i64, i32, i32, C.c_int, u32, P(vp)]),

@@ -18,8 +18,14 @@ __device__ __forceinline__ void report(int32_t* err, int32_t code) {
   if (err) atomicCAS(err, 0, code);
 }
 
-// A bounded wait gives up after this many nanoseconds of %globaltimer.
-constexpr uint64_t kWaitLimitNs = 4000000000ull;
+// A bounded wait gives up after the context's wait limit, in nanoseconds of
+// %globaltimer (staple_set_wait_limit; the kernels receive it in their
+// parameters).
+// Bound of the waits on the abort path, for asynchronous work the block has
+// already issued (copies, MMAs) and must let finish before its shared and
+// tensor memory go away.  That work completes in microseconds; the bound only
+// keeps a logic error from turning into a hang.
+constexpr uint64_t kDrainNs = 20000000ull;
 
 __device__ __forceinline__ uint64_t globaltimer() {
   uint64_t t;
@@ -91,20 +97,44 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 
 // Wait for phase `parity` of `bar` to complete.  Gives up (returns false)
 // when another role of the block has already given up (*abort set) or when
-// the wait exceeds kWaitLimitNs; in the latter case it sets *abort and
-// records STAPLE_ETIMEOUT in the device error word.
+// the wait exceeds limit_ns; in the latter case it sets *abort and records
+// STAPLE_ETIMEOUT in the device error word.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
-                                          int32_t* err) {
+                                          int32_t* err, uint64_t limit_ns) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer();
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
     if (*abort) return false;
-    if (globaltimer() - t0 > kWaitLimitNs) {
+    if (globaltimer() - t0 > limit_ns) {
       *abort = 1;
       report(err, STAPLE_ETIMEOUT);
       return false;
     }
+  }
+}
+
+// Abort path: wait (bounded by kDrainNs) for phase `parity` of `bar`.
+__device__ __forceinline__ void mbar_drain(uint64_t* bar, uint32_t parity) {
+  if (mbar_try_wait(bar, parity)) return;
+  const uint64_t t0 = globaltimer();
+  while (!mbar_try_wait(bar, parity) && globaltimer() - t0 < kDrainNs) {
+  }
+}
+
+// Abort path of a TMA producer: stage `s` / phase `ph` is the next one it
+// would have filled and `issued` the fills so far.  Waits until every fill
+// still possibly in flight (the last min(issued, stages) ones) has landed.
+// Fills that a consumer already took have completed, so this also costs
+// nothing on the normal path.
+__device__ __forceinline__ void drain_ring(uint64_t* full, int stages, int s, uint32_t ph,
+                                           int issued) {
+  for (int k = 0; k < stages && k < issued; ++k) {
+    if (--s < 0) {
+      s = stages - 1;
+      ph ^= 1;
+    }
+    mbar_drain(&full[s], ph);
   }
 }
 

@@ -95,6 +95,7 @@ struct Params {
   uint32_t* queue;     // [2]: next chunk to reduce, events seen
   float* part;         // [Dt * maxp_d][N][128]
   int32_t* err;
+  uint64_t wait_ns;    // bound of every wait and flag spin (STAPLE_ETIMEOUT past it)
 };
 
 __host__ __device__ inline int range_start(int c, int U, int grid) {
@@ -149,15 +150,15 @@ __device__ __forceinline__ void add4(float4& a, const float4 b) {
   a.w += b.w;
 }
 // Bounded spin until *a >= want (acquire).  False (and *abort set, the
-// error word written) after kWaitLimitNs.
+// error word written) after limit_ns.
 __device__ __forceinline__ bool spin_until(const uint32_t* a, uint32_t want, volatile int* abort,
-                                           int32_t* err) {
+                                           int32_t* err, uint64_t limit_ns) {
   if (ld_acquire(a) >= want) return true;
   const uint64_t t0 = globaltimer();
   while (ld_acquire(a) < want) {
     __nanosleep(64);
     if (*abort) return false;
-    if (globaltimer() - t0 > kWaitLimitNs) {
+    if (globaltimer() - t0 > limit_ns) {
       *abort = 1;
       report(err, STAPLE_ETIMEOUT);
       return false;
@@ -203,6 +204,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   int* s_epi_fail = s_flag + 1;
   uint64_t* rbar = reinterpret_cast<uint64_t*>(tail + 320);  // partial slices landed
   uint64_t* obar = reinterpret_cast<uint64_t*>(tail + 328);  // down-step order written
+  uint64_t* dbar = reinterpret_cast<uint64_t*>(tail + 336);  // MMA drain before TMEM is freed
   // Down-step order (blocks with at most kMaxOrder down units): within each
   // piece, the units whose z is ready first (lateness 0) come first.  The
   // weight loader, the activation loader and the MMA thread all follow it.
@@ -249,6 +251,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     mbar_init(rbar, 1);
     mbar_init(obar, 1);
+    mbar_init(dbar, 1);
     *abort_flag = 0;
     *s_epi_fail = 0;
     fence_barrier_init();
@@ -298,9 +301,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint64_t once = l2_policy_evict_first();  // weights are read once per call
       int s = 0;
       uint32_t ph = 0;
+      int issued = 0;
       for (int i = 0; i < nsteps; ++i) {
-        if (i == ngs && ordered && !mbar_wait(obar, 0, abort_flag, p.err)) break;
-        if (!mbar_wait(&emptyA[s], ph ^ 1, abort_flag, p.err)) break;
+        if (i == ngs && ordered && !mbar_wait(obar, 0, abort_flag, p.err, p.wait_ns)) break;
+        if (!mbar_wait(&emptyA[s], ph ^ 1, abort_flag, p.err, p.wait_ns)) break;
         mbar_arrive_expect_tx(&fullA[s], a_stage);
         uint8_t* a = sA + s * a_stage;
         for (int j = 0; j < p.sub; ++j) {
@@ -315,27 +319,32 @@ __global__ void __launch_bounds__(kThreads, 1)
             tma_load_3d_hint(&tm_wd, &fullA[s], a, 0, tile * BM, u * p.sub, once);
           }
         }
+        ++issued;
         if (++s == S) {
           s = 0;
           ph ^= 1;
         }
       }
+      // after an abort, copies still in flight land before the block exits
+      drain_ring(fullA, S, s, ph, issued);
     }
   } else if (warp == 2) {
     // ---------------------------------------------------- activation (B) loads
     grid_dep_wait();
     int s = 0;
     uint32_t ph = 0;
+    int issued = 0;   // lane 0's fills
     bool ok = true;
     // x for the gate/up steps
     if (lane == 0) {
       for (int i = 0; i < ngs && ok; ++i) {
-        ok = mbar_wait(&emptyB[s], ph ^ 1, abort_flag, p.err);
+        ok = mbar_wait(&emptyB[s], ph ^ 1, abort_flag, p.err, p.wait_ns);
         if (!ok) break;
         const int u = i % p.ug;
         uint8_t* b = sB + s * b_stage;
         mbar_arrive_expect_tx(&fullB[s], b_stage);
         tma_load_3d(&tm_x, &fullB[s], b, 0, 0, u * p.sub);
+        ++issued;
         if (++s == SB) {
           s = 0;
           ph ^= 1;
@@ -356,7 +365,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int f_lo = ((d0 + k) % p.ud) * p.sub * BK;
         const int f_hi = min(p.F, f_lo + p.sub * BK);
         for (int t = f_lo / 64; t <= (f_hi - 1) / 64 && mine; ++t)
-          mine = spin_until(&p.ready[t], 1u, abort_flag, p.err);
+          mine = spin_until(&p.ready[t], 1u, abort_flag, p.err, p.wait_ns);
       }
       return __all_sync(0xffffffffu, mine);
     };
@@ -366,10 +375,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (; k < nd; ++k) {
         const int x = unit(k);
         if (stop_at_late && reorder && s_late[x - d0] != 0) break;
-        if (!mbar_wait(&emptyB[s], ph ^ 1, abort_flag, p.err)) return false;
+        if (!mbar_wait(&emptyB[s], ph ^ 1, abort_flag, p.err, p.wait_ns)) return false;
         uint8_t* b = sB + s * b_stage;
         mbar_arrive_expect_tx(&fullB[s], b_stage);
         tma_load_3d(&tm_z, &fullB[s], b, 0, 0, (x % p.ud) * p.sub);
+        ++issued;
         if (++s == SB) {
           s = 0;
           ph ^= 1;
@@ -377,7 +387,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       return true;
     };
-    if (ok && ordered) ok = __all_sync(0xffffffffu, mbar_wait(obar, 0, abort_flag, p.err));
+    if (ok && ordered)
+      ok = __all_sync(0xffffffffu, mbar_wait(obar, 0, abort_flag, p.err, p.wait_ns));
     if (ok && nd > 0) {
       ok = poll(false);
       if (lane == 0 && ok) ok = issue(true);
@@ -390,6 +401,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
     }
+    if (lane == 0) drain_ring(fullB, SB, s, ph, issued);
   } else if (warp == 1) {
     if (lane == 0) {
       // ---------------------------------------------------------------- MMA
@@ -406,7 +418,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           // they land; each copy's commit frees its ring stage for the next
           // unit's weights, so W_down streams while z is still being made.
           for (int k = 0; k < n_stage; ++k) {
-            if (!mbar_wait(&fullA[sa], pha, abort_flag, p.err)) {
+            if (!mbar_wait(&fullA[sa], pha, abort_flag, p.err, p.wait_ns)) {
               ok = false;
               break;
             }
@@ -435,14 +447,15 @@ __global__ void __launch_bounds__(kThreads, 1)
           nunits = min(d1, (x / p.ud + 1) * p.ud) - x;
         }
         const int buf = piece & 1;
-        if (!mbar_wait(&tempty[buf], ((piece >> 1) & 1) ^ 1, abort_flag, p.err)) break;
+        if (!mbar_wait(&tempty[buf], ((piece >> 1) & 1) ^ 1, abort_flag, p.err, p.wait_ns))
+          break;
         tc_fence_after();
         const uint32_t dacc = tmem_base + uint32_t(buf) * ncols;
         for (int i = 0; i < nunits; ++i) {
           const int du = i0 + i - ngs;  // down unit index (negative for gate/up)
           const bool staged = du >= 0 && du < n_stage;
-          if ((!staged && !mbar_wait(&fullA[sa], pha, abort_flag, p.err)) ||
-              !mbar_wait(&fullB[sb], phb, abort_flag, p.err)) {
+          if ((!staged && !mbar_wait(&fullA[sa], pha, abort_flag, p.err, p.wait_ns)) ||
+              !mbar_wait(&fullB[sb], phb, abort_flag, p.err, p.wait_ns)) {
             ok = false;
             break;
           }
@@ -492,6 +505,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         i0 += nunits;
         if (ok) umma_commit(&tfull[buf]);
       }
+      // every MMA and tensor-memory copy issued here completes before tensor
+      // memory and the ring are released (after an abort some may still run)
+      umma_commit(dbar);
+      mbar_drain(dbar, 0);
     }
   } else {
     // ----------------------------------------------------------- epilogue
@@ -538,7 +555,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       const int buf = piece & 1;
-      const bool ok = mbar_wait(&tfull[buf], (piece >> 1) & 1, abort_flag, p.err);
+      const bool ok = mbar_wait(&tfull[buf], (piece >> 1) & 1, abort_flag, p.err, p.wait_ns);
       if (!__all_sync(0xffffffffu, ok) && lane == 0) *s_epi_fail = 1;
       epi_bar();
       if (*s_epi_fail) {
@@ -596,7 +613,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int idx = blockIdx.x - owner(tile * p.ud, p.Ud, grid);
       x = x_end;
       const int buf = piece & 1;
-      const bool ok = mbar_wait(&tfull[buf], (piece >> 1) & 1, abort_flag, p.err);
+      const bool ok = mbar_wait(&tfull[buf], (piece >> 1) & 1, abort_flag, p.err, p.wait_ns);
       if (!__all_sync(0xffffffffu, ok) && lane == 0) *s_epi_fail = 1;
       epi_bar();
       if (*s_epi_fail) {
@@ -635,6 +652,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint8_t* rbuf = sA;
     const int slice = p.N * kChunkRows * 4;   // bytes of one piece's [N][16] fp32 slice
     uint32_t rph = 0;
+    // thread et == 0 issues the slice loads; a batch it issued and has not
+    // seen land (after an abort) is waited for before the block exits
+    bool r_pending = false;
+    uint32_t r_phase = 0;
     auto event = [&]() {
       if (atomicAdd(&p.queue[1], 1u) == nevents - 1) {
         for (int k = 0; k < p.Dt; ++k) p.cnt[k] = 0u;
@@ -657,12 +678,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int tl = code / chunks_per_tile;
           const int first = owner(tl * p.ud, p.Ud, grid);
           const int np = owner((tl + 1) * p.ud - 1, p.Ud, grid) - first + 1;
-          if (!spin_until(&p.cnt[tl], uint32_t(np), abort_flag, p.err)) {
+          if (!spin_until(&p.cnt[tl], uint32_t(np), abort_flag, p.err, p.wait_ns)) {
             code = -1;
           } else {
             fence_async_global();
             const int nb = min(np, p.rcap);
             const int r0 = (code % chunks_per_tile) * kChunkRows;
+            r_pending = true;
+            r_phase = rph;
             mbar_arrive_expect_tx(rbar, uint32_t(nb * slice));
             for (int i = 0; i < nb; ++i)
               tma_load_2d(&tm_part, rbar, rbuf + i * slice, r0, (tl * p.maxp_d + i) * p.N);
@@ -692,13 +715,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (i0 > 0) {
           epi_bar();  // the previous batch has been read
           if (et == 0) {
+            r_pending = true;
+            r_phase = rph;
             mbar_arrive_expect_tx(rbar, uint32_t(nb * slice));
             for (int i = 0; i < nb; ++i)
               tma_load_2d(&tm_part, rbar, rbuf + i * slice, r0,
                           (tile * p.maxp_d + i0 + i) * p.N);
           }
         }
-        ok = mbar_wait(rbar, rph, abort_flag, p.err);
+        ok = mbar_wait(rbar, rph, abort_flag, p.err, p.wait_ns);
+        if (ok && et == 0) r_pending = false;
         rph ^= 1u;
         if (!__all_sync(0xffffffffu, ok) && lane == 0) *s_epi_fail = 1;
         epi_bar();
@@ -735,6 +761,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (et == 0) event();
     }
+    if (et == 0 && r_pending) mbar_drain(rbar, r_phase);
   }
 
   tc_fence_before();

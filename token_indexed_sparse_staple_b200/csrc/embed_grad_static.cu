@@ -11,11 +11,15 @@
 // The array is part of the library's device image: every GPU that loads the
 // library holds kStaticScratchBytes until the process exits.  Host code may
 // not use the array's name as a device address (on the host it names a
-// stand-in object), so its device address is looked up once per device with
-// cudaGetSymbolAddress, with that device current, on the first call.  Every
-// call shares the one array: calls that overlap on the GPU (on different
-// streams without ordering) race on it.  Nothing in it needs to start at zero:
-// each call writes every partial slot it later reads.
+// stand-in object), so its device address is looked up with
+// cudaGetSymbolAddress, with the device current, on the first call in each
+// CUDA context of a device and kept for later calls in that context.  A new
+// context on the device (after cudaDeviceReset, for instance) loads the
+// library's device image again, possibly elsewhere, so the address is looked
+// up again there.  Every call shares the one array: calls that overlap on the
+// GPU (on different streams without ordering) race on it.  Nothing in it
+// needs to start at zero: each call writes every partial slot it later reads.
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include <mutex>
@@ -30,20 +34,43 @@ constexpr int kMaxDevices = 64;
 
 static __device__ __align__(256) float g_seg_scratch[kStaticScratchBytes / sizeof(float)];
 
+using CtxGetCurrent = CUresult (*)(CUcontext*);
+
 std::mutex g_addr_mu;
 float* g_addr[kMaxDevices] = {};
+CUcontext g_addr_ctx[kMaxDevices] = {};
 
-// Device address of g_seg_scratch on `device` (which must be current).
+// The current CUDA context of the calling thread, through the driver entry
+// point (the runtime has made it current by the time this runs).
+CUcontext current_context() {
+  static CtxGetCurrent fn = [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &f, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return CtxGetCurrent(nullptr);
+    return reinterpret_cast<CtxGetCurrent>(f);
+  }();
+  CUcontext c = nullptr;
+  if (!fn || fn(&c) != CUDA_SUCCESS) return nullptr;
+  return c;
+}
+
+// Device address of g_seg_scratch on `device` (which must be current), looked
+// up once per context of that device.
 staple_status scratch_address(int device, float** out) {
   std::lock_guard<std::mutex> lock(g_addr_mu);
   if (device < 0 || device >= kMaxDevices) return STAPLE_EUNSUPPORTED;
-  if (!g_addr[device]) {
+  const CUcontext ctx = current_context();
+  if (!g_addr[device] || ctx == nullptr || ctx != g_addr_ctx[device]) {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_seg_scratch) != cudaSuccess || p == nullptr) {
       cudaGetLastError();
+      g_addr[device] = nullptr;
       return STAPLE_ECUDA;
     }
     g_addr[device] = static_cast<float*>(p);
+    g_addr_ctx[device] = ctx;
   }
   *out = g_addr[device];
   return STAPLE_OK;
@@ -60,11 +87,14 @@ extern "C" staple_status staple_embed_grad_static(staple_dtype dtype, int32_t T,
                                                   float* dE, staple_stream stream) {
   if (dtype != STAPLE_BF16 && dtype != STAPLE_F32) return STAPLE_EINVAL;
   if (T < 0 || F <= 0 || (F % 8) != 0 || ld < F) return STAPLE_EINVAL;
+  // Sizes are checked before the pointers: a request the built-in scratch
+  // cannot hold (or longer than a dedup can produce) is refused as such.
+  if (T > stp::kMaxDedupT || stp::seg_reduce_workspace(T, F) > kStaticScratchBytes)
+    return STAPLE_EUNSUPPORTED;
   if (T == 0) return STAPLE_OK;
   if (!dh || !sorted_pos || !inverse || !seg_off || !dE) return STAPLE_EINVAL;
   const size_t esz = dtype == STAPLE_BF16 ? 2 : 4;
   if (!aligned16(dh) || !aligned16(dE) || (size_t(ld) * esz) % 16 != 0) return STAPLE_EINVAL;
-  if (stp::seg_reduce_workspace(T, F) > kStaticScratchBytes) return STAPLE_EINVAL;
   int device = 0;
   if (cudaGetDevice(&device) != cudaSuccess) return STAPLE_ECUDA;
   float* part = nullptr;

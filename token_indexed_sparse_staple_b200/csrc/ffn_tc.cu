@@ -11,7 +11,9 @@
 
 #include <algorithm>
 #include <atomic>
+#include <map>
 #include <mutex>
+#include <tuple>
 
 #include "decode_fused.cuh"
 #include "gemm_tc.cuh"
@@ -114,6 +116,7 @@ staple_status launch(const char* name, const DeviceInfo& di, const CUtensorMap& 
                      const CUtensorMap& b0, const CUtensorMap& b1, tc::Params p, cudaStream_t st,
                      const CUtensorMap* o = nullptr) {
   p.k_blocks = (p.K + tc::BK - 1) / tc::BK;
+  p.wait_ns = di.wait_ns;
   const int ntiles = p.tiles_m * p.tiles_n;
   if (ntiles == 0) return STAPLE_OK;
   if (p.group_m <= 0) p.group_m = 16;
@@ -251,10 +254,16 @@ staple_status tc_decode_fwd(const DeviceInfo& di, int T, int D, int F, const voi
   p.queue = words + pl.Dt + pl.G;
   p.part = static_cast<float*>(part);
   p.err = err;
+  p.wait_ns = di.wait_ns;
 
   // down-step ordering only where some block makes two or more gate/up tiles
   const int order = pl.G > pl.grid ? 1 : 0;
   auto kern = order ? fused::decode_fused_kernel<true> : fused::decode_fused_kernel<false>;
+  const int smem = fused::smem_bytes(pl.N, pl.sub);
+  // Blocks wait (bounded) on flags other blocks raise, so the whole grid must
+  // be resident at once.  Checked once per device, kernel and shared-memory
+  // size (queried outside any stream capture on first use): the grid may not
+  // exceed the SMs times the blocks one SM can hold.
   static std::atomic<uint64_t> attr_done[2];
   const uint64_t bit = uint64_t(1) << (di.device & 63);
   if (!(attr_done[order].load() & bit)) {
@@ -263,10 +272,26 @@ staple_status tc_decode_fwd(const DeviceInfo& di, int T, int D, int F, const voi
       return STAPLE_ECUDA;
     attr_done[order].fetch_or(bit);
   }
+  int per_sm = 0;
+  {
+    static std::mutex mu;
+    static std::map<std::tuple<int, int, int>, int> resident;   // (order, device, smem)
+    std::lock_guard<std::mutex> lock(mu);
+    const auto key = std::make_tuple(order, di.device, smem);
+    auto it = resident.find(key);
+    if (it == resident.end()) {
+      if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, fused::kThreads, smem) !=
+          cudaSuccess)
+        return STAPLE_ECUDA;
+      it = resident.emplace(key, per_sm).first;
+    }
+    per_sm = it->second;
+  }
+  if (per_sm <= 0 || pl.grid > per_sm * di.num_sms) return STAPLE_EUNSUPPORTED;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(pl.grid);
   cfg.blockDim = dim3(fused::kThreads);
-  cfg.dynamicSmemBytes = fused::smem_bytes(pl.N, pl.sub);
+  cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;

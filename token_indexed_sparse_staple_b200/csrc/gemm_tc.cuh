@@ -74,6 +74,7 @@ struct Params {
   const uint16_t* h_in;
   uint16_t* dgh;              // [M][2 * ldf]: dg in [0, F), dh in [F, 2F)
   int32_t* err;
+  uint64_t wait_ns;           // bound of every wait (STAPLE_ETIMEOUT past it)
 };
 
 __device__ __forceinline__ void tile_coords(int t, const Params& p, int& mb, int& nb) {
@@ -302,7 +303,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* empty = full + STAGES;
   uint64_t* tfull = empty + STAGES;
   uint64_t* tempty = tfull + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tempty + 2);
+  uint64_t* dbar = tempty + 2;   // MMA drain before tensor memory is freed
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(dbar + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5;
@@ -318,6 +320,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(&tfull[1], 1);
     mbar_init(&tempty[0], 4);
     mbar_init(&tempty[1], 4);
+    mbar_init(dbar, 1);
     *abort_flag = 0;
     fence_barrier_init();
     tma_prefetch_desc(&tmA);
@@ -346,7 +349,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tile_coords(t, p, mb, nb);
         const int m0 = mb * BM;
         for (int kb = 0; kb < p.k_blocks; ++kb) {
-          if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag, p.err)) {
+          if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag, p.err, p.wait_ns)) {
             ok = false;
             break;
           }
@@ -388,18 +391,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       }
-      if (!ok) {
-        // Let the copies already issued land before the block goes away.
-        for (int i = 0; i < STAGES && issued > 0; ++i, --issued) {
-          if (--stage < 0) {
-            stage = STAGES - 1;
-            phase ^= 1;
-          }
-          const uint64_t t0 = globaltimer();
-          while (!mbar_try_wait(&full[stage], phase) && globaltimer() - t0 < 1000000ull) {
-          }
-        }
-      }
+      // Let the copies still in flight land before the block goes away (on
+      // the normal path every fill was consumed and this returns at once).
+      drain_ring(full, STAGES, stage, phase, issued);
     }
   } else if (warp == 1) {
     if (lane == 0) {
@@ -412,11 +406,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x, ++iter) {
         const int buf = iter & 1;
         const uint32_t use = uint32_t(iter >> 1);
-        if (!mbar_wait(&tempty[buf], (use & 1) ^ 1, abort_flag, p.err)) break;
+        if (!mbar_wait(&tempty[buf], (use & 1) ^ 1, abort_flag, p.err, p.wait_ns)) break;
         tc_fence_after();
         const uint32_t dacc = tmem_base + uint32_t(buf * BN);
         for (int kb = 0; kb < p.k_blocks; ++kb) {
-          if (!mbar_wait(&full[stage], phase, abort_flag, p.err)) {
+          if (!mbar_wait(&full[stage], phase, abort_flag, p.err, p.wait_ns)) {
             ok = false;
             break;
           }
@@ -439,6 +433,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if (ok) umma_commit(&tfull[buf]);
       }
+      // Every MMA this thread issued completes before tensor memory and the
+      // operand stages are released (after an abort some may still run).
+      umma_commit(dbar);
+      mbar_drain(dbar, 0);
     }
   } else {
     // -------------------------------------------------------------- epilogue
@@ -452,7 +450,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t use = uint32_t(iter >> 1);
       int mb, nb;
       tile_coords(t, p, mb, nb);
-      const bool ok = mbar_wait(&tfull[buf], use & 1, abort_flag, p.err);
+      const bool ok = mbar_wait(&tfull[buf], use & 1, abort_flag, p.err, p.wait_ns);
       if (!__all_sync(0xffffffffu, ok)) break;
       tc_fence_after();
       const uint32_t tacc = tmem_base + (uint32_t(q * 32) << 16) + uint32_t(buf * BN);

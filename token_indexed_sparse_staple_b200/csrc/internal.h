@@ -11,10 +11,14 @@ namespace stp {
 
 constexpr int kMaxDedupT = 32768;  // one-block dedup keeps the batch in shared memory
 constexpr int kSegChunk = 64;      // sorted positions per block in the dE reduction
+// Kernel waits: default and largest bound (staple_set_wait_limit), in ns.
+constexpr uint64_t kWaitLimitNs = 4000000000ull;
+constexpr int64_t kMaxWaitLimitNs = 60000000000ll;
 
 struct DeviceInfo {
   int device;
   int num_sms;
+  uint64_t wait_ns;   // bound of every kernel wait (staple_set_wait_limit)
 };
 
 // trace.cu: optional per-kernel CUDA-event timing of a context

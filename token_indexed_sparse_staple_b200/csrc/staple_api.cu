@@ -141,6 +141,7 @@ staple_status staple_context_create(int device, staple_context** out) {
   if (!c) return STAPLE_ENOMEM;
   c->di.device = device;
   c->di.num_sms = prop.multiProcessorCount;
+  c->di.wait_ns = stp::kWaitLimitNs;
   if (lib_malloc(reinterpret_cast<void**>(&c->d_err), sizeof(int32_t), "context_err") !=
       cudaSuccess) {
     cudaGetLastError();
@@ -156,6 +157,12 @@ staple_status staple_context_create(int device, staple_context** out) {
   }
   c->tracer = stp::tracer_create(device);
   *out = c;
+  return STAPLE_OK;
+}
+
+staple_status staple_set_wait_limit(staple_context* ctx, int64_t limit_ns) {
+  if (!ctx || limit_ns < 1 || limit_ns > stp::kMaxWaitLimitNs) return STAPLE_EINVAL;
+  ctx->di.wait_ns = uint64_t(limit_ns);
   return STAPLE_OK;
 }
 
@@ -440,7 +447,10 @@ staple_status staple_gather_unique_rows_bulk(staple_context* ctx, const staple_c
   const uint8_t* src = static_cast<const uint8_t*>(table->base);
   uint8_t* hs = static_cast<uint8_t*>(staging_host);
   uint8_t* ds = static_cast<uint8_t*>(staging_dev);
-  const int32_t nchunks = (n + chunk_rows - 1) / chunk_rows;
+  // a chunk never exceeds the batch, so the chunk arithmetic below stays in
+  // range for any chunk_rows >= 1
+  const int32_t crows = std::max<int32_t>(1, std::min<int32_t>(chunk_rows, std::max(n, 1)));
+  const int32_t nchunks = int32_t((int64_t(n) + crows - 1) / crows);
   int nt = threads > 0 ? threads : int(std::thread::hardware_concurrency());
   nt = std::max(1, std::min(nt, nchunks));
   // one pool per call: workers claim chunks and mark each one packed; this
@@ -451,8 +461,8 @@ staple_status staple_gather_unique_rows_bulk(staple_context* ctx, const staple_c
   for (auto& a : packed) a.store(0, std::memory_order_relaxed);
   auto worker = [&]() {
     for (int32_t c; (c = next.fetch_add(1)) < nchunks;) {
-      const int32_t c1 = std::min(n, (c + 1) * chunk_rows);
-      for (int32_t i = c * chunk_rows; i < c1; ++i) {
+      const int32_t c1 = int32_t(std::min<int64_t>(n, (int64_t(c) + 1) * crows));
+      for (int32_t i = c * crows; i < c1; ++i) {
         // the host reads its own memory here: an id outside the table (the
         // dedup reports it, it does not clamp) must not steer the read
         const int32_t pos = ml[i];
@@ -473,7 +483,7 @@ staple_status staple_gather_unique_rows_bulk(staple_context* ctx, const staple_c
   cudaError_t ce = cudaSuccess;
   for (int32_t c = 0; c < nchunks; ++c) {
     while (!packed[size_t(c)].load(std::memory_order_acquire)) std::this_thread::yield();
-    const int32_t c0 = c * chunk_rows, c1 = std::min(n, c0 + chunk_rows);
+    const int32_t c0 = c * crows, c1 = int32_t(std::min<int64_t>(n, int64_t(c0) + crows));
     if (ce == cudaSuccess)
       ce = cudaMemcpyAsync(ds + int64_t(c0) * row_bytes, hs + int64_t(c0) * row_bytes,
                            size_t(c1 - c0) * size_t(row_bytes), cudaMemcpyHostToDevice, st);
@@ -534,9 +544,14 @@ staple_status staple_ffn_fwd(staple_context* ctx, staple_dtype dtype, int32_t T,
     return STAPLE_EINVAL;
   STP_TRY(set_device(ctx));
   stp::TraceScope trace_scope(ctx->tracer);
-  if (decode)
-    return stp::tc_decode_fwd(ctx->di, T, D, F, x, embed, w_gate, w_up, w_down, z, y, g_save,
-                              h_save, workspace, ctx->d_err, cs(stream));
+  if (decode) {
+    // the decode kernel refuses (before launching anything) a shape whose
+    // down tiles its clusters cannot own, or a device that cannot hold its
+    // grid at once; the tiled kernels then compute the same layer
+    const staple_status s = stp::tc_decode_fwd(ctx->di, T, D, F, x, embed, w_gate, w_up, w_down, z,
+                                               y, g_save, h_save, workspace, ctx->d_err, cs(stream));
+    if (s != STAPLE_EUNSUPPORTED) return s;
+  }
   if (dtype == STAPLE_BF16)
     return stp::tc_ffn_fwd(ctx->di, T, D, F, x, embed, w_gate, w_up, w_down, z, y, g_save, h_save,
                            ctx->d_err, cs(stream));
