@@ -19,6 +19,7 @@ __all__ = [
     "silu", "silu_grad", "dedup", "hot_set", "probe", "gather_rows",
     "ffn_forward", "ffn_backward", "forward_rows", "embed_grad_rows",
     "weight_grad_entries", "dx_rows", "cache_rows_for", "paper_shapes", "adamw_rows",
+    "stem_forward", "stem_backward",
 ]
 
 
@@ -171,6 +172,54 @@ def ffn_backward(dy, x, ids, w_gate, w_up, w_down, fwd: dict) -> dict:
         "dx": dg @ wg + dh @ wu,
         "dW_gate": dg.T @ x, "dW_up": dh.T @ x, "dW_down": dy.T @ fwd["z"],
     }
+
+
+# --------------------------------------------------------------------------
+# STEM, the replacement variant STAPLE builds on ([ABS]; [AIS] Interpretation)
+# --------------------------------------------------------------------------
+
+def stem_forward(x, ids, w_gate, w_down, table) -> dict:
+    """STEM's FFN: the token-indexed row replaces the up-projection instead of
+    being added to it ([ABS]: STEM replaces FFN up-projections with
+    token-indexed embeddings; [AIS] Interpretation: the replacement drops the
+    up-projection), still gated by SiLU of the gate projection:
+
+        g = W_gate x,  h = E[id],  z = SiLU(g) * h,  y = W_down z.
+
+    Reading: the pages give no formula for STEM beyond "replace the
+    up-projection"; the gate and down projections are kept as in the SwiGLU
+    FFN (its FLOPs and weights then drop by one d_model x d_ff matrix per
+    layer, which is what [TLA] Table 4 prints for STEM-12L).
+    Returns g, a = SiLU(g), h, z, y (fp64)."""
+    x = np.asarray(x, dtype=np.float64)
+    g = x @ np.asarray(w_gate, dtype=np.float64).T
+    a = silu(g)
+    h = np.asarray(table, dtype=np.float64)[np.asarray(ids, dtype=np.int64)]
+    z = a * h
+    y = z @ np.asarray(w_down, dtype=np.float64).T
+    return {"g": g, "a": a, "h": h, "z": z, "y": y}
+
+
+def stem_backward(dy, x, ids, w_gate, w_down, fwd: dict) -> dict:
+    """Gradients of <dY, y> for stem_forward:
+
+        dz = W_down^T dY,  dh = dz * SiLU(g),  dg = dz * h * SiLU'(g)
+        dE[j] = sum of dh over the tokens whose id is unique_j   (U rows)
+        dx = W_gate^T dg,  dW_gate = sum_i dg_i x_i^T,  dW_down = sum_i dY_i z_i^T
+
+    (no up-projection, so no dW_up and no W_up^T dh term in dx)."""
+    dy = np.asarray(dy, dtype=np.float64)
+    x = np.asarray(x, dtype=np.float64)
+    wg = np.asarray(w_gate, dtype=np.float64)
+    wd = np.asarray(w_down, dtype=np.float64)
+    dz = dy @ wd
+    dh = dz * fwd["a"]
+    dg = dz * fwd["h"] * silu_grad(fwd["g"])
+    unique, inverse, _, _ = dedup(ids)
+    dE = np.zeros((unique.size, dh.shape[1]), dtype=np.float64)
+    np.add.at(dE, inverse.astype(np.int64), dh)
+    return {"dz": dz, "dh": dh, "dg": dg, "unique": unique, "dE": dE, "dx": dg @ wg,
+            "dW_gate": dg.T @ x, "dW_down": dy.T @ fwd["z"]}
 
 
 # --------------------------------------------------------------------------

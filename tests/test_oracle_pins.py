@@ -441,3 +441,139 @@ def test_planted_adamw_mistake_is_caught(monkeypatch):
     monkeypatch.setattr(oracle, "adamw_rows", no_bias_correction)
     with pytest.raises(AssertionError):
         test_adamw_first_step_closed_form_and_untouched_rows()
+
+
+# --------------------------------------------------------------------------
+# STEM, the replacement variant (the row replaces the up-projection)
+# --------------------------------------------------------------------------
+
+def brute_stem(dy, x, ids, wg, wd, E):
+    """Per-token plain-Python loops of the STEM layer and its gradients."""
+    T, D = len(x), len(x[0])
+    F = len(wg)
+    out = {k: [] for k in ("g", "h", "z", "y")}
+    dE, dx = {}, [[0.0] * D for _ in range(T)]
+    dWg = [[0.0] * D for _ in range(F)]
+    dWd = [[0.0] * F for _ in range(D)]
+    for t in range(T):
+        g = [sum(wg[f][d] * x[t][d] for d in range(D)) for f in range(F)]
+        h = [E[ids[t]][f] for f in range(F)]
+        z = [g[f] * _sig(g[f]) * h[f] for f in range(F)]
+        y = [sum(wd[d][f] * z[f] for f in range(F)) for d in range(D)]
+        for k, v in (("g", g), ("h", h), ("z", z), ("y", y)):
+            out[k].append(v)
+        for f in range(F):
+            s = _sig(g[f])
+            dz = sum(wd[d][f] * dy[t][d] for d in range(D))
+            dh = dz * g[f] * s
+            dg = dz * h[f] * (s + g[f] * s * (1.0 - s))
+            row = dE.setdefault(ids[t], [0.0] * F)
+            row[f] += dh
+            for d in range(D):
+                dx[t][d] += wg[f][d] * dg
+                dWg[f][d] += dg * x[t][d]
+        for d in range(D):
+            for f in range(F):
+                dWd[d][f] += dy[t][d] * z[f]
+    keys = sorted(dE)
+    res = {k: np.array(v) for k, v in out.items()}
+    res.update(unique=np.array(keys), dE=np.array([dE[k] for k in keys]), dx=np.array(dx),
+               dW_gate=np.array(dWg), dW_down=np.array(dWd))
+    return res
+
+
+@pytest.mark.parametrize("seed", [0, 4])
+def test_stem_matches_brute_force(seed):
+    x, ids, wg, _, wd, E, dy = _tiny(seed)
+    fw = oracle.stem_forward(x, ids, wg, wd, E)
+    bw = oracle.stem_backward(dy, x, ids, wg, wd, fw)
+    ref = brute_stem(*_lists(dy, x), ids.tolist(), *_lists(wg, wd, E))
+    for k in ("g", "h", "z", "y"):
+        np.testing.assert_allclose(fw[k], ref[k], rtol=1e-12, atol=1e-12, err_msg=k)
+    np.testing.assert_array_equal(bw["unique"], ref["unique"])
+    for k in ("dE", "dx", "dW_gate", "dW_down"):
+        np.testing.assert_allclose(bw[k], ref[k], rtol=1e-11, atol=1e-11, err_msg=k)
+
+
+def test_stem_is_staple_with_a_zero_up_projection():
+    """h = W_up x + E[id] with W_up = 0 is h = E[id]: the two definitions agree
+    exactly on everything STEM has (the STAPLE oracle is pinned on its own)."""
+    x, ids, wg, wu, wd, E, dy = _tiny(2)
+    zero = np.zeros_like(wu)
+    st = oracle.stem_forward(x, ids, wg, wd, E)
+    sp = oracle.ffn_forward(x, ids, wg, zero, wd, E)
+    for k in ("g", "h", "z", "y"):
+        np.testing.assert_array_equal(st[k], sp[k], err_msg=k)
+    bs = oracle.stem_backward(dy, x, ids, wg, wd, st)
+    bp = oracle.ffn_backward(dy, x, ids, wg, zero, wd, sp)
+    for k in ("dh", "dg", "dE", "dx", "dW_gate", "dW_down"):
+        np.testing.assert_array_equal(bs[k], bp[k], err_msg=k)
+    # with a nonzero up-projection the layers differ (STEM drops it)
+    assert not np.allclose(oracle.ffn_forward(x, ids, wg, wu, wd, E)["y"], st["y"])
+
+
+def test_stem_gradients_match_finite_differences():
+    x, ids, wg, _, wd, E, dy = _tiny(5, T=4, D=3, F=4, V=6)
+
+    def loss(x_, wg_, wd_, E_):
+        return float(np.sum(dy * oracle.stem_forward(x_, ids, wg_, wd_, E_)["y"]))
+
+    fw = oracle.stem_forward(x, ids, wg, wd, E)
+    bw = oracle.stem_backward(dy, x, ids, wg, wd, fw)
+    eps = 1e-6
+    for name, arr, grad in (("x", x, bw["dx"]), ("W_gate", wg, bw["dW_gate"]),
+                            ("W_down", wd, bw["dW_down"])):
+        num = np.zeros_like(arr)
+        for idx in np.ndindex(arr.shape):
+            a = arr.copy()
+            a[idx] += eps
+            args_p = [x, wg, wd, E]
+            args_p[["x", "W_gate", "W_down"].index(name)] = a
+            lp = loss(*args_p)
+            a[idx] -= 2 * eps
+            args_m = [x, wg, wd, E]
+            args_m[["x", "W_gate", "W_down"].index(name)] = a
+            lm = loss(*args_m)
+            num[idx] = (lp - lm) / (2 * eps)
+        np.testing.assert_allclose(grad, num, rtol=1e-6, atol=1e-8, err_msg=name)
+    numE = np.zeros_like(E)
+    for idx in np.ndindex(E.shape):
+        a = E.copy()
+        a[idx] += eps
+        lp = loss(x, wg, wd, a)
+        a[idx] -= 2 * eps
+        lm = loss(x, wg, wd, a)
+        numE[idx] = (lp - lm) / (2 * eps)
+    np.testing.assert_allclose(bw["dE"], numE[bw["unique"]], rtol=1e-6, atol=1e-8)
+
+
+def test_stem_single_token_table_gradient_closed_form():
+    x, ids, wg, _, wd, E, dy = _tiny(6, T=1)
+    fw = oracle.stem_forward(x, ids, wg, wd, E)
+    bw = oracle.stem_backward(dy, x, ids, wg, wd, fw)
+    closed = oracle.silu(wg @ x[0]) * (wd.T @ dy[0])
+    np.testing.assert_allclose(bw["dE"][0], closed, rtol=1e-13, atol=1e-13)
+
+
+def _mutant_stem(kind):
+    real = oracle.stem_forward
+
+    def bad(x, ids, wg, wd, table):
+        out = real(x, ids, wg, wd, table)
+        if kind == "adds_to_gate":
+            g = out["g"] + out["h"]
+            out["z"] = oracle.silu(g) * out["h"]
+        elif kind == "ungated":
+            out["z"] = out["h"]
+        elif kind == "wrong_row":
+            out["z"] = out["a"] * np.asarray(table)[(np.asarray(ids) + 1) % table.shape[0]]
+        out["y"] = out["z"] @ np.asarray(wd).T
+        return out
+    return bad
+
+
+@pytest.mark.parametrize("kind", ["adds_to_gate", "ungated", "wrong_row"])
+def test_planted_stem_mistakes_are_caught(kind, monkeypatch):
+    monkeypatch.setattr(oracle, "stem_forward", _mutant_stem(kind))
+    with pytest.raises(AssertionError):
+        test_stem_matches_brute_force(0)
