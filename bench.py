@@ -240,18 +240,22 @@ def decode_setup(stp, w, local):
     st["emb"] = [stp.make_embed(stp.STAPLE_EMBED_TABLE, st["table"], F, st["ids"][s], V)
                  for s in range(S)]
     st["emb_none"] = stp.make_embed(stp.STAPLE_EMBED_NONE)
+    st["emb_stem"] = [stp.make_embed(stp.STAPLE_EMBED_TABLE, st["table"], F, st["ids"][s], V,
+                                     flags=stp.STAPLE_EMBED_REPLACE_UP) for s in range(S)]
     st["wsb"] = stp.staple_workspace_bytes(T, D, F)
     st["ws"] = torch.zeros(st["wsb"], dtype=torch.uint8, device="cuda")
     return st
 
 
-def decode_step(stp, ctx, w, st, s, stream, dense=False):
+def decode_step(stp, ctx, w, st, s, stream, mode="staple"):
+    """One decode step.  mode: "staple" (row added), "dense" (E path off) or
+    "stem" (row replaces the up-projection; W_up not passed)."""
     r = s % st["R"]
     b = s % st["S"]
-    emb = st["emb_none"] if dense else st["emb"][b]
+    emb = {"staple": st["emb"], "stem": st["emb_stem"]}[mode][b] if mode != "dense" else st["emb_none"]
     stp.staple_ffn_fwd(ctx, stp.STAPLE_BF16, w.T, w.D, w.F, st["x"][b], emb, st["wg"][r],
-                       st["wu"][r], st["wd"][r], st["z"], st["y"], None, None, st["ws"], st["wsb"],
-                       stream=stream)
+                       None if mode == "stem" else st["wu"][r], st["wd"][r], st["z"], st["y"],
+                       None, None, st["ws"], st["wsb"], stream=stream)
 
 
 def capture_steps(step, n, stream):
@@ -303,11 +307,9 @@ def run_decode(stp, ctx, w, args, world, local):
     G = st["R"] * st["S"] // 4   # steps per captured graph (cycles weights 16x)
     K = max(1, args.steps)
     out = {}
-    for mode in ("staple", "dense"):
-        dense = mode == "dense"
-
-        def step(s, dense=dense):
-            decode_step(stp, ctx, w, st, s, stream, dense)
+    for mode in ("staple", "dense", "stem"):
+        def step(s, mode=mode):
+            decode_step(stp, ctx, w, st, s, stream, mode)
 
         with torch.cuda.stream(stream):
             for s in range(max(args.warmup, 3)):
@@ -319,7 +321,8 @@ def run_decode(stp, ctx, w, args, world, local):
         out[mode] = {"ms": ms_max, "ms_local": ms, "clocks": clocks}
     res = {"K": K, "ms": out["staple"]["ms"], "ms_local": out["staple"]["ms_local"],
            "clocks": out["staple"]["clocks"], "dense_ms": out["dense"]["ms"],
-           "dense_clocks": out["dense"]["clocks"]}
+           "dense_clocks": out["dense"]["clocks"], "stem_ms": out["stem"]["ms"],
+           "stem_ms_local": out["stem"]["ms_local"]}
     # the same steps again with per-kernel CUDA events recorded around every
     # launch: the kernel list and shares (events between launches stop the
     # programmatic overlap of consecutive launches, so these steps are slower)
@@ -412,6 +415,8 @@ def run_train(stp, ctx, w, steps, warmup, world, local):
                                          torch.empty(1, **i32))
             self.rows = torch.empty((T, F), dtype=torch.bfloat16, device="cuda")
             self.emb = stp.make_embed(stp.STAPLE_EMBED_ROWS, self.rows, F, self.inverse, T)
+            self.emb_stem = stp.make_embed(stp.STAPLE_EMBED_ROWS, self.rows, F, self.inverse, T,
+                                           flags=stp.STAPLE_EMBED_REPLACE_UP)
             self.ready = torch.cuda.Event()   # rows gathered (prefetch streams)
             self.free = torch.cuda.Event()    # last reader done (main stream)
 
@@ -442,35 +447,42 @@ def run_train(stp, ctx, w, steps, warmup, world, local):
                                side=pf_side)
         r.ready.record(pf)
 
-    def step(s, staple=True):
+    def step(s, staple=True, stem=False):
+        """staple: the E path on (with stem: the row replaces the
+        up-projection, no W_up in the forward or backward); else the dense run."""
         b = s % S
         r = buf[s % 2]
         if staple:
             prefetch(s + 1)
             stream.wait_event(r.ready)
-        stp.staple_ffn_fwd(ctx, stp.STAPLE_BF16, T, D, F, x[b], r.emb if staple else emb_none,
-                           wg, wu, wd, z, y, g, h, ws, wsb, stream=stream)
+        emb = (r.emb_stem if stem else r.emb) if staple else emb_none
+        stp.staple_ffn_fwd(ctx, stp.STAPLE_BF16, T, D, F, x[b], emb, wg, None if stem else wu, wd,
+                           z, y, g, h, ws, wsb, stream=stream)
         stp.staple_embed_bwd(ctx, stp.STAPLE_BF16, T, D, F, dy[b], g, h, wd, r.sorted_pos,
                              r.inverse, r.seg, r.U, dgh, dE if staple else None, ws, wsb,
                              stream=stream)
         if staple:
             r.free.record(stream)
-        stp.staple_ffn_bwd(ctx, stp.STAPLE_BF16, T, D, F, dy[b], x[b], z, dgh, wg, wu, dx, dwg, dwu,
-                           dwd, stream=stream)
+        stp.staple_ffn_bwd(ctx, stp.STAPLE_BF16, T, D, F, dy[b], x[b], z, dgh, wg,
+                           None if stem else wu, dx, dwg, None if stem else dwu, dwd, stream=stream)
 
     out = {}
     try:
-        for mode in ("staple", "dense"):
-            staple = mode == "staple"
+        # (name, E path on, STEM, SMs the GEMMs leave to the prefetch kernels)
+        for mode, staple, stem, reserve in (("staple_r0", True, False, 0),
+                                            ("staple", True, False, 1),
+                                            ("dense", False, False, 0),
+                                            ("stem", True, True, 1)):
+            stp.staple_set_sm_reserve(ctx, reserve)
             nw = max(warmup, 3)
             with torch.cuda.stream(stream):
                 if staple:
                     prefetch(0)
                 for s in range(nw):
-                    step(s, staple)
+                    step(s, staple, stem)
             torch.cuda.synchronize()
             assert stp.staple_get_error(ctx, stream) == 0
-            if staple:
+            if mode == "staple":
                 stp.staple_trace_enable(ctx, True)
             barrier(world)
             ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -480,7 +492,7 @@ def run_train(stp, ctx, w, steps, warmup, world, local):
                 with torch.cuda.stream(stream):
                     ev0.record(stream)
                     for s in range(nw, nw + steps):
-                        step(s, staple)
+                        step(s, staple, stem)
                     if staple:   # the last prefetch ends inside the timed region too
                         stream.wait_event(buf[(nw + steps) % 2].ready)
                     ev1.record(stream)
@@ -488,8 +500,8 @@ def run_train(stp, ctx, w, steps, warmup, world, local):
                 t1 = time.time()
             ms = max_over_ranks(ev0.elapsed_time(ev1), world)
             assert stp.staple_get_error(ctx, stream) == 0
-            out[mode] = {"ms": ms, "clocks": clk.summary(t0, t1)}
-            if staple:
+            out[mode] = {"ms": ms, "clocks": clk.summary(t0, t1), "sm_reserve": reserve}
+            if mode == "staple":
                 out[mode]["kernels"] = kernel_table(stp.staple_trace_read(ctx), steps)
                 stp.staple_trace_enable(ctx, False)
                 out["U"] = int(buf[0].U.item())
@@ -523,6 +535,7 @@ def run_train(stp, ctx, w, steps, warmup, world, local):
                               "how": "probe + hits + host pack (all threads) + bulk H2D chunk by "
                                      "chunk + scatter, wall time, median of 5 per chunk size"}
     finally:
+        stp.staple_set_sm_reserve(ctx, 0)
         stp.staple_cache_free(cache)
         stp.staple_table_unregister(tab)
     return out
@@ -719,6 +732,9 @@ def run_stack_train(stp, ctx, w, steps, world, local):
     freq = syn.calibration_freq(V)
     tables = GroupedTables(ctx, host, V, F, G, freq, w.cache_frac)
     S = 4
+    # one SM is left to the next step's dedup and first gather, which run
+    # beside the backward's GEMMs on the prefetch streams
+    stp.staple_set_sm_reserve(ctx, 1)
     try:
         s = TrainStack(ctx, W, tables, T, D, F, V)
         ids = [torch.from_numpy(syn.zipf_ids(T, V, w.zipf_s, seed=syn.SEED_IDS + w.index + 7919 * k)).cuda()
@@ -763,6 +779,7 @@ def run_stack_train(stp, ctx, w, steps, world, local):
         kern = kernel_table(stp.staple_trace_read(ctx), 1)
         stp.staple_trace_enable(ctx, False)
     finally:
+        stp.staple_set_sm_reserve(ctx, 0)
         tables.close()
     step_ms = ms / steps
     flops = 18 * T * D * F * L
@@ -933,13 +950,18 @@ def main():
     K = dec["K"]
     value = job_value(w.T * K, dec["ms"], world)
     kd = dec["kernels"].get(dec["roofline_kernel"], {})
-    # one launch per step: the untraced timed step bounds the launch duration
-    # from above; the traced average is reported beside it
-    one = abs(dec["launches_per_step"] - 1.0) < 1e-9 and kd
+    # Every launch of a step belongs to the decode layer (the fused kernel and
+    # its split-k sum kernel): the untraced timed step bounds the dominant
+    # kernel's duration from above; the traced averages are reported beside
+    # it (trace events between launches stop their programmatic overlap).
+    own = set(dec["kernels"]) <= {"k5k6_decode_fused", "k6r_decode_reduce"}
+    one = own and kd
     launch_us = dec["ms_local"] * 1000.0 / K if one else kd.get("avg_us", float("nan"))
     ach = dec["alg_bytes"] / (launch_us * 1e-6) / 1e9
     traffic, traffic_src = captured_traffic(dec["roofline_kernel"])
     dense_us = dec["dense_ms"] * 1000.0 / K
+    stem_us = dec["stem_ms_local"] * 1000.0 / K
+    stem_bytes = dec["alg_bytes"] - w.F * w.D * 2      # no W_up
     step_us = dec["ms"] * 1000.0 / K
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K,
@@ -952,8 +974,9 @@ def main():
                      "peak_source": pk["source"] + " (copy bandwidth)",
                      "alg_bytes_per_launch": dec["alg_bytes"], "launch_us": r3(launch_us),
                      "traced_launch_us": kd.get("avg_us"),
-                     "duration": ("untraced timed step (one launch per step)" if one else
-                                  "traced per-launch CUDA events")},
+                     "traced_reduce_us": dec["kernels"].get("k6r_decode_reduce", {}).get("avg_us"),
+                     "duration": ("untraced timed step (the decode kernel and its split-k sum "
+                                  "kernel)" if one else "traced per-launch CUDA events")},
         "e2e": {"value": r3(job_value(w.T * dec["e2e"]["K"], dec["e2e"]["ms"], world)),
                 "unit": "tokens/s", "h2d_bytes_per_step": dec["e2e"]["h2d"],
                 "d2h_bytes_per_step": dec["e2e"]["d2h"], "steps": dec["e2e"]["K"],
@@ -963,6 +986,11 @@ def main():
         "decode_dense": {"us_per_step": r3(dense_us), "us_per_step_staple": r3(step_us),
                          "e_path_overhead": r3((step_us - dense_us) / dense_us),
                          "how": "same kernel and steps with STAPLE_EMBED_NONE (no E rows)"},
+        "decode_stem": {"tokens_per_s": r3(job_value(w.T * K, dec["stem_ms"], world)),
+                        "us_per_step": r3(stem_us),
+                        "hbm_frac": r3(stem_bytes / (stem_us * 1e-6) / 1e9 / pk["hbm_gbs"]),
+                        "how": "same steps, STAPLE_EMBED_REPLACE_UP: the row replaces W_up "
+                               "(2*F*D*2 weight bytes per step)"},
     }
     detail["decode_kernels"] = dec["kernels"]
     detail["decode_dense_clocks"] = dec["dense_clocks"]
@@ -974,7 +1002,10 @@ def main():
         try:
             wt = syn.WORKLOADS["olmo2-1b-train-layer"]
             tr = run_train(stp, ctx, wt, args.train_steps, 5, world, local)
-            st_ms = tr["staple"]["ms"] / args.train_steps
+            # the E-path run at its better SM reserve (0: the GEMMs use every
+            # SM; 1: one SM is left to the prefetched retrieval kernels)
+            best = min(("staple", "staple_r0"), key=lambda m: tr[m]["ms"])
+            st_ms = tr[best]["ms"] / args.train_steps
             de_ms = tr["dense"]["ms"] / args.train_steps
             kern = tr["staple"]["kernels"]
             top = max(kern.items(), key=lambda kv: kv[1]["total_ms"])
@@ -995,6 +1026,12 @@ def main():
                 "workload": wt.name, "tokens_per_s": r3(job_value(wt.T, st_ms, world)),
                 "ms_per_step": r3(st_ms), "dense_ms_per_step": r3(de_ms),
                 "e_path_overhead": r3((st_ms - de_ms) / de_ms), "steps": args.train_steps,
+                "sm_reserve": tr[best]["sm_reserve"],
+                "ms_by_sm_reserve": {str(tr[m]["sm_reserve"]): r3(tr[m]["ms"] / args.train_steps)
+                                     for m in ("staple_r0", "staple")},
+                "stem_ms_per_step": r3(tr["stem"]["ms"] / args.train_steps),
+                "stem_tokens_per_s": r3(job_value(wt.T, tr["stem"]["ms"] / args.train_steps,
+                                                  world)),
                 "U": tr["U"], "misses": tr["misses"],
                 "tflops": r3(layer_tf),
                 "layer_frac_sustained": r3(layer_tf / pk["bf16_tflops_sustained"]),

@@ -105,6 +105,15 @@ staple_status staple_get_error(staple_context* ctx, staple_stream stream, int32_
  * captured CUDA graph keeps the limit it was captured with). */
 staple_status staple_set_wait_limit(staple_context* ctx, int64_t limit_ns);
 
+/* SMs that the tiled (persistent) GEMM kernels of this context leave free
+ * from now on, for kernels running beside them on other streams.  Each GEMM
+ * block keeps an SM's shared memory to itself, so a kernel queued on another
+ * stream (the next batch's dedup, which holds one SM's shared memory for a
+ * whole batch) otherwise takes an SM a GEMM block was due to start on, and
+ * that block, with its fixed share of the tiles, finishes late.  Default 0;
+ * EINVAL unless 0 <= sms <= a quarter of the SMs.  Host-only. */
+staple_status staple_set_sm_reserve(staple_context* ctx, int32_t sms);
+
 /* Per-kernel timing.  With tracing enabled, every kernel the library launches
  * for this context is bracketed by two CUDA events on its launch stream (a
  * record costs well under a microsecond of device time).  staple_trace_read
@@ -271,9 +280,16 @@ typedef enum staple_embed_mode {
                              base = gathered rows; n_rows = capacity */
 } staple_embed_mode;
 
+/* staple_embed.flags */
+#define STAPLE_EMBED_REPLACE_UP 1u  /* STEM, the variant STAPLE builds on (abstract: STEM replaces
+                                       the FFN up-projections with token-indexed embeddings;
+                                       ai4snews summary, Interpretation): the row takes the
+                                       up-projection's place, h = E[id], and w_up is not read
+                                       (may be NULL).  Needs mode TABLE or ROWS. */
+
 typedef struct staple_embed {
   int32_t mode;          /* staple_embed_mode */
-  int32_t reserved;
+  uint32_t flags;        /* 0 (STAPLE: the row is added) or STAPLE_EMBED_REPLACE_UP (STEM) */
   const void* base;      /* device; points at this layer's first element (group offset applied) */
   int64_t row_pitch;     /* elements between consecutive rows (groups * F) */
   const int32_t* index;  /* device [T] */
@@ -286,6 +302,8 @@ typedef struct staple_embed {
  * summary, Interpretation: the zero-initialised table leaves the seed FFN's
  * output unchanged, and the gate makes the added row context-dependent):
  *     g = W_gate x,  h = W_up x + E[id],  z = SiLU(g) * h,  y = W_down z.
+ * With embed->flags = STAPLE_EMBED_REPLACE_UP it computes STEM instead,
+ * h = E[id] (w_up not read, may be NULL).
  *   x[T][D], w_gate[F][D], w_up[F][D], w_down[D][F]   inputs (dtype)
  *   z[T][F]     out: SiLU(g) * h, the down projection's input (kept for dW_down)
  *   y[T][D]     out: layer output
@@ -372,6 +390,8 @@ staple_status staple_embed_grad_to_host(staple_context* ctx, int32_t F, int32_t 
  *   dw_up[F][D]    = sum_t dh_t x_t^T       (fp32; NULL: frozen up-projection,
  *                    the warmup recipe of the ai4snews summary, Interpretation)
  *   dw_down[D][F]  = sum_t dY_t z_t^T       (fp32; NULL: not computed)
+ * w_up == NULL (with dw_up == NULL) is the STEM layer, which has no
+ * up-projection (STAPLE_EMBED_REPLACE_UP): dx = dg W_gate.
  * Gradients are written, not accumulated. */
 staple_status staple_ffn_bwd(staple_context* ctx, staple_dtype dtype, int32_t T, int32_t D,
                              int32_t F, const void* dy, const void* x, const void* z,

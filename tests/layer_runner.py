@@ -9,15 +9,19 @@ from tests.helpers import dev, empty, f64
 
 
 def run_layer(stp, ctx, inp, D, F, V, *, embed="table", training=True, rows_table=None,
-              freeze_up=False, cache_frac=None, freq=None):
+              freeze_up=False, cache_frac=None, freq=None, stem=False):
     """inp: synthetic.LayerInputs.  embed in {"none", "table", "rows"}.
     rows_table: host numpy table registered as pinned host memory for the
-    "rows" mode (default: the device table)."""
+    "rows" mode (default: the device table).  stem: the STEM layer (the row
+    replaces the up-projection; W_up is passed as NULL)."""
     import torch
     dt = inp.dtype
     sdt = stp.STAPLE_BF16 if dt == "bf16" else stp.STAPLE_F32
     T = inp.ids.size
     x, wg, wu, wd = (dev(getattr(inp, k), dt) for k in ("x", "w_gate", "w_up", "w_down"))
+    embed_flags = stp.STAPLE_EMBED_REPLACE_UP if stem else 0
+    if stem:
+        wu = None
     ids = torch.from_numpy(inp.ids).cuda()
     z, g, h = (empty((T, F), dt) for _ in range(3))
     y = empty((T, D), dt)
@@ -30,7 +34,7 @@ def run_layer(stp, ctx, inp, D, F, V, *, embed="table", training=True, rows_tabl
     elif embed == "table":
         tab = dev(inp.table, dt)
         keep.append(tab)
-        e = stp.make_embed(stp.STAPLE_EMBED_TABLE, tab, F, ids, V)
+        e = stp.make_embed(stp.STAPLE_EMBED_TABLE, tab, F, ids, V, flags=embed_flags)
     else:
         unique, inverse, sorted_pos, slot, miss = (empty(max(T, 1), "i32") for _ in range(5))
         seg, U, mc = empty(T + 1, "i32"), empty(1, "i32"), empty(1, "i32")
@@ -49,7 +53,7 @@ def run_layer(stp, ctx, inp, D, F, V, *, embed="table", training=True, rows_tabl
         side = torch.cuda.Stream()
         stp.staple_gather_rows(ctx, cache, table_handle, ids, T, unique, inverse, seg, sorted_pos, U,
                                slot, miss, mc, rows, side=side)
-        e = stp.make_embed(stp.STAPLE_EMBED_ROWS, rows, F, inverse, max(T, 1))
+        e = stp.make_embed(stp.STAPLE_EMBED_ROWS, rows, F, inverse, max(T, 1), flags=embed_flags)
         keep.append(rows)
         out["miss_count"] = int(mc.item())
     wsb = stp.staple_workspace_bytes(T, D, F)
@@ -76,7 +80,7 @@ def run_layer(stp, ctx, inp, D, F, V, *, embed="table", training=True, rows_tabl
             dwu = torch.full((F, D), 7.0, dtype=torch.float32, device="cuda")
             dwd = torch.empty((D, F), dtype=torch.float32, device="cuda")
             stp.staple_ffn_bwd(ctx, sdt, T, D, F, dy, x, z, dgh, wg, wu, dx, dwg,
-                               None if freeze_up else dwu, dwd)
+                               None if (freeze_up or stem) else dwu, dwd)
             err = stp.staple_get_error(ctx)
             assert err == 0, stp.staple_status_string(err)
             u = int(U.item())

@@ -43,14 +43,15 @@ def _small_layer_matches_oracle(stp, ctx, T):
         assert_close(got[k], ref[k], TOL["bf16"], k)
 
 
-@pytest.mark.parametrize("T", [64, 384])
-def test_wait_limit_runs_out_then_context_recovers(stp, ctx, T):
-    """d_model 32768 makes every gate/up tile stream 8 MB (decode kernel,
-    T = 64) or 24 MB (tiled GEMM, T = 384) of weights through one SM before
-    its accumulator is ready, tens of microseconds at least, so a 10 us limit
-    runs out in the first wait for an accumulator."""
+@pytest.mark.parametrize("T,D", [(64, 8192), (384, 32768)])
+def test_wait_limit_runs_out_then_context_recovers(stp, ctx, T, D):
+    """A long d_model makes every gate/up tile stream megabytes of weights
+    through one SM before its accumulator is ready: 2 MB per tile in the decode
+    kernel (T = 64, d_model 8192), 24 MB in the tiled GEMM (T = 384, d_model
+    32768), tens of microseconds at least, so a 10 us limit runs out in the
+    first wait for an accumulator."""
     import torch
-    D, F, V = 32768, 256, 100
+    F, V = 256, 100
     g = torch.Generator(device="cuda")
     g.manual_seed(5)
 

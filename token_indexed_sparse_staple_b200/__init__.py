@@ -23,6 +23,7 @@ STAPLE_ETIMEOUT, STAPLE_EUNSUPPORTED, STAPLE_ENODEV = -5, -6, -7
 STAPLE_BF16, STAPLE_F32 = 0, 1
 STAPLE_EMBED_NONE, STAPLE_EMBED_TABLE, STAPLE_EMBED_ROWS = 0, 1, 2
 STAPLE_TABLE_DEVICE, STAPLE_TABLE_HOST_PINNED, STAPLE_TABLE_HOST_REGISTER = 1, 2, 4
+STAPLE_EMBED_REPLACE_UP = 1
 
 __all__ = [n for n in _lib.SIGNATURES] + [
     "StapleError", "staple_embed", "staple_adamw", "make_embed", "lib",
@@ -65,8 +66,11 @@ def _ok(status: int, where: str) -> None:
         raise StapleError(status, where)
 
 
-def make_embed(mode: int, base=None, row_pitch: int = 0, index=None, n_rows: int = 0) -> staple_embed:
-    return staple_embed(mode, 0, _p(base), row_pitch, _p(index), n_rows)
+def make_embed(mode: int, base=None, row_pitch: int = 0, index=None, n_rows: int = 0,
+               flags: int = 0) -> staple_embed:
+    """flags = STAPLE_EMBED_REPLACE_UP: the STEM layer (the row replaces the
+    up-projection)."""
+    return staple_embed(mode, flags, _p(base), row_pitch, _p(index), n_rows)
 
 
 # ------------------------------------------------------------------ context
@@ -98,6 +102,11 @@ def staple_get_error(ctx: int, stream=None) -> int:
 def staple_set_wait_limit(ctx: int, limit_ns: int) -> None:
     """Bound of every kernel wait of later launches, in ns (see include/staple.h)."""
     _ok(lib().staple_set_wait_limit(ctx, int(limit_ns)), "staple_set_wait_limit")
+
+
+def staple_set_sm_reserve(ctx: int, sms: int) -> None:
+    """SMs the tiled GEMMs leave free for work on other streams (see include/staple.h)."""
+    _ok(lib().staple_set_sm_reserve(ctx, int(sms)), "staple_set_sm_reserve")
 
 
 def staple_trace_enable(ctx: int, enable: bool = True) -> None:

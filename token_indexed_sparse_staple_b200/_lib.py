@@ -24,7 +24,7 @@ class staple_trace_record(C.Structure):
 
 
 class staple_embed(C.Structure):
-    _fields_ = [("mode", i32), ("reserved", i32), ("base", vp), ("row_pitch", i64),
+    _fields_ = [("mode", i32), ("flags", u32), ("base", vp), ("row_pitch", i64),
                 ("index", vp), ("n_rows", i64)]
 
 
@@ -41,6 +41,7 @@ SIGNATURES = {
     "staple_context_destroy": (c_status, [vp]),
     "staple_get_error": (c_status, [vp, vp, P(i32)]),
     "staple_set_wait_limit": (c_status, [vp, i64]),
+    "staple_set_sm_reserve": (c_status, [vp, i32]),
     "staple_trace_enable": (c_status, [vp, C.c_int]),
     "staple_trace_read": (c_status, [vp, vp, i32, P(i32)]),
     "staple_table_register": (c_status, [vp, vp, sz, i64, i32, i32, C.c_int, u32, P(vp)]),

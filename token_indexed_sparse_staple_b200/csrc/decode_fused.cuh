@@ -1,6 +1,7 @@
-// One persistent tcgen05 kernel for the STAPLE layer at decode sizes
-// (T <= 256 tokens): gate/up with the fused E-row add and SiLU gating, then
-// the down projection, in a single launch.
+// The STAPLE layer at decode sizes (T <= 256 tokens) in two launches: one
+// persistent tcgen05 kernel for gate/up (with the fused E-row add and SiLU
+// gating) and the down projection's split-k pieces, then a small kernel that
+// sums the pieces.
 //
 // With a handful of tokens the layer streams its weights once per step and
 // is bound by HBM bandwidth, so the kernel is organised around that stream:
@@ -12,13 +13,15 @@
 //    in runs of sub * 128 bytes (short runs per row leave HBM far below its
 //    bandwidth).  Weights and activations have separate rings: the weight
 //    ring is deep (HBM latency), the activation ring shallow (it hits L2).
+//    Weights depend on nothing earlier, so the first ring fills are issued
+//    before the block's set-up barrier.
 //  * Phase 1, gate/up: whole tiles are spread over the blocks.  A block
 //    finishes a tile straight from tensor memory, 16 tokens at a time: g and
 //    u rows go to shared memory, then each of the 128 epilogue threads
 //    computes 8 consecutive features of one token, h = u + E[id_t][f] (E rows
 //    prefetched into shared memory during the main loop) and z = SiLU(g) h
-//    (g and h saved when asked), written 16 bytes at a time; then the
-//    tile's ready flag goes up.
+//    (g and h saved when asked), written 16 bytes at a time; then one thread
+//    publishes the tile with a release store of its ready flag.
 //  * Phase 2, down: the down units (tile x `sub` k blocks) are split evenly
 //    over the blocks (stream-K), so every SM streams the same share of
 //    W_down.  The first units' weights are copied from the ring into the
@@ -29,24 +32,24 @@
 //    flags of the gate/up tiles that produced the block's z columns; weight
 //    loads do not wait.  Each block's piece of a tile leaves an fp32 partial
 //    [N][128] in the workspace (L2-resident; a warp writes 128 contiguous
-//    bytes per token) and bumps the tile's counter.
-//  * The down sums are spread over all blocks: once a block has finished its
-//    own pieces, its epilogue warps take 16-row chunks from an atomic work
-//    queue, wait (bounded) until the chunk's tile is complete, bring every
-//    piece's 16 x N slice into the (then idle) ring memory with TMA loads
-//    that are all in flight at once, sum them in piece order
-//    (deterministic) and write y = bf16(sum).
+//    bytes per token), and the block is done.
+//  * The split-k sums run in decode_reduce_kernel, launched right behind as
+//    a programmatic dependent (see there), which also clears the ready flags.
 //  * Every block finishes its gate/up tiles before it needs anybody's z, so
-//    all waits end while all blocks are resident (grid <= SMs, one block
-//    per SM).  Counters, flags and queue counters live in the first bytes of
-//    the workspace; the last event of a call resets them, so a zero-filled
+//    all waits end while all blocks are resident (grid <= SMs, one block per
+//    SM, checked by the launcher).  The ready flags live in the first bytes
+//    of the workspace and are zero again after every call, so a zero-filled
 //    workspace stays valid across calls and graph replays.
+//
+// The STEM variant (kStem: the row replaces the up-projection) streams no
+// W_up: a gate tile is 128 W_gate rows (128 features) and h = E[id_t].
 //
 // Warps: 0 weight (A) loads, 1 MMA issue + tensor memory, 2 activation (B)
 // loads, 3..6 epilogue (each owns one 32-lane quarter of tensor memory).
-// Every mbarrier wait and flag spin is bounded (STAPLE_ETIMEOUT).  The
-// kernel is launched as a programmatic dependent: weights stream before
-// griddepcontrol.wait; activations, outputs and counters only after it.
+// Every mbarrier wait and flag spin is bounded (STAPLE_ETIMEOUT); after a
+// timeout each role lets its issued copies and MMAs finish before the block
+// exits.  The kernel is launched as a programmatic dependent: weights stream
+// before griddepcontrol.wait; activations, outputs and flags only after it.
 #pragma once
 
 #include "common.cuh"
@@ -64,20 +67,23 @@ constexpr int kStagesB = 3;
 constexpr int kChunkRows = 16;        // rows of a down tile per reduction chunk
 constexpr int kXStride = 17;          // fp32 words per row of the g/u exchange chunk
 // shared memory after the rings: barriers + flags (512 B), token ids,
-// g/u exchange chunk [128][17] fp32; then the E tile [N][64] bf16
+// g/u exchange chunk [128][17] fp32; then the E tile [N][features per tile] bf16
 constexpr int kTailFixed = 512 + kMaxN * 4 + 128 * kXStride * 4;
+// features per gate/up tile: 64 W_gate over the matching 64 W_up rows, or
+// (STEM) 128 W_gate rows
+template <bool kStem>
+constexpr int tile_features() { return kStem ? 128 : 64; }
 
 struct Params {
   int32_t T, N, D, F;
   int32_t sub;         // k blocks per unit (and per pipeline stage)
   int32_t stages;      // depth of the weight ring
   int32_t stages_b;    // depth of the activation ring
-  int32_t G;           // gate/up tiles (F / 64)
+  int32_t G;           // gate/up tiles (F / features per tile)
   int32_t Dt;          // down tiles (ceil(D / 128))
   int32_t ug, ud;      // units per gate/up tile, per down tile
   int32_t Ud;          // down units (Dt * ud)
   int32_t maxp_d;      // partial slots per down tile
-  int32_t rcap;        // partial slices per reduction batch (ring memory / slice)
   int32_t stage_tmem;  // stage down-unit weights in spare tensor memory
   // activations / outputs
   uint16_t* z;
@@ -90,10 +96,8 @@ struct Params {
   int64_t e_rows;
   int32_t e_mode;
   // workspace
-  uint32_t* cnt;       // [Dt] pieces finished per down tile
-  uint32_t* ready;     // [G] gate/up tile finished
-  uint32_t* queue;     // [2]: next chunk to reduce, events seen
-  float* part;         // [Dt * maxp_d][N][128]
+  uint32_t* ready;     // [G] gate/up tile finished (reset by the split-k sum kernel)
+  float* part;         // [Dt * maxp_d][N][128] fp32 partial sums, summed by the next kernel
   int32_t* err;
   uint64_t wait_ns;    // bound of every wait and flag spin (STAPLE_ETIMEOUT past it)
 };
@@ -113,14 +117,12 @@ __host__ __device__ inline int owner(int x, int U, int grid) {
 // flag rises later the further it sits in its block's range.  The lateness of
 // down unit x is the largest such position among the tiles that make the z
 // columns x reads (0 when each is its block's first tile).
+template <int FT>
 __device__ inline int unit_lateness(int x, const Params& p, int grid) {
-  const int u = x % p.ud;
+  const int f_lo = (x % p.ud) * p.sub * BK, f_hi = min(p.F, f_lo + p.sub * BK);
   int late = 0;
-  for (int j = 0; j < p.sub; ++j) {
-    const int t = u * p.sub + j;  // gate/up tile: 64 features = one 64-wide k block of z
-    if (t >= p.G) break;
+  for (int t = f_lo / FT; t <= (f_hi - 1) / FT; ++t)
     late = max(late, t - range_start(owner(t, p.G, grid), p.G, grid));
-  }
   return late;
 }
 
@@ -139,9 +141,6 @@ __device__ __forceinline__ void st_release(uint32_t* a, uint32_t v) {
 }
 __device__ __forceinline__ void fence_async_global() {
   asm volatile("fence.proxy.async.global;" ::: "memory");
-}
-__device__ __forceinline__ float4 ldcg4(const float* a) {
-  return __ldcg(reinterpret_cast<const float4*>(a));
 }
 __device__ __forceinline__ void add4(float4& a, const float4 b) {
   a.x += b.x;
@@ -172,14 +171,15 @@ __device__ __forceinline__ bool spin_until(const uint32_t* a, uint32_t want, vol
 // kOrder false that code is compiled out, which keeps the kernel body small
 // (the gate/up epilogue runs while the memory queues are full, where extra
 // code shows up as instruction-fetch stalls).
-template <bool kOrder>
+template <bool kOrder, bool kStem>
 __global__ void __launch_bounds__(kThreads, 1)
     decode_fused_kernel(const __grid_constant__ CUtensorMap tm_wg,
                         const __grid_constant__ CUtensorMap tm_wu,
                         const __grid_constant__ CUtensorMap tm_wd,
                         const __grid_constant__ CUtensorMap tm_x,
                         const __grid_constant__ CUtensorMap tm_z,
-                        const __grid_constant__ CUtensorMap tm_part, const Params p) {
+                        const Params p) {
+  constexpr int FT = tile_features<kStem>();
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align_smem_1024(smem_raw);
   const int b_block = p.N * BK * 2;
@@ -202,7 +202,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   // set by an epilogue warp whose wait failed, read by all four after a
   // barrier, so every epilogue warp takes the same path through bar.sync
   int* s_epi_fail = s_flag + 1;
-  uint64_t* rbar = reinterpret_cast<uint64_t*>(tail + 320);  // partial slices landed
   uint64_t* obar = reinterpret_cast<uint64_t*>(tail + 328);  // down-step order written
   uint64_t* dbar = reinterpret_cast<uint64_t*>(tail + 336);  // MMA drain before TMEM is freed
   // Down-step order (blocks with at most kMaxOrder down units): within each
@@ -213,7 +212,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* s_order = tail + 448;  // [kMaxOrder] down step k -> unit d0 + s_order[k]
   int32_t* s_ids = reinterpret_cast<int32_t*>(tail + 512);            // [kMaxN]
   float* s_x = reinterpret_cast<float*>(s_ids + kMaxN);               // [128][kXStride]
-  uint16_t* s_e = reinterpret_cast<uint16_t*>(s_x + 128 * kXStride);  // [N][64]
+  uint16_t* s_e = reinterpret_cast<uint16_t*>(s_x + 128 * kXStride);  // [N][FT]
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -236,7 +235,38 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int nslots = p.stage_tmem ? int((512 - 2 * ncols) / slot_cols) : 0;
   const uint32_t tmem_cols = nslots > 0 ? 512 : 2 * ncols;
 
+  // the unit of the block's k-th down step
+  auto unit = [&](int k) { return d0 + (reorder ? int(s_order[k]) : k); };
+  const bool ordered = reorder && nd > 0;
+  // The weights of local step i into ring stage s (bytes counted on fullA[s]).
+  auto issue_weights = [&](int i, int s, uint64_t once) {
+    mbar_arrive_expect_tx(&fullA[s], a_stage);
+    uint8_t* a = sA + s * a_stage;
+    if (i < ngs) {
+      const int tile = t0 + i / p.ug, u = i % p.ug;
+      for (int j = 0; j < p.sub; ++j) {
+        const int k0 = (u * p.sub + j) * BK;
+        if (kStem) {   // 128 W_gate rows (the map's box is 128 rows)
+          tma_load_2d_hint(&tm_wg, &fullA[s], a + j * A_BLOCK, k0, tile * FT, once);
+        } else {       // 64 W_gate rows over the matching 64 W_up rows
+          tma_load_2d_hint(&tm_wg, &fullA[s], a + j * A_BLOCK, k0, tile * FT, once);
+          tma_load_2d_hint(&tm_wu, &fullA[s], a + j * A_BLOCK + A_BLOCK / 2, k0, tile * FT, once);
+        }
+      }
+    } else {
+      // one 3-D copy brings all `sub` k blocks of the unit
+      const int x = unit(i - ngs), tile = x / p.ud, u = x % p.ud;
+      tma_load_3d_hint(&tm_wd, &fullA[s], a, 0, tile * BM, u * p.sub, once);
+    }
+  };
+  // Weights depend on no earlier kernel and on nothing else of the set-up,
+  // so the weight loader (thread 0) fills the whole ring before the block
+  // barrier, while tensor memory is being allocated (the down steps of a
+  // block that orders them wait for the order, worked out after the barrier).
+  const int early = min(S, ordered ? ngs : nsteps);
   if (threadIdx.x == 0) {
+    tma_prefetch_desc(&tm_wg);
+    tma_prefetch_desc(kStem ? &tm_wd : &tm_wu);
     for (int s = 0; s < S; ++s) {
       mbar_init(&fullA[s], 1);
       mbar_init(&emptyA[s], 1);
@@ -249,18 +279,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&tfull[b], 1);
       mbar_init(&tempty[b], 4);
     }
-    mbar_init(rbar, 1);
     mbar_init(obar, 1);
     mbar_init(dbar, 1);
     *abort_flag = 0;
     *s_epi_fail = 0;
     fence_barrier_init();
-    tma_prefetch_desc(&tm_wg);
-    tma_prefetch_desc(&tm_wu);
+    const uint64_t once = l2_policy_evict_first();
+    for (int i = 0; i < early; ++i) issue_weights(i, i, once);
     tma_prefetch_desc(&tm_wd);
     tma_prefetch_desc(&tm_x);
     tma_prefetch_desc(&tm_z);
-    tma_prefetch_desc(&tm_part);
   }
   if (warp == 1) {
     tmem_alloc(tmem_slot, tmem_cols);
@@ -270,15 +298,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
-  // the unit of the block's k-th down step
-  auto unit = [&](int k) { return d0 + (reorder ? int(s_order[k]) : k); };
   // The step order is worked out by an epilogue warp (idle until the first
   // gate/up tile is done), off the path of the first weight loads; the
   // loaders wait for it on obar before their first down step.
-  const bool ordered = reorder && nd > 0;
   if (warp == 3 && ordered) {
     for (int k = lane; k < nd; k += 32)
-      s_late[k] = uint8_t(min(255, unit_lateness(d0 + k, p, grid)));
+      s_late[k] = uint8_t(min(255, unit_lateness<FT>(d0 + k, p, grid)));
     __syncwarp();
     if (lane == 0) {
       int pos = 0;
@@ -299,26 +324,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       // ---------------------------------------------------- weight (A) loads
       const uint64_t once = l2_policy_evict_first();  // weights are read once per call
-      int s = 0;
-      uint32_t ph = 0;
-      int issued = 0;
-      for (int i = 0; i < nsteps; ++i) {
+      // the first `early` steps went out before the block barrier
+      int s = early % S;
+      uint32_t ph = early == S ? 1u : 0u;
+      int issued = early;
+      for (int i = early; i < nsteps; ++i) {
         if (i == ngs && ordered && !mbar_wait(obar, 0, abort_flag, p.err, p.wait_ns)) break;
         if (!mbar_wait(&emptyA[s], ph ^ 1, abort_flag, p.err, p.wait_ns)) break;
-        mbar_arrive_expect_tx(&fullA[s], a_stage);
-        uint8_t* a = sA + s * a_stage;
-        for (int j = 0; j < p.sub; ++j) {
-          if (i < ngs) {
-            const int tile = t0 + i / p.ug, u = i % p.ug;
-            const int k0 = (u * p.sub + j) * BK;
-            tma_load_2d_hint(&tm_wg, &fullA[s], a + j * A_BLOCK, k0, tile * 64, once);
-            tma_load_2d_hint(&tm_wu, &fullA[s], a + j * A_BLOCK + A_BLOCK / 2, k0, tile * 64, once);
-          } else if (j == 0) {
-            // one 3-D copy brings all `sub` k blocks of the unit
-            const int x = unit(i - ngs), tile = x / p.ud, u = x % p.ud;
-            tma_load_3d_hint(&tm_wd, &fullA[s], a, 0, tile * BM, u * p.sub, once);
-          }
-        }
+        issue_weights(i, s, once);
         ++issued;
         if (++s == S) {
           s = 0;
@@ -361,10 +374,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool mine = true;
       for (int k = lane; k < nd && mine; k += 32) {
         if (reorder && ((s_late[k] != 0) != late_round)) continue;
-        // unit d0 + k reads z columns [f_lo, f_hi), made by tiles f_lo/64 .. (f_hi-1)/64
+        // unit d0 + k reads z columns [f_lo, f_hi), made by tiles f_lo/FT .. (f_hi-1)/FT
         const int f_lo = ((d0 + k) % p.ud) * p.sub * BK;
         const int f_hi = min(p.F, f_lo + p.sub * BK);
-        for (int t = f_lo / 64; t <= (f_hi - 1) / 64 && mine; ++t)
+        for (int t = f_lo / FT; t <= (f_hi - 1) / FT && mine; ++t)
           mine = spin_until(&p.ready[t], 1u, abort_flag, p.err, p.wait_ns);
       }
       return __all_sync(0xffffffffu, mine);
@@ -529,29 +542,30 @@ __global__ void __launch_bounds__(kThreads, 1)
     int piece = 0;
     bool alive = true;
     // ---- phase 1: whole gate/up tiles, finished from tensor memory
+    constexpr int kVecs = FT / 8;   // 16-byte pieces of a token's E row slice
     for (int tile = t0; tile < t1 && alive; ++tile, ++piece) {
-      const int f0 = tile * 64;
-      // E[id_t][f0 .. f0+63] for every token: 128 bytes per row, 16-byte loads
-      // issued while the tile's main loop is still streaming.  Up to 8 loads
-      // per thread are put in flight before any of them is stored (behind a
-      // saturated weight stream each round trip is long).
-      for (int vb = et; vb < p.T * 8; vb += 8 * 128) {
+      const int f0 = tile * FT;
+      // E[id_t][f0 .. f0+FT) for every token, 16-byte loads issued while the
+      // tile's main loop is still streaming.  Up to 8 loads per thread are
+      // put in flight before any of them is stored (behind a saturated weight
+      // stream each round trip is long).
+      for (int vb = et; vb < p.T * kVecs; vb += 8 * 128) {
         uint4 w[8];
 #pragma unroll
         for (int k = 0; k < 8; ++k) {
           const int v = vb + k * 128;
           w[k] = make_uint4(0u, 0u, 0u, 0u);
-          if (v < p.T * 8) {
-            const int id = s_ids[v >> 3];
+          if (v < p.T * kVecs) {
+            const int id = s_ids[v / kVecs];
             if (id >= 0)
               w[k] = __ldg(reinterpret_cast<const uint4*>(p.e_base + int64_t(id) * p.e_pitch + f0) +
-                           (v & 7));
+                           (v % kVecs));
           }
         }
 #pragma unroll
         for (int k = 0; k < 8; ++k) {
           const int v = vb + k * 128;
-          if (v < p.T * 8) reinterpret_cast<uint4*>(s_e)[v] = w[k];
+          if (v < p.T * kVecs) reinterpret_cast<uint4*>(s_e)[v] = w[k];
         }
       }
       const int buf = piece & 1;
@@ -571,40 +585,50 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int j = 0; j < 16; ++j) s_x[row * kXStride + j] = __uint_as_float(r[j]);
         epi_bar();
-        // thread -> token c + et / 8, features 8 (et % 8) .. +7: one 16-byte
-        // store per output row piece (the memory system is saturated by the
-        // weight stream here, so the number of stores is what costs)
-        const int j = et >> 3, fl0 = (et & 7) * 8, t = c + j;
+        // thread -> token c + et / 8, features FT/8 (et % 8) .. +FT/8-1, in
+        // 16-byte stores (the memory system is saturated by the weight stream
+        // here, so the number of stores is what costs).  Rows f and 64 + f of
+        // the chunk are g and u of feature f; for STEM all 128 rows are g.
+        const int j = et >> 3, t = c + j;
         if (t < p.T) {
-          const uint4 ev = *reinterpret_cast<const uint4*>(s_e + t * 64 + fl0);
-          const uint32_t ew[4] = {ev.x, ev.y, ev.z, ev.w};
-          uint32_t zw[4], gw[4], hw[4];
 #pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            const int f = fl0 + 2 * k;
-            const float g0 = s_x[f * kXStride + j], g1 = s_x[(f + 1) * kXStride + j];
-            const float h0 = s_x[(64 + f) * kXStride + j] + bf_lo(ew[k]);
-            const float h1 = s_x[(65 + f) * kXStride + j] + bf_hi(ew[k]);
-            zw[k] = pack_bf2(g0 * sigmoid_f(g0) * h0, g1 * sigmoid_f(g1) * h1);
-            gw[k] = pack_bf2(g0, g1);
-            hw[k] = pack_bf2(h0, h1);
+          for (int half = 0; half < FT / 64; ++half) {
+            const int fl0 = (et & 7) * (FT / 8) + half * 8;
+            const uint4 ev = *reinterpret_cast<const uint4*>(s_e + t * FT + fl0);
+            const uint32_t ew[4] = {ev.x, ev.y, ev.z, ev.w};
+            uint32_t zw[4], gw[4], hw[4];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              const int f = fl0 + 2 * k;
+              const float g0 = s_x[f * kXStride + j], g1 = s_x[(f + 1) * kXStride + j];
+              const float h0 = kStem ? bf_lo(ew[k]) : s_x[(64 + f) * kXStride + j] + bf_lo(ew[k]);
+              const float h1 = kStem ? bf_hi(ew[k]) : s_x[(65 + f) * kXStride + j] + bf_hi(ew[k]);
+              zw[k] = pack_bf2(g0 * sigmoid_f(g0) * h0, g1 * sigmoid_f(g1) * h1);
+              gw[k] = pack_bf2(g0, g1);
+              hw[k] = pack_bf2(h0, h1);
+            }
+            const int64_t off = int64_t(t) * p.F + f0 + fl0;
+            *reinterpret_cast<uint4*>(p.z + off) = make_uint4(zw[0], zw[1], zw[2], zw[3]);
+            if (p.g_save)
+              *reinterpret_cast<uint4*>(p.g_save + off) = make_uint4(gw[0], gw[1], gw[2], gw[3]);
+            if (p.h_save)
+              *reinterpret_cast<uint4*>(p.h_save + off) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
           }
-          const int64_t off = int64_t(t) * p.F + f0 + fl0;
-          *reinterpret_cast<uint4*>(p.z + off) = make_uint4(zw[0], zw[1], zw[2], zw[3]);
-          if (p.g_save)
-            *reinterpret_cast<uint4*>(p.g_save + off) = make_uint4(gw[0], gw[1], gw[2], gw[3]);
-          if (p.h_save)
-            *reinterpret_cast<uint4*>(p.h_save + off) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
         }
         epi_bar();
       }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&tempty[buf]);
-      __threadfence();
-      fence_async_global();
-      epi_bar();
-      if (et == 0) st_release(&p.ready[tile], 1u);
+      // The last epi_bar ordered every thread's z stores before this point
+      // (CTA scope); one thread's gpu-scope fence and release store then
+      // publish all of them (a release is cumulative), and the consumers'
+      // TMA loads of z follow their acquire of the flag.
+      if (et == 0) {
+        __threadfence();
+        fence_async_global();
+        st_release(&p.ready[tile], 1u);
+      }
     }
     // ---- phase 2: down pieces -> fp32 partial slots
     for (int x = d0; x < d1 && alive; ++piece) {
@@ -635,133 +659,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&tempty[buf]);
-      __threadfence();
-      epi_bar();
-      if (et == 0) atomicAdd(&p.cnt[tile], 1u);
     }
-
-    // ---- down sums: 16-row chunks from the shared work queue.  queue[0]
-    // hands out chunks; queue[1] counts events: each reduced chunk and each
-    // block's final fetch past the end.  The event that completes the count
-    // (nchunks + grid) is the last use of any counter or flag of this call,
-    // so that thread resets them all for the next call.
-    const int chunks_per_tile = BM / kChunkRows;
-    const uint32_t nchunks = uint32_t(p.Dt * chunks_per_tile);
-    const uint32_t nevents = nchunks + uint32_t(grid);
-    // slices land in the ring memory, idle once this block's MMAs are done
-    uint8_t* rbuf = sA;
-    const int slice = p.N * kChunkRows * 4;   // bytes of one piece's [N][16] fp32 slice
-    uint32_t rph = 0;
-    // thread et == 0 issues the slice loads; a batch it issued and has not
-    // seen land (after an abort) is waited for before the block exits
-    bool r_pending = false;
-    uint32_t r_phase = 0;
-    auto event = [&]() {
-      if (atomicAdd(&p.queue[1], 1u) == nevents - 1) {
-        for (int k = 0; k < p.Dt; ++k) p.cnt[k] = 0u;
-        for (int k = 0; k < p.G; ++k) p.ready[k] = 0u;
-        p.queue[0] = 0u;
-        p.queue[1] = 0u;
-        __threadfence();
-      }
-    };
-    // thread et owns the float4 groups g = et + 128 m (token g / 4, rows
-    // 4 (g % 4) .. +3 of the chunk); kMaxN * 4 groups at most
-    constexpr int kGroups = kMaxN * (kChunkRows / 4) / 128;
-    while (alive) {
-      // one thread takes a chunk, waits for its tile and puts the first batch
-      // of slice loads in flight; all follow its verdict
-      epi_bar();
-      if (et == 0) {
-        int code = int(atomicAdd(&p.queue[0], 1u));
-        if (code < int(nchunks)) {
-          const int tl = code / chunks_per_tile;
-          const int first = owner(tl * p.ud, p.Ud, grid);
-          const int np = owner((tl + 1) * p.ud - 1, p.Ud, grid) - first + 1;
-          if (!spin_until(&p.cnt[tl], uint32_t(np), abort_flag, p.err, p.wait_ns)) {
-            code = -1;
-          } else {
-            fence_async_global();
-            const int nb = min(np, p.rcap);
-            const int r0 = (code % chunks_per_tile) * kChunkRows;
-            r_pending = true;
-            r_phase = rph;
-            mbar_arrive_expect_tx(rbar, uint32_t(nb * slice));
-            for (int i = 0; i < nb; ++i)
-              tma_load_2d(&tm_part, rbar, rbuf + i * slice, r0, (tl * p.maxp_d + i) * p.N);
-          }
-        }
-        *s_flag = code;
-      }
-      epi_bar();
-      const int code = *s_flag;
-      if (code < 0) break;
-      const uint32_t c = uint32_t(code);
-      if (c >= nchunks) {
-        if (et == 0) event();
-        break;
-      }
-      const int tile = int(c) / chunks_per_tile;
-      const int r0 = (int(c) % chunks_per_tile) * kChunkRows;
-      const int o0 = owner(tile * p.ud, p.Ud, grid);
-      const int npieces = owner((tile + 1) * p.ud - 1, p.Ud, grid) - o0 + 1;
-      const int ngroups = p.T * (kChunkRows / 4);
-      float4 acc[kGroups];
-#pragma unroll
-      for (int m = 0; m < kGroups; ++m) acc[m] = make_float4(0.f, 0.f, 0.f, 0.f);
-      bool ok = true;
-      for (int i0 = 0; i0 < npieces; i0 += p.rcap) {
-        const int nb = min(npieces - i0, p.rcap);
-        if (i0 > 0) {
-          epi_bar();  // the previous batch has been read
-          if (et == 0) {
-            r_pending = true;
-            r_phase = rph;
-            mbar_arrive_expect_tx(rbar, uint32_t(nb * slice));
-            for (int i = 0; i < nb; ++i)
-              tma_load_2d(&tm_part, rbar, rbuf + i * slice, r0,
-                          (tile * p.maxp_d + i0 + i) * p.N);
-          }
-        }
-        ok = mbar_wait(rbar, rph, abort_flag, p.err, p.wait_ns);
-        if (ok && et == 0) r_pending = false;
-        rph ^= 1u;
-        if (!__all_sync(0xffffffffu, ok) && lane == 0) *s_epi_fail = 1;
-        epi_bar();
-        if (*s_epi_fail) {
-          ok = false;
-          break;
-        }
-        for (int i = 0; i < nb; ++i) {
-          const float4* sl = reinterpret_cast<const float4*>(rbuf + i * slice);
-#pragma unroll
-          for (int m = 0; m < kGroups; ++m) {
-            const int gi = et + 128 * m;
-            if (gi < ngroups) add4(acc[m], sl[gi]);
-          }
-        }
-      }
-      if (!ok) break;
-#pragma unroll
-      for (int m = 0; m < kGroups; ++m) {
-        const int gi = et + 128 * m;
-        if (gi >= ngroups) continue;
-        const int t = gi >> 2, d = tile * BM + r0 + (gi & 3) * 4;
-        uint16_t* dst = p.y + int64_t(t) * p.D + d;
-        if (d + 3 < p.D) {
-          uint2 w;
-          w.x = pack_bf2(acc[m].x, acc[m].y);
-          w.y = pack_bf2(acc[m].z, acc[m].w);
-          *reinterpret_cast<uint2*>(dst) = w;
-        } else {
-          const float a[4] = {acc[m].x, acc[m].y, acc[m].z, acc[m].w};
-          for (int k = 0; k < 4 && d + k < p.D; ++k)
-            dst[k] = __bfloat16_as_ushort(__float2bfloat16_rn(a[k]));
-        }
-      }
-      if (et == 0) event();
-    }
-    if (et == 0 && r_pending) mbar_drain(rbar, r_phase);
   }
 
   tc_fence_before();
@@ -773,24 +671,89 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-// Shared memory after the rings for N tokens.
-inline int tail_bytes(int N) { return kTailFixed + N * 64 * 2; }
+// ---------------------------------------------------------------------------
+// The split-k sum of the down projection, a kernel of its own.  It is
+// launched as a programmatic dependent of the decode kernel, right behind it:
+// its blocks (small, no shared memory) start early and release the next
+// kernel in the stream at once, then wait for the decode kernel to complete,
+// so every partial slot is written and visible and nothing needs to be
+// counted or polled; meanwhile the next decode kernel's blocks take the SMs
+// the decode kernel left and start streaming their weights.  Block b sums
+// 16-row chunk b % 8 of down tile b / 8 over the tile's pieces, in piece
+// order (deterministic), and writes y = bf16(sum); block 0 also clears the
+// gate/up ready flags for the next call.
+// ---------------------------------------------------------------------------
+constexpr int kReduceThreads = 256;
+
+struct ReduceParams {
+  int32_t T, N, D;
+  int32_t G;           // ready flags to clear
+  int32_t ud, Ud;      // down units per tile, in all
+  int32_t grid;        // the decode kernel's grid (its stream-K ranges)
+  int32_t maxp_d;      // partial slots per down tile
+  const float* part;   // [Dt * maxp_d][N][128]
+  uint16_t* y;
+  uint32_t* ready;
+};
+
+__global__ void __launch_bounds__(kReduceThreads)
+    decode_reduce_kernel(const ReduceParams r) {
+  grid_dep_launch();
+  grid_dep_wait();
+  if (blockIdx.x == 0)
+    for (int k = threadIdx.x; k < r.G; k += kReduceThreads) r.ready[k] = 0u;
+  const int tile = blockIdx.x / (BM / kChunkRows);
+  const int r0 = (blockIdx.x % (BM / kChunkRows)) * kChunkRows;
+  if (tile * BM + r0 >= r.D) return;
+  const int first = owner(tile * r.ud, r.Ud, r.grid);
+  const int np = owner((tile + 1) * r.ud - 1, r.Ud, r.grid) - first + 1;
+  const float* base = r.part + int64_t(tile) * r.maxp_d * r.N * BM;
+  // thread -> float4 groups g = tid + 256 m: token g / 4, rows 4 (g % 4) .. +3
+  // of the chunk; pieces go in batches whose loads are all in flight at once
+  constexpr int kBatch = 8;
+  const int ngroups = r.T * (kChunkRows / 4);
+  for (int g = threadIdx.x; g < ngroups; g += kReduceThreads) {
+    const int t = g >> 2;
+    const int64_t off = int64_t(t) * BM + r0 + (g & 3) * 4;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int i0 = 0; i0 < np; i0 += kBatch) {
+      float4 v[kBatch];
+#pragma unroll
+      for (int i = 0; i < kBatch; ++i)
+        if (i0 + i < np)
+          v[i] = __ldcg(reinterpret_cast<const float4*>(base + int64_t(i0 + i) * r.N * BM + off));
+#pragma unroll
+      for (int i = 0; i < kBatch; ++i)
+        if (i0 + i < np) add4(acc, v[i]);
+    }
+    const int d = tile * BM + r0 + (g & 3) * 4;
+    uint16_t* dst = r.y + int64_t(t) * r.D + d;
+    if (d + 3 < r.D) {
+      uint2 w;
+      w.x = pack_bf2(acc.x, acc.y);
+      w.y = pack_bf2(acc.z, acc.w);
+      *reinterpret_cast<uint2*>(dst) = w;
+    } else {
+      const float a[4] = {acc.x, acc.y, acc.z, acc.w};
+      for (int k = 0; k < 4 && d + k < r.D; ++k)
+        dst[k] = __bfloat16_as_ushort(__float2bfloat16_rn(a[k]));
+    }
+  }
+}
+
+// Shared memory after the rings for N tokens and FT features per gate/up tile.
+inline int tail_bytes(int N, int FT) { return kTailFixed + N * FT * 2; }
 // Ring depths: the activation ring keeps kStagesB stages (it is fed from
 // L2), the weight ring takes the rest of shared memory.
 inline int stages_b(int N, int sub) { (void)N; (void)sub; return kStagesB; }
-inline int ring_stages(int N, int sub) {
-  const int budget = 227 * 1024 - 1024 - tail_bytes(N) - stages_b(N, sub) * sub * N * BK * 2;
+inline int ring_stages(int N, int sub, int FT) {
+  const int budget = 227 * 1024 - 1024 - tail_bytes(N, FT) - stages_b(N, sub) * sub * N * BK * 2;
   const int s = budget / (sub * A_BLOCK);
   return s > kMaxStages ? kMaxStages : s;
 }
-// Partial slices (one piece's [N][16] fp32) that fit in the two rings.
-inline int reduce_slices(int N, int sub) {
-  const int ring = ring_stages(N, sub) * sub * A_BLOCK + stages_b(N, sub) * sub * N * BK * 2;
-  return ring / (N * kChunkRows * 4);
-}
-inline int smem_bytes(int N, int sub) {
-  return 1024 + ring_stages(N, sub) * sub * A_BLOCK + stages_b(N, sub) * sub * N * BK * 2 +
-         tail_bytes(N);
+inline int smem_bytes(int N, int sub, int FT) {
+  return 1024 + ring_stages(N, sub, FT) * sub * A_BLOCK + stages_b(N, sub) * sub * N * BK * 2 +
+         tail_bytes(N, FT);
 }
 
 }  // namespace fused

@@ -131,7 +131,7 @@ staple_status launch(const char* name, const DeviceInfo& di, const CUtensorMap& 
       return STAPLE_ECUDA;
     attr_done.fetch_or(bit);
   }
-  const int grid = std::min(ntiles, di.num_sms);
+  const int grid = std::min(ntiles, std::max(1, di.num_sms - di.sm_reserve));
   const CUtensorMap& o0 = o ? o[0] : a;
   const CUtensorMap& o1 = o ? o[1] : a;
   const CUtensorMap& o2 = o ? o[2] : a;
@@ -167,11 +167,12 @@ int piece_bound(int units, int U) {
   return std::min(kMaxDecodeGrid, (units - 1) / minlen + 2);
 }
 
-DecodePlan plan_decode(int T, int D, int F, int num_sms) {
+// FT: features per gate/up tile (64: W_gate over W_up rows; 128: STEM, W_gate alone)
+DecodePlan plan_decode(int T, int D, int F, int FT, int num_sms) {
   DecodePlan pl{};
   pl.N = cdiv(T, 16) * 16;
-  pl.sub = ((D / 64) % 2 == 0 && (F / 64) % 2 == 0 && fused::ring_stages(pl.N, 2) >= 3) ? 2 : 1;
-  pl.G = F / 64;
+  pl.sub = ((D / 64) % 2 == 0 && (F / 64) % 2 == 0 && fused::ring_stages(pl.N, 2, FT) >= 3) ? 2 : 1;
+  pl.G = F / FT;
   pl.Dt = cdiv(D, fused::BM);
   pl.ug = (D / 64) / pl.sub;
   pl.ud = (F / 64) / pl.sub;
@@ -201,8 +202,9 @@ size_t decode_counter_bytes(int D, int F) {
 
 size_t decode_scratch_bytes(int T, int D, int F) {
   if (T < 1 || T > kMaxDecodeT || D % 64 || F % 64) return 0;
-  // the largest grid the launcher may use gives the most pieces per tile
-  const DecodePlan pl = plan_decode(T, D, F, kMaxDecodeGrid);
+  // the largest grid the launcher may use gives the most pieces per tile (the
+  // partial slots do not depend on the gate/up tiling)
+  const DecodePlan pl = plan_decode(T, D, F, 64, kMaxDecodeGrid);
   return pl.part_bytes;
 }
 
@@ -210,16 +212,15 @@ staple_status tc_decode_fwd(const DeviceInfo& di, int T, int D, int F, const voi
                             const staple_embed* e, const void* wg, const void* wu, const void* wd,
                             void* z, void* y, void* g_save, void* h_save, void* ws,
                             int32_t* err, cudaStream_t st) {
-  const DecodePlan pl = plan_decode(T, D, F, di.num_sms);
+  const bool stem = e && (e->flags & STAPLE_EMBED_REPLACE_UP);
+  const int FT = stem ? 128 : 64;
+  if (F % FT) return STAPLE_EUNSUPPORTED;
+  const DecodePlan pl = plan_decode(T, D, F, FT, di.num_sms);
   void* part = static_cast<uint8_t*>(ws) + pl.counter_bytes;
-  CUtensorMap mg, mu, md, mx, mz, mp;
-  if (!kmajor_rows(&mg, wg, F, D, D, 64) || !kmajor_rows(&mu, wu, F, D, D, 64) ||
+  CUtensorMap mg, mu, md, mx, mz;
+  if (!kmajor_rows(&mg, wg, F, D, D, FT) || !kmajor_rows(&mu, stem ? wg : wu, F, D, D, 64) ||
       !kmajor_blocks(&md, wd, D, F, F, fused::BM, pl.sub) ||
-      !kmajor_blocks(&mx, x, T, D, D, pl.N, pl.sub) || !kmajor_blocks(&mz, z, T, F, F, pl.N, pl.sub) ||
-      // partial slots [Dt * maxp_d * N][128] fp32; a box is one piece's
-      // 16-row slice for all N tokens
-      !make_map_f32(&mp, part, fused::BM, uint64_t(pl.Dt) * pl.maxp_d * pl.N, fused::BM,
-                    fused::kChunkRows, uint32_t(pl.N)))
+      !kmajor_blocks(&mx, x, T, D, D, pl.N, pl.sub) || !kmajor_blocks(&mz, z, T, F, F, pl.N, pl.sub))
     return STAPLE_ECUDA;
   fused::Params p{};
   p.T = T;
@@ -227,7 +228,7 @@ staple_status tc_decode_fwd(const DeviceInfo& di, int T, int D, int F, const voi
   p.D = D;
   p.F = F;
   p.sub = pl.sub;
-  p.stages = fused::ring_stages(pl.N, pl.sub);
+  p.stages = fused::ring_stages(pl.N, pl.sub, FT);
   p.stages_b = fused::stages_b(pl.N, pl.sub);
   p.G = pl.G;
   p.Dt = pl.Dt;
@@ -235,7 +236,6 @@ staple_status tc_decode_fwd(const DeviceInfo& di, int T, int D, int F, const voi
   p.ud = pl.ud;
   p.Ud = pl.Ud;
   p.maxp_d = pl.maxp_d;
-  p.rcap = fused::reduce_slices(pl.N, pl.sub);
   p.stage_tmem = 1;
   p.z = static_cast<uint16_t*>(z);
   p.g_save = static_cast<uint16_t*>(g_save);
@@ -249,35 +249,42 @@ staple_status tc_decode_fwd(const DeviceInfo& di, int T, int D, int F, const voi
     p.e_rows = e->n_rows;
   }
   uint32_t* words = static_cast<uint32_t*>(ws);
-  p.cnt = words;
-  p.ready = words + pl.Dt;
-  p.queue = words + pl.Dt + pl.G;
+  p.ready = words;
   p.part = static_cast<float*>(part);
   p.err = err;
   p.wait_ns = di.wait_ns;
 
   // down-step ordering only where some block makes two or more gate/up tiles
   const int order = pl.G > pl.grid ? 1 : 0;
-  auto kern = order ? fused::decode_fused_kernel<true> : fused::decode_fused_kernel<false>;
-  const int smem = fused::smem_bytes(pl.N, pl.sub);
+  using Kern = void (*)(CUtensorMap, CUtensorMap, CUtensorMap, CUtensorMap, CUtensorMap,
+                        fused::Params);
+  // [order][stem]
+  const Kern kerns[2][2] = {{fused::decode_fused_kernel<false, false>,
+                             fused::decode_fused_kernel<false, true>},
+                            {fused::decode_fused_kernel<true, false>,
+                             fused::decode_fused_kernel<true, true>}};
+  const Kern kern = kerns[order][stem ? 1 : 0];
+  const int smem = fused::smem_bytes(pl.N, pl.sub, FT);
   // Blocks wait (bounded) on flags other blocks raise, so the whole grid must
   // be resident at once.  Checked once per device, kernel and shared-memory
   // size (queried outside any stream capture on first use): the grid may not
   // exceed the SMs times the blocks one SM can hold.
-  static std::atomic<uint64_t> attr_done[2];
+  static std::atomic<uint64_t> attr_done{0};
   const uint64_t bit = uint64_t(1) << (di.device & 63);
-  if (!(attr_done[order].load() & bit)) {
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024) !=
-        cudaSuccess)
-      return STAPLE_ECUDA;
-    attr_done[order].fetch_or(bit);
+  if (!(attr_done.load() & bit)) {
+    for (const auto& row : kerns)
+      for (Kern k : row)
+        if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024) !=
+            cudaSuccess)
+          return STAPLE_ECUDA;
+    attr_done.fetch_or(bit);
   }
   int per_sm = 0;
   {
     static std::mutex mu;
-    static std::map<std::tuple<int, int, int>, int> resident;   // (order, device, smem)
+    static std::map<std::tuple<const void*, int, int>, int> resident;   // (kernel, device, smem)
     std::lock_guard<std::mutex> lock(mu);
-    const auto key = std::make_tuple(order, di.device, smem);
+    const auto key = std::make_tuple(reinterpret_cast<const void*>(kern), di.device, smem);
     auto it = resident.find(key);
     if (it == resident.end()) {
       if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, fused::kThreads, smem) !=
@@ -299,7 +306,28 @@ staple_status tc_decode_fwd(const DeviceInfo& di, int T, int D, int F, const voi
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   cudaError_t ce = cudaSuccess;
-  STP_LAUNCH("k5k6_decode_fused", st, ce = cudaLaunchKernelEx(&cfg, kern, mg, mu, md, mx, mz, mp, p));
+  STP_LAUNCH(stem ? "k5k6_decode_fused_stem" : "k5k6_decode_fused", st,
+             ce = cudaLaunchKernelEx(&cfg, kern, mg, mu, md, mx, mz, p));
+  if (ce != cudaSuccess) return STAPLE_ECUDA;
+  // the split-k sums, right behind (programmatic dependent, see the kernel)
+  fused::ReduceParams r{};
+  r.T = T;
+  r.N = pl.N;
+  r.D = D;
+  r.G = pl.G;
+  r.ud = pl.ud;
+  r.Ud = pl.Ud;
+  r.grid = pl.grid;
+  r.maxp_d = pl.maxp_d;
+  r.part = p.part;
+  r.y = p.y;
+  r.ready = p.ready;
+  cudaLaunchConfig_t rcfg = cfg;
+  rcfg.gridDim = dim3(pl.Dt * (fused::BM / fused::kChunkRows));
+  rcfg.blockDim = dim3(fused::kReduceThreads);
+  rcfg.dynamicSmemBytes = 0;
+  STP_LAUNCH("k6r_decode_reduce", st,
+             ce = cudaLaunchKernelEx(&rcfg, fused::decode_reduce_kernel, r));
   return ce == cudaSuccess ? STAPLE_OK : STAPLE_ECUDA;
 }
 
@@ -309,8 +337,9 @@ staple_status tc_ffn_fwd(const DeviceInfo& di, int T, int D, int F, const void* 
                          cudaStream_t st) {
   if (T == 0) return STAPLE_OK;
   CUtensorMap mx, mg, mu, mz, md;
-  if (!kmajor(&mx, x, T, D, D) || !kmajor(&mg, wg, F, D, D) || !kmajor(&mu, wu, F, D, D) ||
-      !kmajor(&mz, z, T, F, F) || !kmajor(&md, wd, D, F, F))
+  if (!kmajor(&mx, x, T, D, D) || !kmajor(&mg, wg, F, D, D) ||
+      !kmajor(&mu, wu ? wu : wg, F, D, D) || !kmajor(&mz, z, T, F, F) ||
+      !kmajor(&md, wd, D, F, F))
     return STAPLE_ECUDA;
   {
     tc::Params p{};
@@ -335,8 +364,16 @@ staple_status tc_ffn_fwd(const DeviceInfo& di, int T, int D, int F, const void* 
     if (!out_map(&mo[0], z, T, F, F) || !out_map(&mo[1], g_save ? g_save : z, T, F, F) ||
         !out_map(&mo[2], h_save ? h_save : z, T, F, F))
       return STAPLE_ECUDA;
-    staple_status s =
-        launch<false, false, tc::B_NHALF, tc::EPI_GATEUP>("k5_gateup", di, mx, mg, mu, p, st, mo);
+    staple_status s;
+    if (e && (e->flags & STAPLE_EMBED_REPLACE_UP)) {
+      // STEM: the gate projection alone, 256 features per tile
+      p.tiles_n = cdiv(F, tc::BN);
+      s = launch<false, false, tc::B_ONE, tc::EPI_GATE_E>("k5_gate_stem", di, mx, mg, mg, p, st,
+                                                            mo);
+    } else {
+      s = launch<false, false, tc::B_NHALF, tc::EPI_GATEUP>("k5_gateup", di, mx, mg, mu, p, st,
+                                                            mo);
+    }
     if (s != STAPLE_OK) return s;
   }
   tc::Params q{};
@@ -390,7 +427,25 @@ staple_status tc_ffn_bwd(const DeviceInfo& di, int T, int D, int F, const void* 
     if (dwd && cudaMemsetAsync(dwd, 0, size_t(F) * D * 4, st) != cudaSuccess) return STAPLE_ECUDA;
     return STAPLE_OK;
   }
-  if (dx) {
+  if (dx && !wu) {
+    // K9 of the STEM layer (no up-projection): dx = dg W_gate, A = the dg
+    // half of dgh (K = F, row pitch 2F), B(n = d, k = f) = W_gate[f][d]
+    CUtensorMap ma, mb0;
+    if (!kmajor(&ma, dgh, T, F, 2 * F) || !mnmajor(&mb0, wg, F, D, D)) return STAPLE_ECUDA;
+    tc::Params p{};
+    p.M = T;
+    p.N = D;
+    p.K = F;
+    p.tiles_m = cdiv(T, tc::BM);
+    p.tiles_n = cdiv(D, tc::BN);
+    p.out = dx;
+    p.ldo = D;
+    p.m_split = T;
+    p.err = err;
+    if ((s = launch<false, true, tc::B_ONE, tc::EPI_BF16>("k9_dx", di, ma, mb0, mb0, p, st)) !=
+        STAPLE_OK)
+      return s;
+  } else if (dx) {
     // K9: A = dgh [T][2F] K-major; B(n = d, k = f') = W_gate[f'][d] | W_up[f' - F][d]: MN-major
     CUtensorMap ma, mb0, mb1;
     if (!kmajor(&ma, dgh, T, 2 * F, 2 * F) || !mnmajor(&mb0, wg, F, D, D) ||

@@ -37,7 +37,9 @@ constexpr int kTmemCols = 512;
 constexpr int kSmemBytes = STAGES * STAGE_BYTES + 1024 /*align*/ + 256 /*barriers*/;
 
 enum BSrc { B_ONE = 0, B_NHALF = 1, B_KSPLIT = 2 };
-enum Epi { EPI_BF16 = 0, EPI_F32 = 1, EPI_GATEUP = 2, EPI_DZ = 3 };
+// EPI_GATE_E: the STEM variant of EPI_GATEUP (the row replaces the
+// up-projection): the tile is 256 W_gate rows, h = E[row], z = SiLU(g) h.
+enum Epi { EPI_BF16 = 0, EPI_F32 = 1, EPI_GATEUP = 2, EPI_DZ = 3, EPI_GATE_E = 4 };
 
 // The heavy epilogues stage every 32-row x 32-column output block of a warp
 // in shared memory (64-byte swizzle) and write it with one TMA store: a
@@ -45,7 +47,9 @@ enum Epi { EPI_BF16 = 0, EPI_F32 = 1, EPI_GATEUP = 2, EPI_DZ = 3 };
 // different row.  2 KB per block: z, g, h for EPI_GATEUP; dg, dh for EPI_DZ.
 constexpr int kOutBox = 32 * 32 * 2;
 template <int EPI>
-constexpr int out_blocks() { return EPI == EPI_GATEUP ? 3 : (EPI == EPI_DZ ? 2 : 0); }
+constexpr int out_blocks() {
+  return (EPI == EPI_GATEUP || EPI == EPI_GATE_E) ? 3 : (EPI == EPI_DZ ? 2 : 0);
+}
 template <int EPI>
 constexpr int smem_bytes() { return kSmemBytes + 4 * out_blocks<EPI>() * kOutBox; }
 
@@ -237,6 +241,48 @@ __device__ __forceinline__ void epilogue_tile(const Params& p, uint32_t tacc, in
         write_row_sw64(stg, lane, z);
         if (use[1]) write_row_sw64(stg + kOutBox, lane, g);
         if (use[2]) write_row_sw64(stg + 2 * kOutBox, lane, h);
+        stage_store(lane, stg, om, use, f, m0w);
+      }
+    }
+  } else if constexpr (EPI == EPI_GATE_E) {
+    // Accumulator columns [0,256): g for features f0..f0+255; h is the row.
+    const uint16_t* erow = nullptr;
+    if (row_ok && p.e_mode != STAPLE_EMBED_NONE) {
+      const int64_t idx = p.e_index[m];
+      if (idx < 0 || idx >= p.e_rows) {
+        report(p.err, STAPLE_EIDRANGE);
+      } else {
+        erow = p.e_base + idx * p.e_pitch;
+      }
+    }
+    const int f0 = nb * BN;
+    // the row's chunk c+1 is loaded while chunk c is computed
+    uint4 ew[4] = {};
+    if (erow && f0 < p.N) load_raw32(erow + f0, ew);
+#pragma unroll 1
+    for (int c = 0; c < BN / 32; ++c) {
+      uint4 ec[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) ec[i] = ew[i];
+      const int f = f0 + c * 32;
+      if (erow && c + 1 < BN / 32 && f + 32 < p.N) load_raw32(erow + f + 32, ew);
+      uint32_t rg[32];
+      tmem_ld32(tacc + c * 32, rg);
+      tmem_ld_wait(rg);
+      if (f < p.N) {   // the same for the whole warp
+        float e[32];
+        unpack32(ec, e);
+        float g[32], z[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          g[i] = __uint_as_float(rg[i]);
+          z[i] = g[i] * sigmoid_f(g[i]) * e[i];
+        }
+        const bool use[3] = {true, p.g_save != nullptr, p.h_save != nullptr};
+        stage_begin(lane);
+        write_row_sw64(stg, lane, z);
+        if (use[1]) write_row_sw64(stg + kOutBox, lane, g);
+        if (use[2]) write_row_sw64(stg + 2 * kOutBox, lane, e);
         stage_store(lane, stg, om, use, f, m0w);
       }
     }

@@ -19,6 +19,7 @@ struct DeviceInfo {
   int device;
   int num_sms;
   uint64_t wait_ns;   // bound of every kernel wait (staple_set_wait_limit)
+  int sm_reserve;     // SMs the persistent GEMMs leave free (staple_set_sm_reserve)
 };
 
 // trace.cu: optional per-kernel CUDA-event timing of a context

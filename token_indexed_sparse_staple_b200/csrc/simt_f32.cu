@@ -179,7 +179,11 @@ staple_status f32_ffn_fwd(int T, int D, int F, const float* x, const staple_embe
     p.e_rows = e->n_rows;
   }
   p.err = err;
-  staple_status s = run<false, false, S_GATEUP, true>(p, st);
+  // STEM (the row replaces the up-projection): the gate product alone, and
+  // the epilogue's second accumulator stays zero, so h = E[row]
+  const bool stem = e && (e->flags & STAPLE_EMBED_REPLACE_UP);
+  staple_status s = stem ? run<false, false, S_GATEUP, false>(p, st)
+                         : run<false, false, S_GATEUP, true>(p, st);
   if (s != STAPLE_OK) return s;
   SParams q{};
   q.M = T; q.N = D; q.K = F;
@@ -203,10 +207,11 @@ staple_status f32_ffn_bwd(int T, int D, int F, const float* dy, const float* x, 
                           float* dwg, float* dwu, float* dwd, cudaStream_t st) {
   staple_status s;
   if (dx) {
-    // dx [T][D] = dgh [T][2F] . [W_gate; W_up] ([2F][D], n = d contiguous)
+    // dx [T][D] = dgh [T][2F] . [W_gate; W_up] ([2F][D], n = d contiguous);
+    // without an up-projection (STEM) only the dg half: dx = dg W_gate
     SParams p{};
-    p.M = T; p.N = D; p.K = 2 * F;
-    p.A = dgh; p.lda = 2 * F; p.B0 = wg; p.B1 = wu; p.ldb = D; p.ksplit = F;
+    p.M = T; p.N = D; p.K = wu ? 2 * F : F;
+    p.A = dgh; p.lda = 2 * F; p.B0 = wg; p.B1 = wu; p.ldb = D; p.ksplit = wu ? F : 0;
     p.out = dx; p.ldo = D; p.m_split = T;
     if ((s = run<false, true, S_STORE, false>(p, st)) != STAPLE_OK) return s;
   }

@@ -68,7 +68,13 @@ staple_status set_device(const staple_context* ctx) {
     if ((expr) != cudaSuccess) return STAPLE_ECUDA;           \
   } while (0)
 
+inline bool replaces_up(const staple_embed* e) {
+  return e && (e->flags & STAPLE_EMBED_REPLACE_UP);
+}
+
 staple_status check_embed(const staple_embed* e, staple_dtype dt, int F) {
+  if (e && (e->flags & ~uint32_t(STAPLE_EMBED_REPLACE_UP))) return STAPLE_EINVAL;
+  if (replaces_up(e) && e->mode == STAPLE_EMBED_NONE) return STAPLE_EINVAL;
   if (!e || e->mode == STAPLE_EMBED_NONE) return STAPLE_OK;
   if (e->mode != STAPLE_EMBED_TABLE && e->mode != STAPLE_EMBED_ROWS) return STAPLE_EINVAL;
   if (!e->base || !e->index || e->n_rows <= 0 || e->row_pitch < F) return STAPLE_EINVAL;
@@ -142,6 +148,7 @@ staple_status staple_context_create(int device, staple_context** out) {
   c->di.device = device;
   c->di.num_sms = prop.multiProcessorCount;
   c->di.wait_ns = stp::kWaitLimitNs;
+  c->di.sm_reserve = 0;
   if (lib_malloc(reinterpret_cast<void**>(&c->d_err), sizeof(int32_t), "context_err") !=
       cudaSuccess) {
     cudaGetLastError();
@@ -163,6 +170,12 @@ staple_status staple_context_create(int device, staple_context** out) {
 staple_status staple_set_wait_limit(staple_context* ctx, int64_t limit_ns) {
   if (!ctx || limit_ns < 1 || limit_ns > stp::kMaxWaitLimitNs) return STAPLE_EINVAL;
   ctx->di.wait_ns = uint64_t(limit_ns);
+  return STAPLE_OK;
+}
+
+staple_status staple_set_sm_reserve(staple_context* ctx, int32_t sms) {
+  if (!ctx || sms < 0 || sms > ctx->di.num_sms / 4) return STAPLE_EINVAL;
+  ctx->di.sm_reserve = sms;
   return STAPLE_OK;
 }
 
@@ -538,7 +551,8 @@ staple_status staple_ffn_fwd(staple_context* ctx, staple_dtype dtype, int32_t T,
                  workspace_bytes < stp::decode_counter_bytes(D, F) +
                                        stp::decode_scratch_bytes(T, D, F)))
     return STAPLE_EINVAL;
-  if (!ptrs_ok(dtype, {w_gate, w_up, w_down})) return STAPLE_EINVAL;
+  if (!ptrs_ok(dtype, {w_gate, w_down})) return STAPLE_EINVAL;
+  if (!replaces_up(embed) && !ptrs_ok(dtype, {w_up})) return STAPLE_EINVAL;
   if (T > 0 && !ptrs_ok(dtype, {x, z, y})) return STAPLE_EINVAL;
   if ((g_save && !ptrs_ok(dtype, {g_save})) || (h_save && !ptrs_ok(dtype, {h_save})))
     return STAPLE_EINVAL;
@@ -661,7 +675,9 @@ staple_status staple_ffn_bwd(staple_context* ctx, staple_dtype dtype, int32_t T,
   if (!ctx) return STAPLE_EINVAL;
   STP_TRY(check_dims(dtype, T, D, F));
   if (T > 0 && !ptrs_ok(dtype, {dy, x, z, dgh})) return STAPLE_EINVAL;
-  if (dx && !ptrs_ok(dtype, {dx, w_gate, w_up})) return STAPLE_EINVAL;
+  if (dx && !ptrs_ok(dtype, {dx, w_gate})) return STAPLE_EINVAL;
+  if (w_up && !ptrs_ok(dtype, {w_up})) return STAPLE_EINVAL;
+  if (!w_up && dw_up) return STAPLE_EINVAL;   // no up-projection (STEM): no dW_up
   for (const float* p : {dw_gate, dw_up, dw_down})
     if (p && !aligned16(p)) return STAPLE_EINVAL;
   STP_TRY(set_device(ctx));
