@@ -482,7 +482,7 @@ def run_train(stp, ctx, w, steps, warmup, world, local):
                     step(s, staple, stem)
             torch.cuda.synchronize()
             assert stp.staple_get_error(ctx, stream) == 0
-            if mode == "staple":
+            if mode in ("staple", "dense"):
                 stp.staple_trace_enable(ctx, True)
             barrier(world)
             ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -501,11 +501,12 @@ def run_train(stp, ctx, w, steps, warmup, world, local):
             ms = max_over_ranks(ev0.elapsed_time(ev1), world)
             assert stp.staple_get_error(ctx, stream) == 0
             out[mode] = {"ms": ms, "clocks": clk.summary(t0, t1), "sm_reserve": reserve}
-            if mode == "staple":
+            if mode in ("staple", "dense"):
                 out[mode]["kernels"] = kernel_table(stp.staple_trace_read(ctx), steps)
                 stp.staple_trace_enable(ctx, False)
-                out["U"] = int(buf[0].U.item())
-                out["misses"] = int(buf[0].mc.item())
+                if mode == "staple":
+                    out["U"] = int(buf[0].U.item())
+                    out["misses"] = int(buf[0].mc.item())
         # the pages' prefill route for the misses on the last batch: packed on
         # the host, bulk copy, scatter (wall time of the whole call, waited for)
         r = buf[0]
@@ -706,15 +707,16 @@ def run_stack_decode(stp, ctx, w, steps, world, local):
         tables.close()
     step_ms = ms / steps
     wbytes = L * 3 * D * F * 2
+    clocks = clk.summary(c0, c1)
     return {"workload": w.name, "layers": L, "groups_of": G, "T": T, "d_model": D, "d_ff": F,
             "steps": steps, "ms_per_step": step_ms, "tokens_per_s": job_value(T * steps, ms, world),
             "U_last_step": U, "misses_last_step_per_group": misses,
             "weight_bytes_per_step": wbytes, "weight_gbs": wbytes / (step_ms * 1e-3) / 1e9,
             "weight_frac": wbytes / (step_ms * 1e-3) / 1e9 / peaks()["hbm_gbs"],
-            "sm_mhz": clk.summary(c0, c1).get("sm_mhz"),
+            "sm_mhz": clocks.get("sm_mhz"),
             "table_bytes_host": L * V * F * 2, "setup_s": setup_s,
             "graph": "one CUDA graph per step: dedup, 4 group gathers on side streams, 16 layers",
-            "clocks": clk.summary(c0, c1), "kernels_4_traced_steps": kern}
+            "clocks": clocks, "kernels_4_traced_steps": kern}
 
 
 def run_stack_train(stp, ctx, w, steps, world, local):
@@ -787,16 +789,17 @@ def run_stack_train(stp, ctx, w, steps, world, local):
     d2h = L * (U * F * 4 + U * 4 + 4)      # dE rows, ids and U of every layer
     pk = peaks()
     tf = flops / (step_ms * 1e-3) / 1e12
+    clocks = clk.summary(c0, c1)
     return {"workload": w.name, "layers": L, "groups_of": G, "T": T, "d_model": D, "d_ff": F,
             "steps": steps, "ms_per_step": step_ms, "tokens_per_s": job_value(T * steps, ms, world),
             "U_last_step": U, "misses_last_step_per_group": misses,
             "tflops": tf, "tensor_frac_sustained": tf / pk["bf16_tflops_sustained"],
-            "sm_mhz": clk.summary(c0, c1).get("sm_mhz"),
+            "sm_mhz": clocks.get("sm_mhz"),
             "host_link": {"h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                           "h2d_gbs": h2d / (step_ms * 1e-3) / 1e9,
                           "d2h_gbs": d2h / (step_ms * 1e-3) / 1e9},
             "table_bytes_host": L * V * F * 2, "setup_s": setup_s,
-            "clocks": clk.summary(c0, c1), "kernels_one_traced_step": kern}
+            "clocks": clocks, "kernels_one_traced_step": kern}
 
 
 def train_flops(w):
@@ -1042,7 +1045,8 @@ def main():
                 "clocks": tr["staple"]["clocks"],
                 "dense_sm_mhz": tr["dense"]["clocks"].get("sm_mhz"),
             }
-            detail["train_layer"] = {"kernels": kern, "host_link": link, "host_adamw": adamw,
+            detail["train_layer"] = {"kernels": kern, "kernels_dense": tr["dense"].get("kernels"),
+                                     "host_link": link, "host_adamw": adamw,
                                      "bulk_misses": tr.get("bulk_misses"),
                                      "dense_clocks": tr["dense"]["clocks"]}
         except Exception as ex:  # the decode line must still print

@@ -113,6 +113,20 @@ __host__ __device__ inline int owner(int x, int U, int grid) {
   return c;
 }
 
+// Gate/up tiles of block b: [gate_start(b), gate_start(b + 1)).  With no
+// more tiles than blocks, tile b goes to block b, so the blocks with the
+// highest indices, which are the last to get an SM when launches follow one
+// another (each SM takes the next block as the previous launch's block on it
+// exits), make no gate/up tile that every block then waits for; otherwise
+// the tiles are spread evenly.
+__host__ __device__ inline int gate_start(int b, int G, int grid) {
+  return G <= grid ? min(b, G) : range_start(b, G, grid);
+}
+// The block that makes gate/up tile t.
+__host__ __device__ inline int gate_owner(int t, int G, int grid) {
+  return G <= grid ? t : owner(t, G, grid);
+}
+
 // A block finishes its gate/up tiles one after the other, so a tile's ready
 // flag rises later the further it sits in its block's range.  The lateness of
 // down unit x is the largest such position among the tiles that make the z
@@ -122,7 +136,7 @@ __device__ inline int unit_lateness(int x, const Params& p, int grid) {
   const int f_lo = (x % p.ud) * p.sub * BK, f_hi = min(p.F, f_lo + p.sub * BK);
   int late = 0;
   for (int t = f_lo / FT; t <= (f_hi - 1) / FT; ++t)
-    late = max(late, t - range_start(owner(t, p.G, grid), p.G, grid));
+    late = max(late, t - gate_start(gate_owner(t, p.G, grid), p.G, grid));
   return late;
 }
 
@@ -219,7 +233,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int grid = gridDim.x;
   // this block's work: gate/up tiles [t0, t1) (ug units each), then down
   // units [d0, d1); local step i < ngs is gate/up, the rest down
-  const int t0 = range_start(blockIdx.x, p.G, grid), t1 = range_start(blockIdx.x + 1, p.G, grid);
+  const int t0 = gate_start(blockIdx.x, p.G, grid), t1 = gate_start(blockIdx.x + 1, p.G, grid);
   const int d0 = range_start(blockIdx.x, p.Ud, grid), d1 = range_start(blockIdx.x + 1, p.Ud, grid);
   const int ngs = (t1 - t0) * p.ug;
   const int nsteps = ngs + (d1 - d0);
@@ -621,11 +635,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&tempty[buf]);
       // The last epi_bar ordered every thread's z stores before this point
-      // (CTA scope); one thread's gpu-scope fence and release store then
-      // publish all of them (a release is cumulative), and the consumers'
-      // TMA loads of z follow their acquire of the flag.
+      // (CTA scope); one thread's release store then publishes all of them (a
+      // release is cumulative), and the consumers' TMA loads of z follow
+      // their acquire of the flag and an async-proxy fence.
       if (et == 0) {
-        __threadfence();
         fence_async_global();
         st_release(&p.ready[tile], 1u);
       }

@@ -55,7 +55,7 @@ staple_status launch_gather_hits(const void* cache_rows, int64_t row_bytes, cons
 staple_status launch_gather_misses(const void* table_dev, int64_t table_pitch_bytes,
                                    int64_t row_bytes, const int32_t* unique,
                                    const int32_t* miss_list, const int32_t* miss_count,
-                                   void* rows, int num_sms, cudaStream_t st);
+                                   void* rows, int num_sms, bool host_table, cudaStream_t st);
 staple_status launch_cache_fill(const int32_t* hot, int K, int32_t* hkeys, int32_t* hvals,
                                 uint32_t hmask, cudaStream_t st);
 staple_status launch_scatter_misses(const void* staging, int64_t row_bytes,

@@ -344,9 +344,14 @@ staple_status launch_gather_hits(const void* cache_rows, int64_t row_bytes, cons
 staple_status launch_gather_misses(const void* table_dev, int64_t table_pitch_bytes,
                                    int64_t row_bytes, const int32_t* unique,
                                    const int32_t* miss_list, const int32_t* miss_count,
-                                   void* rows, int num_sms, cudaStream_t st) {
+                                   void* rows, int num_sms, bool host_table, cudaStream_t st) {
+  // Over the host link a quarter of the SMs' worth of warps (each with 2 KB
+  // of loads in flight) already keeps far more in flight than the link's
+  // bandwidth-delay product; more only takes thread slots from kernels that
+  // run beside the gather.  A table in HBM gets every SM.
+  const int grid = host_table ? (num_sms + 3) / 4 : num_sms;
   STP_LAUNCH("k4_gather_misses", st,
-             gather_kernel<G_MISSES><<<num_sms, 256, 0, st>>>(
+             gather_kernel<G_MISSES><<<grid, 256, 0, st>>>(
                  static_cast<const uint8_t*>(table_dev), table_pitch_bytes, unique, miss_count,
                  nullptr, miss_list, static_cast<uint8_t*>(rows), row_bytes));
   return cudaGetLastError() == cudaSuccess ? STAPLE_OK : STAPLE_ECUDA;

@@ -408,7 +408,8 @@ staple_status staple_gather_unique_rows(staple_context* ctx, const staple_cache*
     STP_CUDA(cudaStreamWaitEvent(sd, ctx->ev_main, 0));
   }
   STP_TRY(stp::launch_gather_misses(table->dev, row_bytes, row_bytes, unique, miss_list,
-                                    miss_count, rows, ctx->di.num_sms, split ? sd : st));
+                                    miss_count, rows, ctx->di.num_sms,
+                                    table->flags != STAPLE_TABLE_DEVICE, split ? sd : st));
   if (cache && cache->K > 0)
     STP_TRY(stp::launch_gather_hits(cache->rows, row_bytes, U_dev, slot, rows, ctx->di.num_sms, st));
   if (split) {
