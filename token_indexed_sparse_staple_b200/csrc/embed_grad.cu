@@ -20,7 +20,6 @@ namespace stp {
 constexpr int kSegThreads = 256;
 constexpr int kSegVec = 8;                           // features per thread
 constexpr int kSegSlice = kSegThreads * kSegVec;     // features per block
-constexpr int kSegBatch = 8;                         // rows loaded ahead per thread
 
 template <bool BF16>
 __device__ __forceinline__ void load8(const void* base, int64_t off, float* v) {
@@ -78,27 +77,21 @@ __global__ void __launch_bounds__(kSegThreads)
       store8(part + (int64_t(2 * c + side)) * F + f, acc);
     }
   };
-  // kSegBatch rows are loaded before any of them is added, so that many
-  // loads per thread are in flight (each row is a separate 16-byte load of a
-  // different token); the adds then follow in position order, as before.
-  for (int q0 = 0; q0 < n; q0 += kSegBatch) {
-    float v[kSegBatch][kSegVec];
+  // One row at a time, in position order.  Many blocks are resident per SM,
+  // which keeps enough loads in flight; loading several rows ahead per thread
+  // measured slower (more registers, fewer resident blocks).
+  for (int q = 0; q < n; ++q) {
+    const int j = s_seg[q];
+    if (j != cur) {
+      flush(cur);
+      cur = j;
 #pragma unroll
-    for (int b = 0; b < kSegBatch; ++b)
-      if (q0 + b < n) load8<BF16>(dh, int64_t(s_pos[q0 + b]) * ld + f, v[b]);
-#pragma unroll
-    for (int b = 0; b < kSegBatch; ++b) {
-      if (q0 + b >= n) break;
-      const int j = s_seg[q0 + b];
-      if (j != cur) {
-        flush(cur);
-        cur = j;
-#pragma unroll
-        for (int i = 0; i < kSegVec; ++i) acc[i] = 0.0f;
-      }
-#pragma unroll
-      for (int i = 0; i < kSegVec; ++i) acc[i] += v[b][i];
+      for (int i = 0; i < kSegVec; ++i) acc[i] = 0.0f;
     }
+    float v[kSegVec];
+    load8<BF16>(dh, int64_t(s_pos[q]) * ld + f, v);
+#pragma unroll
+    for (int i = 0; i < kSegVec; ++i) acc[i] += v[i];
   }
   if (n > 0) flush(cur);
 }
