@@ -80,6 +80,14 @@ def test_wait_limit_runs_out_then_context_recovers(stp, ctx, T, D):
     stp.staple_ffn_fwd(ctx, stp.STAPLE_BF16, T, D, F, x, emb, wg, wu, wd, z, y, None, None, ws,
                        wsb)
     assert stp.staple_get_error(ctx) == 0
+    torch.cuda.synchronize()
+
+    def f64(t):
+        return t.float().cpu().numpy().astype(np.float64)
+
+    ref = oracle.ffn_forward(f64(x), ids.cpu().numpy(), f64(wg), f64(wu), f64(wd), f64(table))
+    for k, got in (("z", z), ("y", y)):
+        assert_close(f64(got), ref[k], TOL["bf16"], k)
     _small_layer_matches_oracle(stp, ctx, T)
 
 

@@ -267,3 +267,43 @@ def test_split_table_gradient_matches_fused(stp, ctx):
     assert torch.equal(dgh, dgh2)
     u = int(U.item())
     assert torch.equal(got[:u], ref[:u])
+
+
+def test_bf16_decode_workspace_reused_across_calls_and_shapes(stp, ctx):
+    """One workspace, zero-filled once, serves a burst of decode calls of
+    different token counts and inputs issued back to back on one stream (no
+    host synchronisation between them): each call's flags must be told apart
+    from every earlier call's, so every output matches the oracle."""
+    import torch
+    D, F, V = 512, 1024, 3000
+    Ts = [64, 17, 64, 200, 1, 64, 256, 64]
+    g = torch.Generator(device="cuda")
+    g.manual_seed(11)
+
+    def rnd(*shape, std):
+        return (torch.randn(shape, generator=g, device="cuda") * std).to(torch.bfloat16)
+
+    wg, wu, wd = rnd(F, D, std=0.05), rnd(F, D, std=0.05), rnd(D, F, std=0.05)
+    table = rnd(V, F, std=0.05)
+    wsb = max(stp.staple_workspace_bytes(T, D, F) for T in Ts)
+    ws = torch.zeros(wsb, dtype=torch.uint8, device="cuda")
+    calls = []
+    for T in Ts:
+        x = rnd(T, D, std=1.0)
+        ids = torch.randint(0, V, (T,), generator=g, device="cuda", dtype=torch.int32)
+        z = torch.empty((T, F), dtype=torch.bfloat16, device="cuda")
+        y = torch.empty((T, D), dtype=torch.bfloat16, device="cuda")
+        emb = stp.make_embed(stp.STAPLE_EMBED_TABLE, table, F, ids, V)
+        stp.staple_ffn_fwd(ctx, stp.STAPLE_BF16, T, D, F, x, emb, wg, wu, wd, z, y, None, None,
+                           ws, wsb)
+        calls.append((x, ids, z, y))
+    torch.cuda.synchronize()
+    assert stp.staple_get_error(ctx) == 0
+
+    def f64(t):
+        return t.float().cpu().numpy().astype(np.float64)
+
+    for x, ids, z, y in calls:
+        ref = oracle.ffn_forward(f64(x), ids.cpu().numpy(), f64(wg), f64(wu), f64(wd), f64(table))
+        assert_close(f64(z), ref["z"], TOL["bf16"], "z")
+        assert_close(f64(y), ref["y"], TOL["bf16"], "y")

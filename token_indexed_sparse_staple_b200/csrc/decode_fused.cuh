@@ -721,13 +721,15 @@ __global__ void __launch_bounds__(kReduceThreads)
   const int first = owner(tile * r.ud, r.Ud, r.grid);
   const int np = owner((tile + 1) * r.ud - 1, r.Ud, r.grid) - first + 1;
   const float* base = r.part + int64_t(tile) * r.maxp_d * r.N * BM;
-  // thread -> float4 groups g = tid + 256 m: token g / 4, rows 4 (g % 4) .. +3
-  // of the chunk; pieces go in batches whose loads are all in flight at once
+  // thread -> float4 groups g = tid + kReduceThreads m: token g / kGpt, rows
+  // 4 (g % kGpt) .. +3 of the chunk; pieces go in batches whose loads are all
+  // in flight at once
   constexpr int kBatch = 8;
-  const int ngroups = r.T * (kChunkRows / 4);
+  constexpr int kGpt = kChunkRows / 4;   // float4 groups per token
+  const int ngroups = r.T * kGpt;
   for (int g = threadIdx.x; g < ngroups; g += kReduceThreads) {
-    const int t = g >> 2;
-    const int64_t off = int64_t(t) * BM + r0 + (g & 3) * 4;
+    const int t = g / kGpt;
+    const int64_t off = int64_t(t) * BM + r0 + (g % kGpt) * 4;
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
     for (int i0 = 0; i0 < np; i0 += kBatch) {
       float4 v[kBatch];
@@ -739,7 +741,7 @@ __global__ void __launch_bounds__(kReduceThreads)
       for (int i = 0; i < kBatch; ++i)
         if (i0 + i < np) add4(acc, v[i]);
     }
-    const int d = tile * BM + r0 + (g & 3) * 4;
+    const int d = tile * BM + r0 + (g % kGpt) * 4;
     uint16_t* dst = r.y + int64_t(t) * r.D + d;
     if (d + 3 < r.D) {
       uint2 w;
