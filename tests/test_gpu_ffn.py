@@ -79,6 +79,9 @@ SMALL = [
     (129, 64, 64, 50),
     (1, 64, 128, 10),
     (640, 256, 512, 3000),
+    # more tokens than the SMs' worth of 128-row tiles' k blocks: the
+    # weight-gradient GEMMs run 18 k blocks over the tokens, the last ragged
+    (1100, 128, 320, 1000),
 ]
 
 
@@ -144,8 +147,10 @@ def test_bf16_frozen_up_projection(stp, ctx):
     assert np.all(got["dW_up"] == 7.0)   # untouched
 
 
-def test_bf16_deterministic(stp, ctx):
-    w = _bf16_workload(640, 256, 512, 3000)
+@pytest.mark.parametrize("T,D,F,V", [(640, 256, 512, 3000), (1100, 128, 320, 1000)])
+def test_bf16_deterministic(stp, ctx, T, D, F, V):
+    """Two runs give the same bits."""
+    w = _bf16_workload(T, D, F, V)
     inp = syn.make_layer_inputs(w)
     a = run_layer(stp, ctx, inp, w.D, w.F, w.V, embed="table")
     b = run_layer(stp, ctx, inp, w.D, w.F, w.V, embed="table")

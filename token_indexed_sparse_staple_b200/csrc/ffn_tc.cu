@@ -109,8 +109,8 @@ bool out_map(CUtensorMap* m, const void* base, int rows, int cols, int64_t ld) {
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// o: the three output maps of a staged epilogue (EPI_GATEUP: z, g, h;
-// EPI_DZ: dg, dh), NULL for the other epilogues.
+// o: the maps of a staged epilogue (EPI_GATEUP: z, g, h; EPI_DZ: dg, dh, then
+// the inputs g, h), NULL for the other epilogues.
 template <bool A_MN, bool B_MN, int BSRC, int EPI>
 staple_status launch(const char* name, const DeviceInfo& di, const CUtensorMap& a,
                      const CUtensorMap& b0, const CUtensorMap& b1, tc::Params p, cudaStream_t st,
@@ -135,8 +135,10 @@ staple_status launch(const char* name, const DeviceInfo& di, const CUtensorMap& 
   const CUtensorMap& o0 = o ? o[0] : a;
   const CUtensorMap& o1 = o ? o[1] : a;
   const CUtensorMap& o2 = o ? o[2] : a;
+  const CUtensorMap& o3 = (o && EPI == tc::EPI_DZ) ? o[3] : a;
   STP_LAUNCH(name, st,
-             kern<<<grid, tc::kThreads, tc::smem_bytes<EPI>(), st>>>(a, b0, b1, o0, o1, o2, p));
+             kern<<<grid, tc::kThreads, tc::smem_bytes<EPI>(), st>>>(a, b0, b1, o0, o1, o2, o3,
+                                                                      p));
   return cudaGetLastError() == cudaSuccess ? STAPLE_OK : STAPLE_ECUDA;
 }
 
@@ -407,11 +409,12 @@ staple_status tc_dz(const DeviceInfo& di, int T, int D, int F, const void* dy, c
   p.dgh = static_cast<uint16_t*>(dgh);
   p.err = err;
   // dg = columns [0, F) of dgh, dh = [F, 2F): two maps of F columns, row pitch 2F
-  CUtensorMap mo[3];
+  // inputs g and h: [T][F] with row pitch F, the same 32 x 32 box
+  CUtensorMap mo[4];
   if (!out_map(&mo[0], dgh, T, F, 2 * int64_t(F)) ||
-      !out_map(&mo[1], static_cast<uint16_t*>(dgh) + F, T, F, 2 * int64_t(F)))
+      !out_map(&mo[1], static_cast<uint16_t*>(dgh) + F, T, F, 2 * int64_t(F)) ||
+      !out_map(&mo[2], g_save, T, F, F) || !out_map(&mo[3], h_save, T, F, F))
     return STAPLE_ECUDA;
-  mo[2] = mo[1];
   return launch<false, true, tc::B_ONE, tc::EPI_DZ>("k7_dz", di, mdy, mwd, mwd, p, st, mo);
 }
 

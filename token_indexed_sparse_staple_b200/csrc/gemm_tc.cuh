@@ -44,11 +44,13 @@ enum Epi { EPI_BF16 = 0, EPI_F32 = 1, EPI_GATEUP = 2, EPI_DZ = 3, EPI_GATE_E = 4
 // The heavy epilogues stage every 32-row x 32-column output block of a warp
 // in shared memory (64-byte swizzle) and write it with one TMA store: a
 // thread holds one accumulator row, so its own stores would each touch a
-// different row.  2 KB per block: z, g, h for EPI_GATEUP; dg, dh for EPI_DZ.
+// different row.  2 KB per block: z, g, h for EPI_GATEUP; for EPI_DZ two
+// buffers of two blocks, which take the g and h blocks in (by TMA) and then
+// the dg and dh blocks out.
 constexpr int kOutBox = 32 * 32 * 2;
 template <int EPI>
 constexpr int out_blocks() {
-  return (EPI == EPI_GATEUP || EPI == EPI_GATE_E) ? 3 : (EPI == EPI_DZ ? 2 : 0);
+  return (EPI == EPI_GATEUP || EPI == EPI_GATE_E) ? 3 : (EPI == EPI_DZ ? 4 : 0);
 }
 template <int EPI>
 constexpr int smem_bytes() { return kSmemBytes + 4 * out_blocks<EPI>() * kOutBox; }
@@ -143,9 +145,36 @@ __device__ __forceinline__ void write_row_sw64(uint8_t* box, int r, const float*
   }
 }
 
-// Tensor maps the staged output blocks are stored through (box 32 x 32).
+// Row r of a 32 x 32 block in the same layout, as 32 floats.
+__device__ __forceinline__ void read_row_sw64(const uint8_t* box, int r, float* v) {
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const uint4 w = *reinterpret_cast<const uint4*>(box + r * 64 + ((k ^ ((r >> 1) & 3)) << 4));
+    v[8 * k + 0] = bf_lo(w.x);
+    v[8 * k + 1] = bf_hi(w.x);
+    v[8 * k + 2] = bf_lo(w.y);
+    v[8 * k + 3] = bf_hi(w.y);
+    v[8 * k + 4] = bf_lo(w.z);
+    v[8 * k + 5] = bf_hi(w.z);
+    v[8 * k + 6] = bf_lo(w.w);
+    v[8 * k + 7] = bf_hi(w.w);
+  }
+}
+
+// Tensor maps of the staged blocks (box 32 x 32): the outputs (EPI_GATEUP:
+// z, g, h; EPI_DZ: dg, dh) and, for EPI_DZ, the inputs g and h in m[2], m[3].
 struct OutMaps {
-  const CUtensorMap* m[3];
+  const CUtensorMap* m[4];
+};
+
+// EPI_DZ input stream of one epilogue warp: chunk k (counted over all of the
+// warp's tiles) lands in buffer k & 1, on bar[k & 1].
+struct DzIn {
+  uint64_t* bar;          // [2]
+  volatile int* abort;    // the block's abort flag
+  uint32_t next;          // chunks issued so far
+  uint32_t done;          // chunks consumed so far
+  bool ok;                // false once a wait gave up
 };
 
 // Lane 0 waits until the warp's previous block stores have read the staging
@@ -169,9 +198,30 @@ __device__ __forceinline__ void stage_store(int lane, uint8_t* stg, const OutMap
 
 // m = this thread's accumulator row; lane = m % 32; stg = the warp's staging
 // blocks (EPI_GATEUP, EPI_DZ).
+// EPI_DZ: lane 0 issues the g and h blocks of chunk c (columns f, rows from
+// row0) of a tile into the warp's next input buffer.
+__device__ __forceinline__ void dz_load(DzIn& in, uint8_t* stg, const OutMaps& om, int f,
+                                        int row0) {
+  const int b = int(in.next & 1u);
+  uint8_t* buf = stg + b * 2 * kOutBox;
+  mbar_arrive_expect_tx(&in.bar[b], 2 * kOutBox);
+  tma_load_2d(om.m[2], &in.bar[b], buf, f, row0);
+  tma_load_2d(om.m[3], &in.bar[b], buf + kOutBox, f, row0);
+  ++in.next;
+}
+
+// Chunks of 32 features of tile column nb with f < N.
+__device__ __forceinline__ int dz_chunks(const Params& p, int nb) {
+  return min(BN / 32, (p.N - nb * BN + 31) / 32);
+}
+
+
+// nxt_nb / nxt_row0: the warp's next tile (nxt_nb < 0: none), whose first
+// input chunk an EPI_DZ warp requests during this tile's last chunk.
 template <int EPI>
 __device__ __forceinline__ void epilogue_tile(const Params& p, uint32_t tacc, int m, int nb,
-                                              int lane, uint8_t* stg, const OutMaps& om) {
+                                              int lane, uint8_t* stg, const OutMaps& om,
+                                              DzIn& in, int nxt_nb, int nxt_row0) {
   const bool row_ok = m < p.M;
   const int m0w = m - lane;   // the warp's first row
   if constexpr (EPI == EPI_BF16 || EPI == EPI_F32) {
@@ -287,46 +337,50 @@ __device__ __forceinline__ void epilogue_tile(const Params& p, uint32_t tacc, in
       }
     }
   } else {  // EPI_DZ: accumulator = dz for features [nb*256, nb*256 + 256)
-    // g and h of chunk c+1 are loaded while chunk c is computed
-    const int64_t row_off = int64_t(m) * p.ldf + nb * BN;
-    uint4 gw[4] = {}, hw[4] = {};
-    if (row_ok && nb * BN < p.N) {
-      load_raw32(p.g_in + row_off, gw);
-      load_raw32(p.h_in + row_off, hw);
-    }
+    // g and h arrive as 32 x 32 blocks by TMA (rows past M zero-filled) into
+    // two buffers: chunk c+1's (or the next tile's first chunk) is requested
+    // while chunk c is computed.  dg and dh are then staged in the buffer
+    // chunk c came in (each lane reads and writes only its own row) and
+    // stored by TMA.  Before a buffer is loaded again, lane 0 waits until the
+    // stores of the chunk it last held have read it.  (Sending the next
+    // tile's blocks to L2 ahead of time, or the current tile's at its start,
+    // measured slower.)
+    (void)m;
+    const int nch = dz_chunks(p, nb);
 #pragma unroll 1
-    for (int c = 0; c < BN / 32; ++c) {
+    for (int c = 0; c < nch; ++c) {
       const int f = nb * BN + c * 32;
-      uint4 gc[4], hc[4];
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        gc[i] = gw[i];
-        hc[i] = hw[i];
+      const int b = int(in.done & 1u);
+      uint8_t* buf = stg + b * 2 * kOutBox;
+      const bool ok = mbar_wait(&in.bar[b], (in.done >> 1) & 1u, in.abort, p.err, p.wait_ns);
+      if (!__all_sync(0xffffffffu, ok)) {
+        in.ok = false;
+        return;
       }
-      if (row_ok && c + 1 < BN / 32 && f + 32 < p.N) {
-        load_raw32(p.g_in + row_off + (c + 1) * 32, gw);
-        load_raw32(p.h_in + row_off + (c + 1) * 32, hw);
-      }
+      ++in.done;
+      float g[32], h[32];
+      read_row_sw64(buf, lane, g);
+      read_row_sw64(buf + kOutBox, lane, h);
       uint32_t r[32];
       tmem_ld32(tacc + c * 32, r);
       tmem_ld_wait(r);
-      if (f < p.N) {   // the same for the whole warp
-        float g[32], h[32], dg[32], dh[32];
-        unpack32(gc, g);   // zeros for rows past M (staged, never stored)
-        unpack32(hc, h);
+      float dg[32], dh[32];
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const float dz = __uint_as_float(r[i]);
-          const float s = sigmoid_f(g[i]);
-          dh[i] = dz * g[i] * s;
-          dg[i] = dz * h[i] * (s * (1.0f + g[i] * (1.0f - s)));
-        }
-        const bool use[3] = {true, true, false};
-        stage_begin(lane);
-        write_row_sw64(stg, lane, dg);
-        write_row_sw64(stg + kOutBox, lane, dh);
-        stage_store(lane, stg, om, use, f, m0w);
+      for (int i = 0; i < 32; ++i) {
+        const float dz = __uint_as_float(r[i]);
+        const float s = sigmoid_f(g[i]);
+        dh[i] = dz * g[i] * s;
+        dg[i] = dz * h[i] * (s * (1.0f + g[i] * (1.0f - s)));
       }
+      if (lane == 0) {
+        bulk_wait_read0();   // the other buffer's last stores have read it
+        if (c + 1 < nch) dz_load(in, stg, om, f + 32, m0w);
+        else if (nxt_nb >= 0) dz_load(in, stg, om, nxt_nb * BN, nxt_row0);
+      }
+      write_row_sw64(buf, lane, dg);
+      write_row_sw64(buf + kOutBox, lane, dh);
+      const bool use[3] = {true, true, false};
+      stage_store(lane, buf, om, use, f, m0w);
     }
   }
 }
@@ -339,7 +393,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB0,
                 const __grid_constant__ CUtensorMap tmB1, const __grid_constant__ CUtensorMap tmO0,
                 const __grid_constant__ CUtensorMap tmO1, const __grid_constant__ CUtensorMap tmO2,
-                const Params p) {
+                const __grid_constant__ CUtensorMap tmO3, const Params p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align_smem_1024(smem_raw);
   uint8_t* sA = smem;
@@ -350,7 +404,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* tfull = empty + STAGES;
   uint64_t* tempty = tfull + 2;
   uint64_t* dbar = tempty + 2;   // MMA drain before tensor memory is freed
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(dbar + 1);
+  uint64_t* in_bar = dbar + 1;   // [4 warps][2]: EPI_DZ input blocks landed
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(in_bar + 8);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5;
@@ -367,6 +422,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(&tempty[0], 4);
     mbar_init(&tempty[1], 4);
     mbar_init(dbar, 1);
+    if (EPI == EPI_DZ)
+      for (int i = 0; i < 8; ++i) mbar_init(&in_bar[i], 1);
     *abort_flag = 0;
     fence_barrier_init();
     tma_prefetch_desc(&tmA);
@@ -489,23 +546,39 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int q = warp & 3;
     const int row = q * 32 + lane;
     uint8_t* stg = s_out + q * out_blocks<EPI>() * kOutBox;
-    const OutMaps om{{&tmO0, &tmO1, &tmO2}};
+    const OutMaps om{{&tmO0, &tmO1, &tmO2, &tmO3}};
+    DzIn in{in_bar + 2 * q, abort_flag, 0u, 0u, true};
+    if (EPI == EPI_DZ && lane == 0 && int(blockIdx.x) < ntiles) {
+      int mb, nb;
+      tile_coords(blockIdx.x, p, mb, nb);
+      dz_load(in, stg, om, nb * BN, mb * BM + q * 32);   // the first tile's first chunk
+    }
     int iter = 0;
     for (int t = blockIdx.x; t < ntiles; t += gridDim.x, ++iter) {
       const int buf = iter & 1;
       const uint32_t use = uint32_t(iter >> 1);
       int mb, nb;
       tile_coords(t, p, mb, nb);
+      int nxt_nb = -1, nxt_row0 = 0;
+      if (t + int(gridDim.x) < ntiles) {
+        int mb2;
+        tile_coords(t + gridDim.x, p, mb2, nxt_nb);
+        nxt_row0 = mb2 * BM + q * 32;
+      }
       const bool ok = mbar_wait(&tfull[buf], use & 1, abort_flag, p.err, p.wait_ns);
       if (!__all_sync(0xffffffffu, ok)) break;
       tc_fence_after();
       const uint32_t tacc = tmem_base + (uint32_t(q * 32) << 16) + uint32_t(buf * BN);
-      epilogue_tile<EPI>(p, tacc, mb * BM + row, nb, lane, stg, om);
+      epilogue_tile<EPI>(p, tacc, mb * BM + row, nb, lane, stg, om, in, nxt_nb, nxt_row0);
+      if (!in.ok) break;
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&tempty[buf]);
     }
-    // the block's last staged stores must finish before its shared memory goes
+    // input blocks still in flight (after an abort) land before the shared
+    // memory goes away, and so do the block's last staged stores
+    if (EPI == EPI_DZ && lane == 0)
+      for (uint32_t k = in.done; k < in.next; ++k) mbar_drain(&in.bar[k & 1u], (k >> 1) & 1u);
     if (out_blocks<EPI>() > 0 && lane == 0) bulk_wait0();
   }
 
