@@ -168,10 +168,10 @@ class Clocks:
 # to the captured value; otherwise the roofline's traffic is null.
 CAPTURED_TRAFFIC = {
     "k5k6_decode_fused": {
-        "bytes": 104_836_480,   # mean of two launches: 104,961,536 and 104,711,424
+        "bytes": 103_142_400,   # mean of two launches: 104,451,072 and 101,833,728
         "sources": ["token_indexed_sparse_staple_b200/csrc/decode_fused.cuh",
                     "token_indexed_sparse_staple_b200/csrc/common.cuh"],
-        "sha256": "e5a5d0c3a590bbed8fc807c3b305e3b19dfef2477a792dcda8bb92b3dd0c630a",
+        "sha256": "1903f43a08b7a700331893f2d67f201b990186af59acd426e195d86118dd1e7b",
         "profile": "profiles/decode_fused_olmo2_1b_T64.md",
     },
 }
