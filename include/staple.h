@@ -180,8 +180,9 @@ staple_status staple_cache_free(staple_cache* cache);
 /* Bytes of caller-owned device scratch the per-step calls need for T tokens,
  * d_model D, d_ff F (flags reserved, pass 0).  Zero-fill the workspace once
  * (e.g. cudaMemset) before its first use: its first bytes hold the decode
- * kernel's tile counters and ready flags, which every call leaves at zero
- * again (after a call that reported an error, zero-fill it again).  A
+ * kernel's ready flags and the table-gradient reduction's counters, which
+ * every call leaves at zero again (after a call that reported an error,
+ * zero-fill it again).  A
  * workspace of this size (or larger), 256-byte aligned, may be reused by
  * every call with the same D and F and the same or smaller T, one call at a
  * time per workspace. */
@@ -337,7 +338,8 @@ staple_status staple_ffn_fwd(staple_context* ctx, staple_dtype dtype, int32_t T,
  *              sorted_pos from staple_dedup), accumulated in fp32 in
  *              ascending token position, for j < U (U read from U_dev).
  * dE is fp32 [T][F] (capacity T rows; rows >= U untouched).  With
- * dE == NULL only dgh is produced (the dense run). */
+ * dE == NULL only dgh is produced (the dense run).  With dE, T is at most
+ * what one staple_dedup takes (32768; else STAPLE_EUNSUPPORTED). */
 staple_status staple_embed_bwd(staple_context* ctx, staple_dtype dtype, int32_t T, int32_t D,
                                int32_t F, const void* dy, const void* g_save, const void* h_save,
                                const void* w_down, const int32_t* sorted_pos,
@@ -353,8 +355,9 @@ staple_status staple_embed_bwd(staple_context* ctx, staple_dtype dtype, int32_t 
  *   sorted_pos, inverse, seg_off, U_dev   from staple_dedup for the same ids
  *   dE          out, fp32 [>= U][F]; rows >= U untouched
  *   workspace   as for staple_embed_bwd (staple_workspace_bytes(T, D, F)
- *               bytes; its head is left untouched).  Two calls that overlap
- *               on the GPU need two workspaces.
+ *               bytes; of its head only the reduction's counters are used,
+ *               and left at zero).  Two calls that overlap on the GPU need
+ *               two workspaces.  T at most 32768 (STAPLE_EUNSUPPORTED).
  * Same result, bit for bit, as the reduction inside staple_embed_bwd. */
 staple_status staple_embed_grad(staple_context* ctx, staple_dtype dtype, int32_t T, int32_t D,
                                 int32_t F, const void* dh, int64_t ld, const int32_t* sorted_pos,
@@ -450,8 +453,9 @@ staple_status staple_adamw_rows(void* table, int64_t table_pitch, staple_dtype d
  * context of a device looks up the array's device address
  * (cudaGetSymbolAddress) and keeps it for that context; make that first call
  * before any stream capture (and again after a cudaDeviceReset, which starts
- * a new context).  Every call shares the one array, so calls that overlap on
- * the GPU race; nothing in it needs to start at zero.
+ * a new context).  Every call shares the one array (and a small array of
+ * counters beside it, zero at load and left at zero by every call), so calls
+ * that overlap on the GPU race; nothing else needs to start at zero.
  * Returns STAPLE_EUNSUPPORTED, before any pointer is looked at, for a size
  * beyond the array or beyond one dedup: T <= 32768 and
  * 2 * ceil(T / 64) * F * 4 bytes <= 16 MiB (T <= 16384 at F = 8192), and

@@ -36,7 +36,7 @@ def _case(stp, ctx, T, D, F, V, seed):
     dgh = torch.empty((T, 2 * F), dtype=torch.bfloat16, device="cuda")
     dE_ref = torch.full((T, F), float("nan"), dtype=torch.float32, device="cuda")
     wsb = stp.staple_workspace_bytes(T, D, F)
-    ws = torch.empty(wsb, dtype=torch.uint8, device="cuda")
+    ws = torch.zeros(wsb, dtype=torch.uint8, device="cuda")   # zero-filled once, as documented
     stp.staple_embed_bwd(ctx, stp.STAPLE_BF16, T, D, F, dy, gs, hs, wd, sorted_pos, inverse, seg,
                          U, dgh, dE_ref, ws, wsb)
     assert stp.staple_get_error(ctx) == 0

@@ -9,9 +9,13 @@
 // positions; one block per (chunk, 2048-feature slice) sums each segment
 // piece in order with fp32 accumulators.  A segment that lies inside one
 // chunk is written to dE directly; a piece of a segment that crosses a chunk
-// boundary goes to a partial buffer (at most two pieces per chunk), and a
-// second kernel adds the pieces of each crossing segment in chunk order.  No
-// float atomics: the result is deterministic.
+// boundary goes to a partial buffer (at most two pieces per chunk).  Each
+// block then counts its crossing pieces on a per-(segment, slice) counter,
+// and the block that brings the count to the segment's number of pieces adds
+// them in chunk order and writes the row; it also sets the counter back to
+// zero, so the counters are zero again after every call.  No float atomics,
+// and the order of the adds does not depend on which block finishes last:
+// the result is deterministic.
 #include "common.cuh"
 #include "internal.h"
 
@@ -44,13 +48,18 @@ __device__ __forceinline__ void store8(float* dst, const float* v) {
 // Pieces of chunk c: part[(2c + side) * F + f]; side 0 = the chunk's first
 // segment (it started before the chunk), side 1 = its last segment (it
 // continues after the chunk).
+// cnt[c0 * slices + slice]: pieces written so far of the crossing segment
+// that starts in chunk c0 (a chunk starts at most one segment that continues
+// past it).
 template <bool BF16>
 __global__ void __launch_bounds__(kSegThreads)
     seg_reduce_kernel(const void* __restrict__ dh, int64_t ld, const int32_t* __restrict__ sorted_pos,
                       const int32_t* __restrict__ inverse, const int32_t* __restrict__ seg_off,
-                      int T, int F, float* __restrict__ dE, float* __restrict__ part) {
+                      int T, int F, float* __restrict__ dE, float* __restrict__ part,
+                      int32_t* __restrict__ cnt) {
   __shared__ int32_t s_pos[kSegChunk];
   __shared__ int32_t s_seg[kSegChunk];
+  __shared__ int32_t s_fin[2];
   const int c = blockIdx.x;
   const int p0 = c * kSegChunk;
   const int p1 = min(T, p0 + kSegChunk);
@@ -62,7 +71,7 @@ __global__ void __launch_bounds__(kSegThreads)
   }
   __syncthreads();
   const int f = (blockIdx.y * kSegThreads + threadIdx.x) * kSegVec;
-  if (f >= F) return;
+  const bool active = f < F;   // every thread stays for the block barriers below
   const int first_seg = s_seg[0];
   float acc[kSegVec];
 #pragma unroll
@@ -80,7 +89,7 @@ __global__ void __launch_bounds__(kSegThreads)
   // One row at a time, in position order.  Many blocks are resident per SM,
   // which keeps enough loads in flight; loading several rows ahead per thread
   // measured slower (more registers, fewer resident blocks).
-  for (int q = 0; q < n; ++q) {
+  for (int q = 0; q < n && active; ++q) {
     const int j = s_seg[q];
     if (j != cur) {
       flush(cur);
@@ -93,39 +102,52 @@ __global__ void __launch_bounds__(kSegThreads)
 #pragma unroll
     for (int i = 0; i < kSegVec; ++i) acc[i] += v[i];
   }
-  if (n > 0) flush(cur);
-}
-
-// One block per (chunk, slice): the segment that starts in chunk c (the last
-// segment of c) and ends after it is completed here from its pieces.
-__global__ void __launch_bounds__(kSegThreads)
-    seg_fixup_kernel(const int32_t* __restrict__ sorted_pos, const int32_t* __restrict__ inverse,
-                     const int32_t* __restrict__ seg_off, int T, int F, float* __restrict__ dE,
-                     const float* __restrict__ part) {
-  const int c = blockIdx.x;
-  const int p0 = c * kSegChunk;
-  const int plast = min(T, p0 + kSegChunk) - 1;
-  const int j = inverse[sorted_pos[plast]];
-  const int s0 = seg_off[j], s1 = seg_off[j + 1];
-  if (!(s0 >= p0 && s1 > p0 + kSegChunk)) return;
-  const int f = (blockIdx.y * kSegThreads + threadIdx.x) * kSegVec;
-  if (f >= F) return;
-  float acc[kSegVec];
-  {
-    const int side = (s0 == p0) ? 0 : 1;
-    const float4* a = reinterpret_cast<const float4*>(part + int64_t(2 * c + side) * F + f);
-    const float4 x = a[0], y = a[1];
-    acc[0] = x.x; acc[1] = x.y; acc[2] = x.z; acc[3] = x.w;
-    acc[4] = y.x; acc[5] = y.y; acc[6] = y.z; acc[7] = y.w;
+  if (n > 0 && active) flush(cur);
+  __threadfence();   // this thread's pieces before the block's count below
+  // Crossing segments: the chunk's first one (if it started earlier or goes
+  // on past the chunk) and its last one (if it goes on past the chunk).
+  __syncthreads();   // this block's pieces are stored
+  if (threadIdx.x < 2) {
+    int fin = -1;
+    const int j = threadIdx.x == 0 ? first_seg : s_seg[n - 1];
+    const int s0 = seg_off[j], s1 = seg_off[j + 1];
+    const bool crossing = !(s0 >= p0 && s1 <= p1);
+    if (crossing && (threadIdx.x == 0 || j != first_seg)) {
+      const int c0 = s0 / kSegChunk, c1 = (s1 - 1) / kSegChunk;
+      __threadfence();   // the pieces before the count
+      int32_t* k = cnt + int64_t(c0) * gridDim.y + blockIdx.y;
+      if (atomicAdd(k, 1) == c1 - c0) {
+        fin = j;
+        *k = 0;          // every piece has arrived: nobody counts on it again
+      }
+    }
+    s_fin[threadIdx.x] = fin;
   }
-  const int ce = (s1 - 1) / kSegChunk;
-  for (int cc = c + 1; cc <= ce; ++cc) {
-    const float4* a = reinterpret_cast<const float4*>(part + int64_t(2 * cc) * F + f);
-    const float4 x = a[0], y = a[1];
-    acc[0] += x.x; acc[1] += x.y; acc[2] += x.z; acc[3] += x.w;
-    acc[4] += y.x; acc[5] += y.y; acc[6] += y.z; acc[7] += y.w;
+  __syncthreads();
+#pragma unroll 1
+  for (int w = 0; w < 2; ++w) {
+    const int j = s_fin[w];
+    if (j < 0 || !active) continue;
+    __threadfence();     // the other blocks' pieces, seen through the count
+    const int s0 = seg_off[j], s1 = seg_off[j + 1];
+    const int c0 = s0 / kSegChunk, c1 = (s1 - 1) / kSegChunk;
+    // chunk c0's piece is its last segment (side 1) unless the segment starts
+    // the chunk (side 0); every later chunk's piece is its first (side 0)
+    const int side = (s0 == c0 * kSegChunk) ? 0 : 1;
+    float v[kSegVec];
+    const float4* a = reinterpret_cast<const float4*>(part + int64_t(2 * c0 + side) * F + f);
+    float4 x = __ldcg(a), y = __ldcg(a + 1);
+    v[0] = x.x; v[1] = x.y; v[2] = x.z; v[3] = x.w;
+    v[4] = y.x; v[5] = y.y; v[6] = y.z; v[7] = y.w;
+    for (int cc = c0 + 1; cc <= c1; ++cc) {
+      a = reinterpret_cast<const float4*>(part + int64_t(2 * cc) * F + f);
+      x = __ldcg(a);
+      y = __ldcg(a + 1);
+      v[0] += x.x; v[1] += x.y; v[2] += x.z; v[3] += x.w;
+      v[4] += y.x; v[5] += y.y; v[6] += y.z; v[7] += y.w;
+    }
+    store8(dE + int64_t(j) * F + f, v);
   }
-  store8(dE + int64_t(j) * F + f, acc);
 }
 
 size_t seg_reduce_workspace(int T, int F) {
@@ -133,26 +155,28 @@ size_t seg_reduce_workspace(int T, int F) {
   return size_t(chunks) * 2 * size_t(F) * sizeof(float);
 }
 
+size_t seg_counter_bytes(int T, int F) {
+  const int64_t chunks = (int64_t(T) + kSegChunk - 1) / kSegChunk;
+  const int64_t slices = (int64_t(F) + kSegSlice - 1) / kSegSlice;
+  return (size_t(chunks * slices) * sizeof(int32_t) + 255) & ~size_t(255);
+}
+
 staple_status launch_seg_reduce(bool bf16, const void* dh, int64_t ld, const int32_t* sorted_pos,
                                 const int32_t* inverse, const int32_t* seg_off,
                                 const int32_t* U_dev, int T, int F, float* dE, float* part,
-                                cudaStream_t st) {
+                                int32_t* counters, cudaStream_t st) {
   (void)U_dev;
   if (T == 0) return STAPLE_OK;
   const int chunks = (T + kSegChunk - 1) / kSegChunk;
   const dim3 grid(chunks, (F + kSegSlice - 1) / kSegSlice);
   if (bf16)
     STP_LAUNCH("k8_seg_reduce", st,
-               seg_reduce_kernel<true><<<grid, kSegThreads, 0, st>>>(dh, ld, sorted_pos, inverse,
-                                                                     seg_off, T, F, dE, part));
+               seg_reduce_kernel<true><<<grid, kSegThreads, 0, st>>>(
+                   dh, ld, sorted_pos, inverse, seg_off, T, F, dE, part, counters));
   else
     STP_LAUNCH("k8_seg_reduce", st,
-               seg_reduce_kernel<false><<<grid, kSegThreads, 0, st>>>(dh, ld, sorted_pos, inverse,
-                                                                      seg_off, T, F, dE, part));
-  if (chunks > 1)
-    STP_LAUNCH("k8_seg_fixup", st,
-               seg_fixup_kernel<<<grid, kSegThreads, 0, st>>>(sorted_pos, inverse, seg_off, T, F,
-                                                              dE, part));
+               seg_reduce_kernel<false><<<grid, kSegThreads, 0, st>>>(
+                   dh, ld, sorted_pos, inverse, seg_off, T, F, dE, part, counters));
   return cudaGetLastError() == cudaSuccess ? STAPLE_OK : STAPLE_ECUDA;
 }
 

@@ -19,6 +19,8 @@
 // up again there.  Every call shares the one array: calls that overlap on the
 // GPU (on different streams without ordering) race on it.  Nothing in it
 // needs to start at zero: each call writes every partial slot it later reads.
+// A second, small array holds the reduction's crossing-segment counters; it
+// is zero when the image is loaded, and every call leaves it at zero.
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -33,11 +35,17 @@ constexpr size_t kStaticScratchBytes = size_t(16) << 20;  // 16 MiB
 constexpr int kMaxDevices = 64;
 
 static __device__ __align__(256) float g_seg_scratch[kStaticScratchBytes / sizeof(float)];
+// The reduction's crossing-segment counters: zero when the library's device
+// image is loaded, and every call leaves them at zero.  A call the size check
+// admits has ceil(T / 64) * ceil(F / 2048) of them: at most 1024 + 512.
+constexpr int kStaticCounters = 2048;
+static __device__ __align__(256) int32_t g_seg_counters[kStaticCounters];
 
 using CtxGetCurrent = CUresult (*)(CUcontext*);
 
 std::mutex g_addr_mu;
 float* g_addr[kMaxDevices] = {};
+int32_t* g_cnt_addr[kMaxDevices] = {};
 CUcontext g_addr_ctx[kMaxDevices] = {};
 
 // The current CUDA context of the calling thread, through the driver entry
@@ -56,23 +64,28 @@ CUcontext current_context() {
   return c;
 }
 
-// Device address of g_seg_scratch on `device` (which must be current), looked
-// up once per context of that device.
-staple_status scratch_address(int device, float** out) {
+// Device addresses of g_seg_scratch and g_seg_counters on `device` (which
+// must be current), looked up once per context of that device.
+staple_status scratch_address(int device, float** out, int32_t** counters) {
   std::lock_guard<std::mutex> lock(g_addr_mu);
   if (device < 0 || device >= kMaxDevices) return STAPLE_EUNSUPPORTED;
   const CUcontext ctx = current_context();
   if (!g_addr[device] || ctx == nullptr || ctx != g_addr_ctx[device]) {
     void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_seg_scratch) != cudaSuccess || p == nullptr) {
+    void* c = nullptr;
+    if (cudaGetSymbolAddress(&p, g_seg_scratch) != cudaSuccess || p == nullptr ||
+        cudaGetSymbolAddress(&c, g_seg_counters) != cudaSuccess || c == nullptr) {
       cudaGetLastError();
       g_addr[device] = nullptr;
+      g_cnt_addr[device] = nullptr;
       return STAPLE_ECUDA;
     }
     g_addr[device] = static_cast<float*>(p);
+    g_cnt_addr[device] = static_cast<int32_t*>(c);
     g_addr_ctx[device] = ctx;
   }
   *out = g_addr[device];
+  *counters = g_cnt_addr[device];
   return STAPLE_OK;
 }
 
@@ -89,7 +102,8 @@ extern "C" staple_status staple_embed_grad_static(staple_dtype dtype, int32_t T,
   if (T < 0 || F <= 0 || (F % 8) != 0 || ld < F) return STAPLE_EINVAL;
   // Sizes are checked before the pointers: a request the built-in scratch
   // cannot hold (or longer than a dedup can produce) is refused as such.
-  if (T > stp::kMaxDedupT || stp::seg_reduce_workspace(T, F) > kStaticScratchBytes)
+  if (T > stp::kMaxDedupT || stp::seg_reduce_workspace(T, F) > kStaticScratchBytes ||
+      stp::seg_counter_bytes(T, F) > sizeof(int32_t) * kStaticCounters)
     return STAPLE_EUNSUPPORTED;
   if (T == 0) return STAPLE_OK;
   if (!dh || !sorted_pos || !inverse || !seg_off || !dE) return STAPLE_EINVAL;
@@ -98,8 +112,10 @@ extern "C" staple_status staple_embed_grad_static(staple_dtype dtype, int32_t T,
   int device = 0;
   if (cudaGetDevice(&device) != cudaSuccess) return STAPLE_ECUDA;
   float* part = nullptr;
-  const staple_status s = scratch_address(device, &part);
+  int32_t* counters = nullptr;
+  const staple_status s = scratch_address(device, &part, &counters);
   if (s != STAPLE_OK) return s;
   return stp::launch_seg_reduce(dtype == STAPLE_BF16, dh, ld, sorted_pos, inverse, seg_off,
-                                nullptr, T, F, dE, part, reinterpret_cast<cudaStream_t>(stream));
+                                nullptr, T, F, dE, part, counters,
+                                reinterpret_cast<cudaStream_t>(stream));
 }

@@ -202,9 +202,13 @@ DecodePlan plan_decode(int T, int D, int F, int FT, int num_sms) {
 
 }  // namespace
 
-size_t decode_counter_bytes(int D, int F) {
+size_t decode_flag_bytes(int D, int F) {
   const size_t words = size_t((F / 64) + cdiv(D, fused::BM) + 2);
   return (words * sizeof(uint32_t) + 255) & ~size_t(255);
+}
+
+size_t decode_counter_bytes(int D, int F) {
+  return decode_flag_bytes(D, F) + seg_counter_bytes(kMaxDedupT, F);
 }
 
 size_t decode_scratch_bytes(int T, int D, int F) {

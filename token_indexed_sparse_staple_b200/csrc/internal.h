@@ -70,11 +70,16 @@ staple_status launch_copy_rows(const void* table_dev, int64_t table_pitch_bytes,
                                void* dst, int num_sms, cudaStream_t st);
 
 // embed_grad.cu
+// k8 scratch: the partial pieces (seg_reduce_workspace bytes, after the
+// workspace's counter head) and the crossing-segment counters
+// (seg_counter_bytes, in the counter head after the decode flags; zero before
+// the first call and zero again after every call)
 size_t seg_reduce_workspace(int T, int F);
+size_t seg_counter_bytes(int T, int F);
 staple_status launch_seg_reduce(bool bf16, const void* dh, int64_t ld, const int32_t* sorted_pos,
                                 const int32_t* inverse, const int32_t* seg_off,
                                 const int32_t* U_dev, int T, int F, float* dE, float* part,
-                                cudaStream_t st);
+                                int32_t* counters, cudaStream_t st);
 staple_status launch_grad_to_host(const float* dE, const int32_t* unique, const int32_t* U_dev,
                                   int F, int cap, float* host_dE, int32_t* host_unique,
                                   int32_t* host_U, int num_sms, cudaStream_t st);
@@ -96,6 +101,10 @@ constexpr int kMaxDecodeT = 256;
 constexpr int kMaxDecodeGrid = 160;   // blocks of the persistent decode kernel (<= one per SM)
 // Workspace layout: [decode counters, decode_counter_bytes(D, F), zero-filled
 // once by the caller and left at zero by every call][shared scratch].
+// The workspace's counter head: the decode kernel's flags
+// (decode_flag_bytes), then the table-gradient counters for up to kMaxDedupT
+// tokens.  Left untouched by everything else.
+size_t decode_flag_bytes(int D, int F);
 size_t decode_counter_bytes(int D, int F);
 size_t decode_scratch_bytes(int T, int D, int F);
 staple_status tc_decode_fwd(const DeviceInfo& di, int T, int D, int F, const void* x,

@@ -91,6 +91,12 @@ staple_status check_dims(staple_dtype dt, int32_t T, int32_t D, int32_t F) {
   return STAPLE_OK;
 }
 
+// The table-gradient counters in the workspace's counter head.
+int32_t* k8_counters(void* workspace, int D, int F) {
+  return reinterpret_cast<int32_t*>(static_cast<uint8_t*>(workspace) +
+                                    stp::decode_flag_bytes(D, F));
+}
+
 bool ptrs_ok(staple_dtype dt, std::initializer_list<const void*> ps) {
   for (const void* p : ps) {
     if (!p) return false;
@@ -592,6 +598,7 @@ staple_status staple_embed_bwd(staple_context* ctx, staple_dtype dtype, int32_t 
   const size_t head = stp::decode_counter_bytes(D, F);  // left untouched
   if (dE) {
     if (!sorted_pos || !inverse || !seg_off || !U_dev || !aligned16(dE)) return STAPLE_EINVAL;
+    if (T > stp::kMaxDedupT) return STAPLE_EUNSUPPORTED;   // more than one dedup holds
     const size_t need = head + stp::seg_reduce_workspace(T, F);
     if (T > 0 && (!workspace || workspace_bytes < need || !aligned16(workspace)))
       return STAPLE_EINVAL;
@@ -611,7 +618,7 @@ staple_status staple_embed_bwd(staple_context* ctx, staple_dtype dtype, int32_t 
   return stp::launch_seg_reduce(dtype == STAPLE_BF16, dh, 2 * int64_t(F), sorted_pos, inverse,
                                 seg_off, U_dev, T, F, dE,
                                 reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + head),
-                                st);
+                                k8_counters(workspace, D, F), st);
 }
 
 staple_status staple_embed_grad(staple_context* ctx, staple_dtype dtype, int32_t T, int32_t D,
@@ -625,6 +632,7 @@ staple_status staple_embed_grad(staple_context* ctx, staple_dtype dtype, int32_t
   if (!dh || ld < F || !sorted_pos || !inverse || !seg_off || !U_dev || !dE || !aligned16(dE) ||
       !aligned16(dh) || (ld * int64_t(esize(dtype))) % 16)
     return STAPLE_EINVAL;
+  if (T > stp::kMaxDedupT) return STAPLE_EUNSUPPORTED;   // more than one dedup holds
   const size_t head = stp::decode_counter_bytes(D, F);  // left untouched
   if (!workspace || workspace_bytes < head + stp::seg_reduce_workspace(T, F) ||
       !aligned16(workspace))
@@ -634,7 +642,7 @@ staple_status staple_embed_grad(staple_context* ctx, staple_dtype dtype, int32_t
   return stp::launch_seg_reduce(dtype == STAPLE_BF16, dh, ld, sorted_pos, inverse, seg_off, U_dev,
                                 T, F, dE,
                                 reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + head),
-                                cs(stream));
+                                k8_counters(workspace, D, F), cs(stream));
 }
 
 staple_status staple_embed_grad_to_host(staple_context* ctx, int32_t F, int32_t capacity,
