@@ -312,3 +312,62 @@ def test_bf16_decode_workspace_reused_across_calls_and_shapes(stp, ctx):
         ref = oracle.ffn_forward(f64(x), ids.cpu().numpy(), f64(wg), f64(wu), f64(wd), f64(table))
         assert_close(f64(z), ref["z"], TOL["bf16"], "z")
         assert_close(f64(y), ref["y"], TOL["bf16"], "y")
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_empty_batch(stp, ctx, dtype):
+    """T = 0 (a step with no tokens): every call of the layer succeeds, writes
+    no activation, and the weight gradients of the empty batch are zero (a
+    sum over no tokens)."""
+    import torch
+    D, F, V = 256, 512, 100
+    tdt = torch.bfloat16 if dtype == "bf16" else torch.float32
+    sdt = stp.STAPLE_BF16 if dtype == "bf16" else stp.STAPLE_F32
+    g = torch.Generator(device="cuda")
+    g.manual_seed(21)
+
+    def rnd(*shape):
+        return (torch.randn(shape, generator=g, device="cuda") * 0.05).to(tdt)
+
+    wg, wu, wd, table = rnd(F, D), rnd(F, D), rnd(D, F), rnd(V, F)
+    ids = torch.zeros(1, dtype=torch.int32, device="cuda")
+    emb = stp.make_embed(stp.STAPLE_EMBED_TABLE, table, F, ids, V)
+    x, dy, dx = (torch.full((1, D), 7.0, dtype=tdt, device="cuda") for _ in range(3))
+    z, gs, hs = (torch.full((1, F), 7.0, dtype=tdt, device="cuda") for _ in range(3))
+    y = torch.full((1, D), 7.0, dtype=tdt, device="cuda")
+    dgh = torch.full((1, 2 * F), 7.0, dtype=tdt, device="cuda")
+    dE = torch.full((1, F), 7.0, dtype=torch.float32, device="cuda")
+    i32 = dict(dtype=torch.int32, device="cuda")
+    sorted_pos, inverse, seg, U = (torch.zeros(2, **i32) for _ in range(4))
+    dwg, dwu, dwd = (torch.full(s, 3.0, dtype=torch.float32, device="cuda")
+                     for s in ((F, D), (F, D), (D, F)))
+    wsb = stp.staple_workspace_bytes(0, D, F)
+    ws = torch.zeros(max(wsb, 256), dtype=torch.uint8, device="cuda")
+    stp.staple_ffn_fwd(ctx, sdt, 0, D, F, x, emb, wg, wu, wd, z, y, gs, hs, ws, wsb)
+    stp.staple_embed_bwd(ctx, sdt, 0, D, F, dy, gs, hs, wd, sorted_pos, inverse, seg, U, dgh, dE,
+                         ws, wsb)
+    stp.staple_ffn_bwd(ctx, sdt, 0, D, F, dy, x, z, dgh, wg, wu, dx, dwg, dwu, dwd, ws, wsb)
+    torch.cuda.synchronize()
+    assert stp.staple_get_error(ctx) == 0
+    for t in (y, z, gs, hs, dgh, dx):
+        assert bool((t.float() == 7.0).all())
+    assert bool((dE == 7.0).all())
+    for t in (dwg, dwu, dwd):
+        assert bool((t == 0.0).all())
+
+
+def test_table_gradient_refuses_more_tokens_than_one_dedup(stp, ctx):
+    """The reduction's counters cover the 32768 tokens one staple_dedup takes;
+    a longer batch with dE requested is refused before anything runs (the
+    addresses below are never touched)."""
+    fake = 1 << 12
+    wsb = stp.staple_workspace_bytes(32769, 64, 64)
+    for call in (
+            lambda: stp.staple_embed_bwd(ctx, stp.STAPLE_BF16, 32769, 64, 64, fake, fake, fake, fake,
+                                         fake, fake, fake, fake, fake, fake, fake, wsb),
+            lambda: stp.staple_embed_grad(ctx, stp.STAPLE_BF16, 32769, 64, 64, fake, 64, fake, fake,
+                                          fake, fake, fake, fake, wsb)):
+        with pytest.raises(stp.StapleError) as ex:
+            call()
+        assert ex.value.status == stp.STAPLE_EUNSUPPORTED
+    assert stp.staple_get_error(ctx) == 0

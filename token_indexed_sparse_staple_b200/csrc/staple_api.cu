@@ -566,9 +566,10 @@ staple_status staple_ffn_fwd(staple_context* ctx, staple_dtype dtype, int32_t T,
   STP_TRY(set_device(ctx));
   stp::TraceScope trace_scope(ctx->tracer);
   if (decode) {
-    // the decode kernel refuses (before launching anything) a shape whose
-    // down tiles its clusters cannot own, or a device that cannot hold its
-    // grid at once; the tiled kernels then compute the same layer
+    // the decode kernel refuses (before launching anything) a STEM layer
+    // whose d_ff is not a multiple of its 128-feature gate tiles, or a device
+    // that cannot hold its whole grid at once; the tiled kernels then compute
+    // the same layer
     const staple_status s = stp::tc_decode_fwd(ctx->di, T, D, F, x, embed, w_gate, w_up, w_down, z,
                                                y, g_save, h_save, workspace, ctx->d_err, cs(stream));
     if (s != STAPLE_EUNSUPPORTED) return s;
