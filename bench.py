@@ -467,46 +467,94 @@ def run_train(stp, ctx, w, steps, warmup, world, local):
                            None if stem else wu, dx, dwg, None if stem else dwu, dwd, stream=stream)
 
     out = {}
+
+    def timed(staple, stem, s0, n):
+        """n consecutive steps from step s0, CUDA events on the layer's stream
+        around them.  The first step's retrieval is done before the events (as
+        for a pipeline already running), every later one, up to the prefetch of
+        the step after the last, falls inside; nothing of another run is still
+        on the GPU when the first event is recorded."""
+        ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            if staple:
+                prefetch(s0)
+        torch.cuda.synchronize()
+        with torch.cuda.stream(stream):
+            ev0.record(stream)
+            for s in range(s0, s0 + n):
+                step(s, staple, stem)
+            if staple:
+                stream.wait_event(buf[(s0 + n) % 2].ready)
+            ev1.record(stream)
+        return ev0, ev1
+
+    def warm(staple, stem, s0):
+        nw = max(warmup, 3)
+        with torch.cuda.stream(stream):
+            if staple:
+                prefetch(s0)
+            for s in range(s0, s0 + nw):
+                step(s, staple, stem)
+            if staple:
+                stream.wait_event(buf[(s0 + nw) % 2].ready)
+        torch.cuda.synchronize()
+        assert stp.staple_get_error(ctx, stream) == 0
+
     try:
-        # (name, E path on, STEM, SMs the GEMMs leave to the prefetch kernels)
-        for mode, staple, stem, reserve in (("staple_r0", True, False, 0),
-                                            ("staple", True, False, 1),
-                                            ("dense", False, False, 0),
-                                            ("stem", True, True, 1)):
-            stp.staple_set_sm_reserve(ctx, reserve)
-            nw = max(warmup, 3)
-            with torch.cuda.stream(stream):
-                if staple:
-                    prefetch(0)
-                for s in range(nw):
-                    step(s, staple, stem)
+        # The E-path and dense runs alternate in rounds of steps, so that both
+        # see the same clocks under the power cap; all of these steps run
+        # untraced.  (name, E path on, STEM, SMs the GEMMs leave to the
+        # prefetch kernels)
+        rounds = 5 if steps >= 5 else 1
+        per = [steps // rounds + (1 if r < steps % rounds else 0) for r in range(rounds)]
+        stp.staple_set_sm_reserve(ctx, 0)
+        warm(True, False, 0)
+        warm(False, False, 0)
+        barrier(world)
+        evs = {"staple_r0": [], "dense": []}
+        s_next = 16
+        with Clocks(local) as clk:
             torch.cuda.synchronize()
-            assert stp.staple_get_error(ctx, stream) == 0
-            if mode in ("staple", "dense"):
-                stp.staple_trace_enable(ctx, True)
+            t0 = time.time()
+            for r in range(rounds):
+                for mode, staple in (("staple_r0", True), ("dense", False)):
+                    evs[mode].append(timed(staple, False, s_next, per[r]))
+                    s_next += per[r] + 2
+            torch.cuda.synchronize()
+            t1 = time.time()
+        assert stp.staple_get_error(ctx, stream) == 0
+        clocks = clk.summary(t0, t1)
+        for mode in ("staple_r0", "dense"):
+            ms = sum(e0.elapsed_time(e1) for e0, e1 in evs[mode])
+            out[mode] = {"ms": max_over_ranks(ms, world), "clocks": clocks, "sm_reserve": 0}
+        # one reserved SM, and STEM: timed on their own
+        for mode, stem, reserve in (("staple", False, 1), ("stem", True, 1)):
+            stp.staple_set_sm_reserve(ctx, reserve)
+            warm(True, stem, s_next)
+            s_next += 16
             barrier(world)
-            ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             with Clocks(local) as clk:
                 torch.cuda.synchronize()
                 t0 = time.time()
-                with torch.cuda.stream(stream):
-                    ev0.record(stream)
-                    for s in range(nw, nw + steps):
-                        step(s, staple, stem)
-                    if staple:   # the last prefetch ends inside the timed region too
-                        stream.wait_event(buf[(nw + steps) % 2].ready)
-                    ev1.record(stream)
+                e0, e1 = timed(True, stem, s_next, steps)
                 torch.cuda.synchronize()
                 t1 = time.time()
-            ms = max_over_ranks(ev0.elapsed_time(ev1), world)
+            s_next += steps + 2
             assert stp.staple_get_error(ctx, stream) == 0
-            out[mode] = {"ms": ms, "clocks": clk.summary(t0, t1), "sm_reserve": reserve}
-            if mode in ("staple", "dense"):
-                out[mode]["kernels"] = kernel_table(stp.staple_trace_read(ctx), steps)
-                stp.staple_trace_enable(ctx, False)
-                if mode == "staple":
-                    out["U"] = int(buf[0].U.item())
-                    out["misses"] = int(buf[0].mc.item())
+            out[mode] = {"ms": max_over_ranks(e0.elapsed_time(e1), world),
+                         "clocks": clk.summary(t0, t1), "sm_reserve": reserve}
+        # the kernel tables: a separate traced run of a few steps per mode
+        stp.staple_set_sm_reserve(ctx, 0)
+        nt = min(steps, 10)
+        for mode, staple in (("staple_r0", True), ("dense", False)):
+            stp.staple_trace_enable(ctx, True)
+            timed(staple, False, s_next, nt)
+            torch.cuda.synchronize()
+            out[mode]["kernels"] = kernel_table(stp.staple_trace_read(ctx), nt)
+            stp.staple_trace_enable(ctx, False)
+            s_next += nt + 2
+        out["U"] = int(buf[0].U.item())
+        out["misses"] = int(buf[0].mc.item())
         # the pages' prefill route for the misses on the last batch: packed on
         # the host, bulk copy, scatter (wall time of the whole call, waited for)
         r = buf[0]
@@ -1005,12 +1053,11 @@ def main():
         try:
             wt = syn.WORKLOADS["olmo2-1b-train-layer"]
             tr = run_train(stp, ctx, wt, args.train_steps, 5, world, local)
-            # the E-path run at its better SM reserve (0: the GEMMs use every
-            # SM; 1: one SM is left to the prefetched retrieval kernels)
-            best = min(("staple", "staple_r0"), key=lambda m: tr[m]["ms"])
-            st_ms = tr[best]["ms"] / args.train_steps
+            # the E-path and dense runs timed in alternating rounds (the same
+            # clocks), untraced; the kernel tables come from a separate traced run
+            st_ms = tr["staple_r0"]["ms"] / args.train_steps
             de_ms = tr["dense"]["ms"] / args.train_steps
-            kern = tr["staple"]["kernels"]
+            kern = tr["staple_r0"]["kernels"]
             top = max(kern.items(), key=lambda kv: kv[1]["total_ms"])
             gemm_flops = {"k5_gateup": 4, "k6_down": 2, "k7_dz": 2, "k9_dx": 4, "k10_dw_gate_up": 4,
                           "k10_dw_down": 2}
@@ -1029,7 +1076,8 @@ def main():
                 "workload": wt.name, "tokens_per_s": r3(job_value(wt.T, st_ms, world)),
                 "ms_per_step": r3(st_ms), "dense_ms_per_step": r3(de_ms),
                 "e_path_overhead": r3((st_ms - de_ms) / de_ms), "steps": args.train_steps,
-                "sm_reserve": tr[best]["sm_reserve"],
+                "sm_reserve": 0,
+                "timing": "E path and dense run alternated in rounds of steps, untraced",
                 "ms_by_sm_reserve": {str(tr[m]["sm_reserve"]): r3(tr[m]["ms"] / args.train_steps)
                                      for m in ("staple_r0", "staple")},
                 "stem_ms_per_step": r3(tr["stem"]["ms"] / args.train_steps),
@@ -1042,8 +1090,7 @@ def main():
                              "peak": pk["bf16_tflops_sustained"], "unit": "TFLOP/s",
                              "frac": None if tf is None else r3(tf / pk["bf16_tflops_sustained"]),
                              "peak_source": pk["source"] + " (cuBLAS bf16, sustained)"},
-                "clocks": tr["staple"]["clocks"],
-                "dense_sm_mhz": tr["dense"]["clocks"].get("sm_mhz"),
+                "clocks": tr["staple_r0"]["clocks"],
             }
             detail["train_layer"] = {"kernels": kern, "kernels_dense": tr["dense"].get("kernels"),
                                      "host_link": link, "host_adamw": adamw,
