@@ -43,15 +43,17 @@ def _small_layer_matches_oracle(stp, ctx, T):
         assert_close(got[k], ref[k], TOL["bf16"], k)
 
 
-@pytest.mark.parametrize("T,D", [(64, 8192), (384, 32768)])
-def test_wait_limit_runs_out_then_context_recovers(stp, ctx, T, D):
+@pytest.mark.parametrize("T,D,F", [(64, 8192, 256), (64, 4096, 512), (384, 32768, 256)])
+def test_wait_limit_runs_out_then_context_recovers(stp, ctx, T, D, F):
     """A long d_model makes every gate/up tile stream megabytes of weights
     through one SM before its accumulator is ready: 2 MB per tile in the decode
-    kernel (T = 64, d_model 8192), 24 MB in the tiled GEMM (T = 384, d_model
-    32768), tens of microseconds at least, so a 10 us limit runs out in the
-    first wait for an accumulator."""
+    kernel's two-launch path (T = 64, d_model 8192: 64 down tiles, more than
+    the clusters the device holds at once), 1 MB in its cluster path (d_model
+    4096, d_ff 512), 24 MB in the tiled GEMM (T = 384, d_model 32768), tens of
+    microseconds at least, so a 10 us limit runs out in the first wait for an
+    accumulator."""
     import torch
-    F, V = 256, 100
+    V = 100
     g = torch.Generator(device="cuda")
     g.manual_seed(5)
 

@@ -213,11 +213,16 @@ def test_bf16_decode_saves_g_and_h(stp, ctx):
     compare(got, oracle_layer(inp), TOL["bf16"], FWD + SAVED + BWD)
 
 
-@pytest.mark.parametrize("D,F", [(2048, 1024), (1024, 8192), (4096, 11008)])
+@pytest.mark.parametrize("D,F", [(2048, 1024), (1024, 8192), (4096, 11008), (4096, 1024),
+                                 (128, 192), (4352, 1024)])
 def test_bf16_decode_split_k_shapes(stp, ctx, D, F):
-    """Down tiles whose K is split over a few to many blocks, and the 7B shape
-    (d_ff 11008 = 172 gate/up tiles over at most 148 blocks, so some blocks
-    make two)."""
+    """Both decode paths.  Two launches (the split-k sum in its own kernel):
+    down tiles whose K is split over a few to many blocks (d_model 2048 and
+    1024), d_ff 192 (fewer k units per down tile than a cluster has blocks),
+    d_model 4352 (more down tiles, 34, than clusters fit on the device at
+    once).  One launch in clusters (one cluster per down tile, the sum in
+    shared memory): d_model 4096 with d_ff 1024, and the 7B shape (d_ff
+    11008 = 172 gate/up tiles over 128 blocks, so some blocks make two)."""
     w = _bf16_workload(64, D, F, 2000)
     inp = syn.make_layer_inputs(w, with_dy=False)
     got = run_layer(stp, ctx, inp, w.D, w.F, w.V, embed="table", training=False)
@@ -274,13 +279,16 @@ def test_split_table_gradient_matches_fused(stp, ctx):
     assert torch.equal(got[:u], ref[:u])
 
 
-def test_bf16_decode_workspace_reused_across_calls_and_shapes(stp, ctx):
+@pytest.mark.parametrize("D,F", [(512, 1024), (4096, 512)])
+def test_bf16_decode_workspace_reused_across_calls_and_shapes(stp, ctx, D, F):
     """One workspace, zero-filled once, serves a burst of decode calls of
     different token counts and inputs issued back to back on one stream (no
     host synchronisation between them): each call's flags must be told apart
-    from every earlier call's, so every output matches the oracle."""
+    from every earlier call's, so every output matches the oracle.  d_model
+    512 takes the two-launch path (its sum kernel clears the flags), 4096 the
+    cluster path (the last block past its poll clears them)."""
     import torch
-    D, F, V = 512, 1024, 3000
+    V = 3000
     Ts = [64, 17, 64, 200, 1, 64, 256, 64]
     g = torch.Generator(device="cuda")
     g.manual_seed(11)

@@ -57,7 +57,7 @@ def test_stem_f32(stp, ctx, embed):
 
 
 @pytest.mark.parametrize("T,D,F,V", [(300, 128, 320, 1000), (640, 256, 512, 3000), (64, 256, 576, 4000),
-                                     (1, 64, 128, 10)])
+                                     (1, 64, 128, 10), (64, 4096, 1024, 2000)])
 def test_stem_bf16(stp, ctx, T, D, F, V):
     inp = syn.make_layer_inputs(_w(T, D, F, V))
     got = run_layer(stp, ctx, inp, D, F, V, embed="table", stem=True)

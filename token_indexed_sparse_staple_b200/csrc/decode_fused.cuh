@@ -1,7 +1,9 @@
-// The STAPLE layer at decode sizes (T <= 256 tokens) in two launches: one
-// persistent tcgen05 kernel for gate/up (with the fused E-row add and SiLU
-// gating) and the down projection's split-k pieces, then a small kernel that
-// sums the pieces.
+// The STAPLE layer at decode sizes (T <= 256 tokens): one persistent tcgen05
+// kernel for gate/up (with the fused E-row add and SiLU gating) and the down
+// projection's split-k pieces.  The pieces are summed either by a small
+// kernel launched right behind it (two-launch path) or, when the layer has
+// enough down tiles, inside the same launch by clusters of blocks through
+// distributed shared memory (cluster path).
 //
 // With a handful of tokens the layer streams its weights once per step and
 // is bound by HBM bandwidth, so the kernel is organised around that stream:
@@ -33,11 +35,21 @@
 //    loads do not wait.  Each block's piece of a tile leaves an fp32 partial
 //    [N][128] in the workspace (L2-resident; a warp writes 128 contiguous
 //    bytes per token), and the block is done.
-//  * The split-k sums run in decode_reduce_kernel, launched right behind as
-//    a programmatic dependent (see there), which also clears the ready flags.
+//  * Two-launch path: the split-k sums run in decode_reduce_kernel, launched
+//    right behind as a programmatic dependent (see there), which also clears
+//    the ready flags.
+//  * Cluster path (kClu): the grid is one cluster of kCluster blocks per down
+//    tile, and the tile's units are split over the cluster's blocks.  At the
+//    end each block pushes its accumulator rows into the shared memory of the
+//    block that sums them (block r of the cluster sums rows 32r .. 32r+31),
+//    and after a cluster barrier each block adds the cluster's pieces in
+//    block order and writes its rows of y.  No partial leaves the SMs, and
+//    the next call's activations are ready as soon as this launch completes.
+//    The last block to finish polling clears the ready flags.
 //  * Every block finishes its gate/up tiles before it needs anybody's z, so
-//    all waits end while all blocks are resident (grid <= SMs, one block per
-//    SM, checked by the launcher).  The ready flags live in the first bytes
+//    all waits end while all blocks are resident (one block per SM; the
+//    launcher checks the grid against the blocks, or clusters, the device
+//    holds at once).  The ready flags live in the first bytes
 //    of the workspace and are zero again after every call, so a zero-filled
 //    workspace stays valid across calls and graph replays.
 //
@@ -66,6 +78,8 @@ constexpr int kMaxN = 256;
 constexpr int kStagesB = 3;
 constexpr int kChunkRows = 16;        // rows of a down tile per reduction chunk
 constexpr int kXStride = 17;          // fp32 words per row of the g/u exchange chunk
+constexpr int kCluster = 4;           // blocks per cluster (cluster path)
+constexpr int kRowsPer = BM / kCluster;  // rows of a down tile each cluster block sums
 // shared memory after the rings: barriers + flags (512 B), token ids,
 // g/u exchange chunk [128][17] fp32; then the E tile [N][features per tile] bf16
 constexpr int kTailFixed = 512 + kMaxN * 4 + 128 * kXStride * 4;
@@ -96,10 +110,12 @@ struct Params {
   int64_t e_rows;
   int32_t e_mode;
   // workspace
-  uint32_t* ready;     // [G] gate/up tile finished (reset by the split-k sum kernel)
-  float* part;         // [Dt * maxp_d][N][128] fp32 partial sums, summed by the next kernel
+  uint32_t* ready;     // [G] gate/up tile finished (reset after every call)
+  float* part;         // two-launch path: [Dt * maxp_d][N][128] fp32 partial sums, summed
+                       // by the next kernel
   int32_t* err;
   uint64_t wait_ns;    // bound of every wait and flag spin (STAPLE_ETIMEOUT past it)
+  uint32_t* fin;       // cluster path: blocks whose z poll is over; the last one clears `ready`
 };
 
 __host__ __device__ inline int range_start(int c, int U, int grid) {
@@ -145,6 +161,33 @@ __device__ __forceinline__ void grid_dep_launch() {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 __device__ __forceinline__ void epi_bar() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ uint32_t cluster_id() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%clusterid.x;" : "=r"(r));
+  return r;
+}
+// Every thread of every block of the cluster; stores before it (shared
+// memory of any block of the cluster included) are seen after it.
+__device__ __forceinline__ void cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" :::
+                   "memory");
+}
+// The address of this block's shared-memory word `a` in block `rank` of the cluster.
+__device__ __forceinline__ uint32_t map_peer(uint32_t a, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(rank));
+  return r;
+}
+__device__ __forceinline__ void st_peer4(uint32_t a, uint32_t x, uint32_t y, uint32_t z, uint32_t w) {
+  asm volatile("st.shared::cluster.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(x), "r"(y), "r"(z),
+               "r"(w)
+               : "memory");
+}
 __device__ __forceinline__ uint32_t ld_acquire(const uint32_t* a) {
   uint32_t v;
   asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(a) : "memory");
@@ -152,6 +195,11 @@ __device__ __forceinline__ uint32_t ld_acquire(const uint32_t* a) {
 }
 __device__ __forceinline__ void st_release(uint32_t* a, uint32_t v) {
   asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(a), "r"(v) : "memory");
+}
+__device__ __forceinline__ uint32_t atom_add_acq_rel(uint32_t* a, uint32_t v) {
+  uint32_t old;
+  asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], %2;" : "=r"(old) : "l"(a), "r"(v) : "memory");
+  return old;
 }
 __device__ __forceinline__ void fence_async_global() {
   asm volatile("fence.proxy.async.global;" ::: "memory");
@@ -185,7 +233,9 @@ __device__ __forceinline__ bool spin_until(const uint32_t* a, uint32_t want, vol
 // kOrder false that code is compiled out, which keeps the kernel body small
 // (the gate/up epilogue runs while the memory queues are full, where extra
 // code shows up as instruction-fetch stalls).
-template <bool kOrder, bool kStem>
+// kClu: the cluster path (launched in clusters of kCluster blocks, see the
+// end of the kernel): the split-k sum is done inside the launch.
+template <bool kOrder, bool kStem, bool kClu>
 __global__ void __launch_bounds__(kThreads, 1)
     decode_fused_kernel(const __grid_constant__ CUtensorMap tm_wg,
                         const __grid_constant__ CUtensorMap tm_wu,
@@ -234,7 +284,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   // this block's work: gate/up tiles [t0, t1) (ug units each), then down
   // units [d0, d1); local step i < ngs is gate/up, the rest down
   const int t0 = gate_start(blockIdx.x, p.G, grid), t1 = gate_start(blockIdx.x + 1, p.G, grid);
-  const int d0 = range_start(blockIdx.x, p.Ud, grid), d1 = range_start(blockIdx.x + 1, p.Ud, grid);
+  // Cluster path: cluster c takes down tile c, its blocks split the tile's
+  // units (one piece per block).
+  const uint32_t crank = kClu ? cluster_rank() : 0u;
+  const int ctile = kClu ? int(cluster_id()) : 0;
+  const int d0 = kClu ? ctile * p.ud + range_start(int(crank), p.ud, kCluster)
+                      : range_start(blockIdx.x, p.Ud, grid);
+  const int d1 = kClu ? ctile * p.ud + range_start(int(crank) + 1, p.ud, kCluster)
+                      : range_start(blockIdx.x + 1, p.Ud, grid);
   const int ngs = (t1 - t0) * p.ug;
   const int nsteps = ngs + (d1 - d0);
   const int nd = d1 - d0;
@@ -248,6 +305,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t slot_cols = uint32_t(p.sub) * (BK / 2);
   const int nslots = p.stage_tmem ? int((512 - 2 * ncols) / slot_cols) : 0;
   const uint32_t tmem_cols = nslots > 0 ? 512 : 2 * ncols;
+
+  // cluster path: the accumulator that holds the block's down piece, once
+  // the epilogue has seen it complete (-1: none, or the block gave up)
+  int acc_buf = -1;
 
   // the unit of the block's k-th down step
   auto unit = [&](int k) { return d0 + (reorder ? int(s_order[k]) : k); };
@@ -426,6 +487,18 @@ __global__ void __launch_bounds__(kThreads, 1)
           ok = poll(true);
           if (lane == 0 && ok) issue(false);
         }
+      }
+    }
+    if (kClu) {
+      // The block's last look at the ready flags is behind it (every lane's
+      // poll, ordered by the warp barrier and the release).  Every tile is
+      // polled by some block after it was published, so once every block has
+      // counted itself here the last one clears the flags for the next call
+      // (which reads them only after this launch completes).
+      __syncwarp();
+      if (lane == 0 && atom_add_acq_rel(p.fin, 1u) == uint32_t(grid - 1)) {
+        for (int t = 0; t < p.G; ++t) p.ready[t] = 0u;
+        *p.fin = 0u;
       }
     }
     if (lane == 0) drain_ring(fullB, SB, s, ph, issued);
@@ -643,11 +716,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         st_release(&p.ready[tile], 1u);
       }
     }
-    // ---- phase 2: down pieces -> fp32 partial slots
+    // ---- phase 2: down pieces -> fp32 partial slots (cluster path: the one
+    // piece stays in tensor memory for the cluster's sum at the end)
     for (int x = d0; x < d1 && alive; ++piece) {
       const int tile = x / p.ud;
       const int x_end = min(d1, (tile + 1) * p.ud);
-      const int idx = blockIdx.x - owner(tile * p.ud, p.Ud, grid);
       x = x_end;
       const int buf = piece & 1;
       const bool ok = mbar_wait(&tfull[buf], (piece >> 1) & 1, abort_flag, p.err, p.wait_ns);
@@ -658,6 +731,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         break;
       }
       tc_fence_after();
+      if (kClu) {
+        acc_buf = buf;
+        break;
+      }
+      const int idx = blockIdx.x - owner(tile * p.ud, p.Ud, grid);
       float* mine = p.part + int64_t(tile * p.maxp_d + idx) * p.N * BM;
       const uint32_t tacc = tmem_base + (uint32_t(q * 32) << 16) + uint32_t(buf) * ncols;
       for (int c = 0; c < p.N; c += 32) {
@@ -678,6 +756,58 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  if (kClu) {
+    // ---- the split-k sum of the cluster path.  (1) After this barrier every
+    // block of the cluster is done with its rings (copies landed, MMAs
+    // drained), and the weight ring takes the pushed accumulator rows:
+    // recv[source block][kRowsPer][N + 4] fp32.  Epilogue warp q holds rows
+    // 32q .. 32q+31 of the block's piece, which block q of the cluster sums.
+    static_assert(kRowsPer == 32, "one epilogue warp's rows per cluster block");
+    cluster_sync();
+    float* recv = reinterpret_cast<float*>(sA);
+    const int rs = p.N + 4;   // padded row: the pushes of a warp's 32 rows spread over the banks
+    if (warp >= 3 && acc_buf >= 0) {
+      const int q = warp & 3;
+      const uint32_t tacc = tmem_base + (uint32_t(q * 32) << 16) + uint32_t(acc_buf) * ncols;
+      const uint32_t dst =
+          map_peer(smem_u32(recv + (int(crank) * kRowsPer + lane) * rs), uint32_t(q));
+      for (int c = 0; c < p.N; c += 32) {
+        uint32_t r[32];
+        tmem_ld32(tacc + c, r);
+        tmem_ld_wait(r);
+        const int cn = min(32, p.N - c);
+#pragma unroll
+        for (int j = 0; j < 32; j += 4)
+          if (j < cn) st_peer4(dst + uint32_t(c + j) * 4u, r[j], r[j + 1], r[j + 2], r[j + 3]);
+      }
+    }
+    tc_fence_before();
+    cluster_sync();   // (2) every push has landed
+    tc_fence_after();
+    if (warp >= 3) {
+      // This block's slice: rows row0 .. row0+31 of y, for every token.  A
+      // thread takes 8 rows of one token (lanes: consecutive tokens) and adds
+      // the cluster's pieces in block order.
+      const int et = threadIdx.x - 96;
+      const int row0 = ctile * BM + int(crank) * kRowsPer;
+      const int nitems = (kRowsPer / 8) * p.N;
+      for (int it = et; it < nitems; it += 128) {
+        const int t = it % p.N, rg = it / p.N;
+        const int d = row0 + rg * 8;
+        if (t >= p.T || d >= p.D) continue;   // D % 64 == 0: 8 rows all in or all out
+        float a[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) a[k] = recv[(rg * 8 + k) * rs + t];
+#pragma unroll
+        for (int src = 1; src < kCluster; ++src)
+#pragma unroll
+          for (int k = 0; k < 8; ++k) a[k] += recv[(src * kRowsPer + rg * 8 + k) * rs + t];
+        *reinterpret_cast<uint4*>(p.y + int64_t(t) * p.D + d) =
+            make_uint4(pack_bf2(a[0], a[1]), pack_bf2(a[2], a[3]), pack_bf2(a[4], a[5]),
+                       pack_bf2(a[6], a[7]));
+      }
+    }
+  }
   if (warp == 1) {
     __syncwarp();
     tmem_dealloc(tmem_base, tmem_cols);

@@ -187,6 +187,16 @@ DecodePlan plan_decode(int T, int D, int F, int FT, int num_sms) {
   // every block needs at least one down unit (so the blocks covering a down
   // tile are consecutive and each writes its partial slot)
   pl.grid = std::max(1, std::min(std::min(num_sms, kMaxDecodeGrid), pl.Ud));
+  // Prefer the largest grid that divides the down units, if it keeps at
+  // least 3/4 of the SMs: every block then streams the same share of W_down,
+  // a down tile's pieces are whole blocks' ranges, and the SMs left over
+  // take the split-k sum kernel's blocks at once (1024 units: 128 blocks of
+  // eight instead of 148 of six or seven).
+  for (int g = pl.grid; 4 * g >= 3 * pl.grid; --g)
+    if (pl.Ud % g == 0) {
+      pl.grid = g;
+      break;
+    }
   // With more gate/up tiles than blocks, use the fewest blocks that take the
   // same largest number of tiles each, so that no block makes more tiles
   // than the others (172 tiles: 86 blocks of two instead of 148 of one or two).
@@ -203,7 +213,9 @@ DecodePlan plan_decode(int T, int D, int F, int FT, int num_sms) {
 }  // namespace
 
 size_t decode_flag_bytes(int D, int F) {
-  const size_t words = size_t((F / 64) + cdiv(D, fused::BM) + 2);
+  (void)D;
+  // ready flags and the cluster path's count of blocks past their z poll
+  const size_t words = size_t((F / 64) + 2);
   return (words * sizeof(uint32_t) + 255) & ~size_t(255);
 }
 
@@ -264,62 +276,111 @@ staple_status tc_decode_fwd(const DeviceInfo& di, int T, int D, int F, const voi
   p.part = static_cast<float*>(part);
   p.err = err;
   p.wait_ns = di.wait_ns;
+  p.fin = words + F / 64;
 
-  // down-step ordering only where some block makes two or more gate/up tiles
-  const int order = pl.G > pl.grid ? 1 : 0;
   using Kern = void (*)(CUtensorMap, CUtensorMap, CUtensorMap, CUtensorMap, CUtensorMap,
                         fused::Params);
-  // [order][stem]
-  const Kern kerns[2][2] = {{fused::decode_fused_kernel<false, false>,
-                             fused::decode_fused_kernel<false, true>},
-                            {fused::decode_fused_kernel<true, false>,
-                             fused::decode_fused_kernel<true, true>}};
-  const Kern kern = kerns[order][stem ? 1 : 0];
+  // [cluster][order][stem]
+  const Kern kerns[2][2][2] = {{{fused::decode_fused_kernel<false, false, false>,
+                                 fused::decode_fused_kernel<false, true, false>},
+                                {fused::decode_fused_kernel<true, false, false>,
+                                 fused::decode_fused_kernel<true, true, false>}},
+                               {{fused::decode_fused_kernel<false, false, true>,
+                                 fused::decode_fused_kernel<false, true, true>},
+                                {fused::decode_fused_kernel<true, false, true>,
+                                 fused::decode_fused_kernel<true, true, true>}}};
   const int smem = fused::smem_bytes(pl.N, pl.sub, FT);
-  // Blocks wait (bounded) on flags other blocks raise, so the whole grid must
-  // be resident at once.  Checked once per device, kernel and shared-memory
-  // size (queried outside any stream capture on first use): the grid may not
-  // exceed the SMs times the blocks one SM can hold.
   static std::atomic<uint64_t> attr_done{0};
   const uint64_t bit = uint64_t(1) << (di.device & 63);
   if (!(attr_done.load() & bit)) {
-    for (const auto& row : kerns)
-      for (Kern k : row)
-        if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024) !=
-            cudaSuccess)
-          return STAPLE_ECUDA;
+    for (const auto& a : kerns)
+      for (const auto& row : a)
+        for (Kern k : row)
+          if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024) !=
+              cudaSuccess)
+            return STAPLE_ECUDA;
     attr_done.fetch_or(bit);
   }
-  int per_sm = 0;
-  {
+  // Blocks wait (bounded) on flags other blocks raise, so the whole grid must
+  // be resident at once.  Checked per device, kernel, shared-memory size and
+  // cluster size (queried outside any stream capture on first use): the
+  // grid may not exceed what the device can hold at once, in blocks or in
+  // clusters.
+  auto resident = [&](Kern k, int cluster) -> int {
     static std::mutex mu;
-    static std::map<std::tuple<const void*, int, int>, int> resident;   // (kernel, device, smem)
+    static std::map<std::tuple<const void*, int, int, int>, int> known;
     std::lock_guard<std::mutex> lock(mu);
-    const auto key = std::make_tuple(reinterpret_cast<const void*>(kern), di.device, smem);
-    auto it = resident.find(key);
-    if (it == resident.end()) {
-      if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, fused::kThreads, smem) !=
-          cudaSuccess)
-        return STAPLE_ECUDA;
-      it = resident.emplace(key, per_sm).first;
+    const auto key = std::make_tuple(reinterpret_cast<const void*>(k), di.device, smem, cluster);
+    auto it = known.find(key);
+    if (it != known.end()) return it->second;
+    int n = 0;
+    if (cluster == 1) {
+      if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, k, fused::kThreads, smem) != cudaSuccess)
+        return -1;
+      n *= di.num_sms;
+    } else {
+      cudaLaunchConfig_t q = {};
+      q.gridDim = dim3(cluster);
+      q.blockDim = dim3(fused::kThreads);
+      q.dynamicSmemBytes = smem;
+      cudaLaunchAttribute ca[1];
+      ca[0].id = cudaLaunchAttributeClusterDimension;
+      ca[0].val.clusterDim.x = cluster;
+      ca[0].val.clusterDim.y = 1;
+      ca[0].val.clusterDim.z = 1;
+      q.attrs = ca;
+      q.numAttrs = 1;
+      if (cudaOccupancyMaxActiveClusters(&n, k, &q) != cudaSuccess) return -1;
     }
-    per_sm = it->second;
+    known.emplace(key, n);
+    return n;
+  };
+  // The cluster path (the split-k sum inside the launch, see the kernel):
+  // one cluster of kCluster blocks per down tile, all resident at once, at
+  // least one down unit per block, the pushed accumulator rows within the
+  // rings, and at least as many blocks as the two-launch path would stream
+  // with (7B layer: 32 tiles, 128 blocks instead of 86).  With fewer tiles
+  // than that (1B layer: 16), a tile would need several clusters whose
+  // partials meet in global memory at the end of the launch, which measured
+  // slower than the sum kernel; those shapes take the two-launch path.
+  int clu = 0;
+  {
+    const int maxcl = resident(kerns[1][0][stem ? 1 : 0], fused::kCluster);
+    if (maxcl < 0) return STAPLE_ECUDA;
+    const size_t rings = size_t(p.stages) * pl.sub * fused::A_BLOCK +
+                         size_t(p.stages_b) * pl.sub * pl.N * fused::BK * 2;
+    const size_t recv = size_t(fused::BM) * (pl.N + 4) * sizeof(float);
+    clu = (maxcl >= pl.Dt && pl.ud >= fused::kCluster && recv <= rings &&
+           pl.Dt * fused::kCluster >= pl.grid) ? 1 : 0;
   }
-  if (per_sm <= 0 || pl.grid > per_sm * di.num_sms) return STAPLE_EUNSUPPORTED;
+  const int grid = clu ? pl.Dt * fused::kCluster : pl.grid;
+  // down-step ordering only where some block makes two or more gate/up tiles
+  const int order = pl.G > grid ? 1 : 0;
+  const Kern kern = kerns[clu][order][stem ? 1 : 0];
+  if (!clu) {
+    const int n = resident(kern, 1);
+    if (n < 0) return STAPLE_ECUDA;
+    if (grid > n) return STAPLE_EUNSUPPORTED;
+  }
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(pl.grid);
+  cfg.gridDim = dim3(grid);
   cfg.blockDim = dim3(fused::kThreads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
+  attr[1].id = cudaLaunchAttributeClusterDimension;
+  attr[1].val.clusterDim.x = fused::kCluster;
+  attr[1].val.clusterDim.y = 1;
+  attr[1].val.clusterDim.z = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = clu ? 2 : 1;
   cudaError_t ce = cudaSuccess;
   STP_LAUNCH(stem ? "k5k6_decode_fused_stem" : "k5k6_decode_fused", st,
              ce = cudaLaunchKernelEx(&cfg, kern, mg, mu, md, mx, mz, p));
   if (ce != cudaSuccess) return STAPLE_ECUDA;
+  if (clu) return STAPLE_OK;
   // the split-k sums, right behind (programmatic dependent, see the kernel)
   fused::ReduceParams r{};
   r.T = T;
