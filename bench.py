@@ -168,10 +168,11 @@ class Clocks:
 # to the captured value; otherwise the roofline's traffic is null.
 CAPTURED_TRAFFIC = {
     "k5k6_decode_fused": {
-        "bytes": 103_142_400,   # mean of two launches: 104,451,072 and 101,833,728
+        "bytes": 103_393_280,   # mean of two launches: 104,610,304 and 102,176,256
         "sources": ["token_indexed_sparse_staple_b200/csrc/decode_fused.cuh",
-                    "token_indexed_sparse_staple_b200/csrc/common.cuh"],
-        "sha256": "1903f43a08b7a700331893f2d67f201b990186af59acd426e195d86118dd1e7b",
+                    "token_indexed_sparse_staple_b200/csrc/common.cuh",
+                    "token_indexed_sparse_staple_b200/csrc/ffn_tc.cu"],   # ffn_tc.cu: grid
+        "sha256": "04d04ec913d1d53d922997e9f2997bd2874e8f90b1c6ba78297ef5c0b7ea0255",
         "profile": "profiles/decode_fused_olmo2_1b_T64.md",
     },
 }
@@ -386,6 +387,29 @@ def run_decode(stp, ctx, w, args, world, local):
 # --------------------------------------------------------------------------
 # Training layer (host table + 5% cache)
 # --------------------------------------------------------------------------
+
+def run_decode_layer(stp, ctx, spec, args, world, local):
+    """Decode steps of one layer of another shape ("D,F": T = 64, vocabulary
+    8192, table in HBM, four rotating weight sets), untraced graph replays:
+    a small case for per-kernel profiling (the 7B shape, 4096,11008, runs the
+    one-launch cluster path).  Prints its own JSON line, not the bench line."""
+    import torch
+    D, F = (int(v) for v in spec.split(","))
+    w = syn.Workload(f"decode-layer-{D}x{F}", T=64, D=D, F=F, V=8192, layers=1, dtype="bf16",
+                     w_std=0.02, e_std=0.01, x_std=1.0, dy_std=1.0, table="device",
+                     cache_frac=0.0, group=1, training=False)
+    st = decode_setup(stp, w, local)
+    stream = torch.cuda.Stream()
+    K = args.steps
+    ms, _, clocks = time_graph_steps(lambda s: decode_step(stp, ctx, w, st, s, stream), K,
+                                     min(64, K), stream, args.warmup, world, local)
+    status = stp.staple_get_error(ctx, stream)
+    alg = 3 * F * D * 2 + w.T * D * 2 + 2 * w.T * F * 2 + 4 * w.T + w.T * D * 2
+    us = ms * 1000.0 / K
+    return {"profile": w.name, "T": w.T, "d_model": D, "d_ff": F, "steps": K,
+            "us_per_step": r3(us), "alg_bytes_per_step": alg,
+            "achieved_gbs": r3(alg / (us * 1e-6) / 1e9), "clocks": clocks, "status": status}
+
 
 def run_train(stp, ctx, w, steps, warmup, world, local):
     import torch
@@ -975,6 +999,8 @@ def main():
     ap.add_argument("--stack-decode-steps", type=int, default=256)
     ap.add_argument("--stack-train-steps", type=int, default=4)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--decode-layer", default=None, metavar="D,F",
+                    help="only time decode steps of one layer of this shape (profiling case)")
     ap.add_argument("--detail", default=None,
                     help="also write every per-kernel table and sub-measurement to this JSON file")
     args = ap.parse_args()
@@ -997,6 +1023,16 @@ def main():
     ctx = stp.staple_context_create(local)
     pk = peaks()
     detail = {}
+    if args.decode_layer:
+        out = run_decode_layer(stp, ctx, args.decode_layer, args, world, local)
+        if rank == 0:
+            print(json.dumps(out), flush=True)
+        stp.staple_context_destroy(ctx)
+        if world > 1:
+            import torch.distributed as dist
+            barrier(world)
+            dist.destroy_process_group()
+        return
     dec = run_decode(stp, ctx, w, args, world, local)
     K = dec["K"]
     value = job_value(w.T * K, dec["ms"], world)
@@ -1058,12 +1094,14 @@ def main():
             st_ms = tr["staple_r0"]["ms"] / args.train_steps
             de_ms = tr["dense"]["ms"] / args.train_steps
             kern = tr["staple_r0"]["kernels"]
-            top = max(kern.items(), key=lambda kv: kv[1]["total_ms"])
             gemm_flops = {"k5_gateup": 4, "k6_down": 2, "k7_dz": 2, "k9_dx": 4, "k10_dw_gate_up": 4,
                           "k10_dw_down": 2}
-            tf = None
-            if top[0] in gemm_flops:
-                tf = gemm_flops[top[0]] * wt.T * wt.D * wt.F / (top[1]["avg_us"] * 1e-6) / 1e12
+            # the dominant kernel of the step's own stream: the largest GEMM (the
+            # miss gather runs on a side stream under the previous microbatch's
+            # GEMMs and is rated against the host link below)
+            top = max(((k, v) for k, v in kern.items() if k in gemm_flops),
+                      key=lambda kv: kv[1]["total_ms"])
+            tf = gemm_flops[top[0]] * wt.T * wt.D * wt.F / (top[1]["avg_us"] * 1e-6) / 1e12
             link = measure_host_link()
             adamw = measure_host_adamw(stp, wt)
             k4 = kern.get("k4_gather_misses")
