@@ -342,35 +342,67 @@ def run_decode(stp, ctx, w, args, world, local):
     # a captured launch holds one pair of trace events, re-recorded by every
     # replay: the records cover the G captured steps once
     res["launches_per_step"] = sum(d["launches"] for d in kern.values()) / G
-    # end to end through the public call with host buffers: H2D of x and ids
-    # from pinned memory, the layer, D2H of y, every step
+    # end to end through the public call with host buffers: every step copies
+    # its x and ids in from pinned memory and its y out.  As a serving loop
+    # would, the copies run on two copy streams, double-buffered, so that a
+    # step's copies overlap its neighbours' layer calls, and the steps are
+    # captured in CUDA graphs of G steps like the kernel-only run.
     Ke = K
     h2d = st["x"][0].numel() * 2 + st["ids"][0].numel() * 4
     d2h = st["y"].numel() * 2
-    xd = torch.empty_like(st["x"][0])
-    idd = torch.empty_like(st["ids"][0])
-    embd = stp.make_embed(stp.STAPLE_EMBED_TABLE, st["table"], w.F, idd, w.V)
+    cin, cout = torch.cuda.Stream(), torch.cuda.Stream()
+    xd = [torch.empty_like(st["x"][0]) for _ in range(2)]
+    idd = [torch.empty_like(st["ids"][0]) for _ in range(2)]
+    yd = [torch.empty_like(st["y"]) for _ in range(2)]
+    embd = [stp.make_embed(stp.STAPLE_EMBED_TABLE, st["table"], w.F, idd[i], w.V) for i in range(2)]
+    ev_in, ev_used, ev_out = ([torch.cuda.Event() for _ in range(2)] for _ in range(3))
 
     def e2e_step(s):
-        r, b = s % st["R"], s % st["S"]
-        xd.copy_(st["x_host"][b], non_blocking=True)
-        idd.copy_(st["ids_host"][b], non_blocking=True)
-        stp.staple_ffn_fwd(ctx, stp.STAPLE_BF16, w.T, w.D, w.F, xd, embd, st["wg"][r], st["wu"][r],
-                           st["wd"][r], st["z"], st["y"], None, None, st["ws"], st["wsb"],
-                           stream=stream)
-        st["y_host"][b].copy_(st["y"], non_blocking=True)
+        i, r, b = s % 2, s % st["R"], s % st["S"]
+        cin.wait_event(ev_used[i])        # the call two steps back has read xd[i], idd[i]
+        with torch.cuda.stream(cin):
+            xd[i].copy_(st["x_host"][b], non_blocking=True)
+            idd[i].copy_(st["ids_host"][b], non_blocking=True)
+        ev_in[i].record(cin)
+        stream.wait_event(ev_in[i])
+        stream.wait_event(ev_out[i])      # yd[i] of two steps back is on the host
+        stp.staple_ffn_fwd(ctx, stp.STAPLE_BF16, w.T, w.D, w.F, xd[i], embd[i], st["wg"][r],
+                           st["wu"][r], st["wd"][r], st["z"], yd[i], None, None, st["ws"],
+                           st["wsb"], stream=stream)
+        ev_used[i].record(stream)
+        cout.wait_event(ev_used[i])
+        with torch.cuda.stream(cout):
+            st["y_host"][b].copy_(yd[i], non_blocking=True)
+        ev_out[i].record(cout)
 
+    def e2e_graph(n):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            for e in ev_used + ev_out:     # fork the copy streams into the capture
+                e.record(stream)
+            for s in range(n):
+                e2e_step(s)
+            stream.wait_stream(cin)        # and join them before it ends
+            stream.wait_stream(cout)
+        return g
+
+    G = min(64, Ke)
+    full = e2e_graph(G)
+    rem = e2e_graph(Ke % G) if Ke % G else None
     with torch.cuda.stream(stream):
-        for s in range(8):
-            e2e_step(s)
+        for _ in range(max(1, args.warmup // G)):
+            full.replay()
         torch.cuda.synchronize()
         barrier(world)
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
-        for s in range(Ke):
-            e2e_step(s)
+        for _ in range(Ke // G):
+            full.replay()
+        if rem is not None:
+            rem.replay()
         e1.record(stream)
         torch.cuda.synchronize()
+    del full, rem
     e_ms = max_over_ranks(e0.elapsed_time(e1), world)
     res["e2e"] = {"K": Ke, "ms": e_ms, "h2d": h2d, "d2h": d2h}
     # dominant (and only) kernel: the fused decode launch.  Algorithmic bytes
@@ -1067,7 +1099,9 @@ def main():
         "e2e": {"value": r3(job_value(w.T * dec["e2e"]["K"], dec["e2e"]["ms"], world)),
                 "unit": "tokens/s", "h2d_bytes_per_step": dec["e2e"]["h2d"],
                 "d2h_bytes_per_step": dec["e2e"]["d2h"], "steps": dec["e2e"]["K"],
-                "how": "per step: pinned H2D of x and ids, staple_ffn_fwd, D2H of y"},
+                "how": ("per step: pinned H2D of x and ids on a copy stream, staple_ffn_fwd, "
+                        "D2H of y on another copy stream; double-buffered, steps in CUDA graphs "
+                        "of 64")},
         "gpu_launches": int(round(dec["launches_per_step"] * K)),
         "clocks": dec["clocks"],
         "decode_dense": {"us_per_step": r3(dense_us), "us_per_step_staple": r3(step_us),
