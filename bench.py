@@ -172,7 +172,7 @@ CAPTURED_TRAFFIC = {
         "sources": ["token_indexed_sparse_staple_b200/csrc/decode_fused.cuh",
                     "token_indexed_sparse_staple_b200/csrc/common.cuh",
                     "token_indexed_sparse_staple_b200/csrc/ffn_tc.cu"],   # ffn_tc.cu: grid
-        "sha256": "04d04ec913d1d53d922997e9f2997bd2874e8f90b1c6ba78297ef5c0b7ea0255",
+        "sha256": "b1b6ba17135675dfabb65430f207951aafebc7d6f7ec3f50aff5152d862db984",
         "profile": "profiles/decode_fused_olmo2_1b_T64.md",
     },
 }

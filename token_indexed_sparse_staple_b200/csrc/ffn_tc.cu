@@ -131,16 +131,41 @@ staple_status launch(const char* name, const DeviceInfo& di, const CUtensorMap& 
       return STAPLE_ECUDA;
     attr_done.fetch_or(bit);
   }
-  // The fewest blocks that take the same largest number of tiles each: with
-  // 512 tiles on 148 SMs, 128 blocks of four finish when 148 blocks of three
-  // or four would, and leave 20 SMs to kernels on other streams.
   const int avail = std::max(1, di.num_sms - di.sm_reserve);
-  const int per_block = (ntiles + avail - 1) / avail;
-  const int grid = (ntiles + per_block - 1) / per_block;
+  // fp32 outputs (the weight gradients): when the tiles of the last, partial
+  // round, taken twice, still fit in one round, each of them runs as two
+  // halves of its k range that add onto a zeroed output.  That round then
+  // takes half as long (dW_down, 512 tiles on 148 SMs: 3.5 rounds of work
+  // instead of 4).  Both halves add onto zero, so the sum (0 + a) + b is the
+  // same whichever lands first.
+  p.nsplit = 0;
+  p.kb_split = 0;
+  if (EPI == tc::EPI_F32 && p.k_blocks >= 2) {
+    const int rem = ntiles % avail;
+    if (rem > 0 && 2 * rem <= avail) {
+      p.nsplit = rem;
+      p.kb_split = p.k_blocks / 2;
+    }
+  }
+  int grid;
+  if (p.nsplit > 0) {
+    grid = std::min(avail, ntiles + p.nsplit);
+  } else {
+    // The fewest blocks that take the same largest number of tiles each
+    // (1024 tiles on 148 SMs: 147 blocks of seven), leaving the rest of the
+    // SMs to kernels on other streams.
+    const int per_block = (ntiles + avail - 1) / avail;
+    grid = (ntiles + per_block - 1) / per_block;
+  }
   const CUtensorMap& o0 = o ? o[0] : a;
   const CUtensorMap& o1 = o ? o[1] : a;
   const CUtensorMap& o2 = o ? o[2] : a;
   const CUtensorMap& o3 = (o && EPI == tc::EPI_DZ) ? o[3] : a;
+  if (p.nsplit > 0) {
+    STP_LAUNCH("gemm_split_zero", st,
+               tc::zero_split_tiles_kernel<<<p.nsplit, 256, 0, st>>>(p));
+    if (cudaGetLastError() != cudaSuccess) return STAPLE_ECUDA;
+  }
   STP_LAUNCH(name, st,
              kern<<<grid, tc::kThreads, tc::smem_bytes<EPI>(), st>>>(a, b0, b1, o0, o1, o2, o3,
                                                                       p));

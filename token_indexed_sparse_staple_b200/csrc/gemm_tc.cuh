@@ -58,6 +58,11 @@ constexpr int smem_bytes() { return kSmemBytes + 4 * out_blocks<EPI>() * kOutBox
 struct Params {
   int32_t M, N, K;            // output rows, output columns (features for GATEUP / DZ), K
   int32_t tiles_m, tiles_n, k_blocks;
+  // EPI_F32: the last nsplit tiles (raster order) run as two work items each,
+  // k blocks [0, kb_split) and [kb_split, k_blocks), which both add their sums
+  // (red.add) onto an output the launcher zeroed: the last, partial round of
+  // tiles then takes half as long.  0: every tile is one item.
+  int32_t nsplit, kb_split;
   int32_t ksplit;             // B_KSPLIT: first k served by the second B tensor
   int32_t group_m;            // tile raster: group_m M-blocks per sweep over N
   // EPI_BF16 / EPI_F32: out[m * ldo + n]; rows m >= m_split go to out2[(m - m_split) * ldo + n]
@@ -82,6 +87,28 @@ struct Params {
   int32_t* err;
   uint64_t wait_ns;           // bound of every wait (STAPLE_ETIMEOUT past it)
 };
+
+// Work item t: its tile and k-block range [kb0, kb1); add: a split tile's half.
+__device__ __forceinline__ int item_tile(int t, const Params& p, int& kb0, int& kb1, bool& add) {
+  const int nfull = p.tiles_m * p.tiles_n - p.nsplit;
+  if (t < nfull) {
+    kb0 = 0;
+    kb1 = p.k_blocks;
+    add = false;
+    return t;
+  }
+  const int h = (t - nfull) & 1;
+  kb0 = h ? p.kb_split : 0;
+  kb1 = h ? p.k_blocks : p.kb_split;
+  add = true;
+  return nfull + ((t - nfull) >> 1);
+}
+
+__device__ __forceinline__ void red_add4(float* a, float x, float y, float z, float w) {
+  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(a), "f"(x), "f"(y), "f"(z),
+               "f"(w)
+               : "memory");
+}
 
 __device__ __forceinline__ void tile_coords(int t, const Params& p, int& mb, int& nb) {
   const int per_group = p.group_m * p.tiles_n;
@@ -221,7 +248,7 @@ __device__ __forceinline__ int dz_chunks(const Params& p, int nb) {
 template <int EPI>
 __device__ __forceinline__ void epilogue_tile(const Params& p, uint32_t tacc, int m, int nb,
                                               int lane, uint8_t* stg, const OutMaps& om,
-                                              DzIn& in, int nxt_nb, int nxt_row0) {
+                                              DzIn& in, int nxt_nb, int nxt_row0, bool add) {
   const bool row_ok = m < p.M;
   const int m0w = m - lane;   // the warp's first row
   if constexpr (EPI == EPI_BF16 || EPI == EPI_F32) {
@@ -241,10 +268,16 @@ __device__ __forceinline__ void epilogue_tile(const Params& p, uint32_t tacc, in
           float* base = m < p.m_split
                             ? static_cast<float*>(p.out) + int64_t(m) * p.ldo
                             : static_cast<float*>(p.out2) + int64_t(m - p.m_split) * p.ldo;
-          float4* d = reinterpret_cast<float4*>(base + n);
+          if (add) {
 #pragma unroll
-          for (int i = 0; i < 8; ++i)
-            d[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+            for (int i = 0; i < 8; ++i)
+              red_add4(base + n + 4 * i, v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+          } else {
+            float4* d = reinterpret_cast<float4*>(base + n);
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+              d[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+          }
         }
       }
     }
@@ -439,6 +472,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
   const int ntiles = p.tiles_m * p.tiles_n;
+  const int nitems = ntiles + p.nsplit;   // work items (a split tile is two)
 
   if (warp == 0) {
     if (lane == 0) {
@@ -447,11 +481,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t phase = 0;
       bool ok = true;
       int issued = 0;
-      for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
-        int mb, nb;
-        tile_coords(t, p, mb, nb);
+      for (int t = blockIdx.x; t < nitems && ok; t += gridDim.x) {
+        int mb, nb, kb0, kb1;
+        bool add;
+        tile_coords(item_tile(t, p, kb0, kb1, add), p, mb, nb);
         const int m0 = mb * BM;
-        for (int kb = 0; kb < p.k_blocks; ++kb) {
+        for (int kb = kb0; kb < kb1; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag, p.err, p.wait_ns)) {
             ok = false;
             break;
@@ -506,13 +541,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t phase = 0;
       int iter = 0;
       bool ok = true;
-      for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x, ++iter) {
+      for (int t = blockIdx.x; t < nitems && ok; t += gridDim.x, ++iter) {
         const int buf = iter & 1;
         const uint32_t use = uint32_t(iter >> 1);
         if (!mbar_wait(&tempty[buf], (use & 1) ^ 1, abort_flag, p.err, p.wait_ns)) break;
         tc_fence_after();
         const uint32_t dacc = tmem_base + uint32_t(buf * BN);
-        for (int kb = 0; kb < p.k_blocks; ++kb) {
+        int kb0, kb1;
+        bool add;
+        item_tile(t, p, kb0, kb1, add);
+        for (int kb = kb0; kb < kb1; ++kb) {
           if (!mbar_wait(&full[stage], phase, abort_flag, p.err, p.wait_ns)) {
             ok = false;
             break;
@@ -526,7 +564,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                                      : sw128_desc(a_addr + k * 32, 16, 1024);
             const uint64_t bd = B_MN ? sw128_desc(b_addr + k * 2048, B_STAGE / 4, 1024)
                                      : sw128_desc(b_addr + k * 32, 16, 1024);
-            umma_bf16(dacc, ad, bd, idesc, (kb | k) != 0 ? 1u : 0u);
+            umma_bf16(dacc, ad, bd, idesc, (kb != kb0 || k != 0) ? 1u : 0u);
           }
           umma_commit(&empty[stage]);
           if (++stage == STAGES) {
@@ -554,13 +592,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       dz_load(in, stg, om, nb * BN, mb * BM + q * 32);   // the first tile's first chunk
     }
     int iter = 0;
-    for (int t = blockIdx.x; t < ntiles; t += gridDim.x, ++iter) {
+    for (int t = blockIdx.x; t < nitems; t += gridDim.x, ++iter) {
       const int buf = iter & 1;
       const uint32_t use = uint32_t(iter >> 1);
-      int mb, nb;
-      tile_coords(t, p, mb, nb);
+      int mb, nb, kb0, kb1;
+      bool add;
+      tile_coords(item_tile(t, p, kb0, kb1, add), p, mb, nb);
       int nxt_nb = -1, nxt_row0 = 0;
-      if (t + int(gridDim.x) < ntiles) {
+      if (t + int(gridDim.x) < ntiles) {   // (EPI_DZ: no split tiles, items are tiles)
         int mb2;
         tile_coords(t + gridDim.x, p, mb2, nxt_nb);
         nxt_row0 = mb2 * BM + q * 32;
@@ -569,7 +608,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!__all_sync(0xffffffffu, ok)) break;
       tc_fence_after();
       const uint32_t tacc = tmem_base + (uint32_t(q * 32) << 16) + uint32_t(buf * BN);
-      epilogue_tile<EPI>(p, tacc, mb * BM + row, nb, lane, stg, om, in, nxt_nb, nxt_row0);
+      epilogue_tile<EPI>(p, tacc, mb * BM + row, nb, lane, stg, om, in, nxt_nb, nxt_row0, add);
       if (!in.ok) break;
       tc_fence_before();
       __syncwarp();
@@ -588,6 +627,21 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 1) {
     __syncwarp();
     tmem_dealloc(tmem_base, kTmemCols);
+  }
+}
+
+// Zero the output of the split tiles (EPI_F32), which both halves then add
+// onto: block i takes split tile i, 128 rows x 256 columns of fp32.
+__global__ void __launch_bounds__(256) zero_split_tiles_kernel(const Params p) {
+  const int t = p.tiles_m * p.tiles_n - p.nsplit + int(blockIdx.x);
+  int mb, nb;
+  tile_coords(t, p, mb, nb);
+  for (int i = threadIdx.x; i < BM * (BN / 4); i += 256) {
+    const int m = mb * BM + i / (BN / 4), n = nb * BN + (i % (BN / 4)) * 4;
+    if (m >= p.M || n >= p.N) continue;
+    float* base = m < p.m_split ? static_cast<float*>(p.out) + int64_t(m) * p.ldo
+                                : static_cast<float*>(p.out2) + int64_t(m - p.m_split) * p.ldo;
+    *reinterpret_cast<float4*>(base + n) = make_float4(0.f, 0.f, 0.f, 0.f);
   }
 }
 
