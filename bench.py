@@ -443,6 +443,47 @@ def run_decode_layer(stp, ctx, spec, args, world, local):
             "achieved_gbs": r3(alg / (us * 1e-6) / 1e9), "clocks": clocks, "status": status}
 
 
+def run_dw_down(stp, ctx, args, world, local):
+    """The training layer's dW_down GEMM alone (staple_ffn_bwd with only
+    dw_down: dW_down = dY^T z, T = 16384, D = 2048, F = 8192), L2 flushed
+    between calls: a small case for capturing it under ncu (about 1 GB on
+    the device).  Prints its own JSON line, not the bench line."""
+    import torch
+    w = syn.WORKLOADS["olmo2-1b-train-layer"]
+    T, D, F = w.T, w.D, w.F
+    dy = bf16_randn((T, D), 1.0, syn.SEED_ACT)
+    z = bf16_randn((T, F), 1.0, syn.SEED_ACT + 1)
+    # x and dgh are passed as the call requires; only dx and dW_gate/up read them
+    x = torch.zeros((T, D), dtype=torch.bfloat16, device="cuda")
+    dgh = torch.zeros((T, 2 * F), dtype=torch.bfloat16, device="cuda")
+    dwd = torch.empty((D, F), dtype=torch.float32, device="cuda")
+    wsb = stp.staple_workspace_bytes(T, D, F)
+    ws = torch.zeros(wsb, dtype=torch.uint8, device="cuda")
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    stream = torch.cuda.current_stream()
+
+    def call():
+        stp.staple_ffn_bwd(ctx, stp.STAPLE_BF16, T, D, F, dy, x, z, dgh, None, None, None,
+                           None, None, dwd, stream=stream)
+
+    for _ in range(max(3, args.warmup)):
+        call()
+    torch.cuda.synchronize()
+    ts = []
+    for _ in range(args.steps):
+        flush.zero_()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        call()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        ts.append(e0.elapsed_time(e1) * 1000.0)
+    us = statistics.median(ts)
+    return {"profile": "dw-down", "T": T, "d_model": D, "d_ff": F, "calls": args.steps,
+            "us_median": r3(us), "tflops": r3(2.0 * T * D * F / (us * 1e-6) / 1e12),
+            "status": stp.staple_get_error(ctx, stream)}
+
+
 def run_train(stp, ctx, w, steps, warmup, world, local):
     import torch
     T, D, F, V = w.T, w.D, w.F, w.V
@@ -1031,6 +1072,8 @@ def main():
     ap.add_argument("--stack-decode-steps", type=int, default=256)
     ap.add_argument("--stack-train-steps", type=int, default=4)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--dw-down", action="store_true",
+                    help="only time the training layer's dW_down GEMM (profiling case)")
     ap.add_argument("--decode-layer", default=None, metavar="D,F",
                     help="only time decode steps of one layer of this shape (profiling case)")
     ap.add_argument("--detail", default=None,
@@ -1055,8 +1098,9 @@ def main():
     ctx = stp.staple_context_create(local)
     pk = peaks()
     detail = {}
-    if args.decode_layer:
-        out = run_decode_layer(stp, ctx, args.decode_layer, args, world, local)
+    if args.decode_layer or args.dw_down:
+        out = (run_dw_down(stp, ctx, args, world, local) if args.dw_down
+               else run_decode_layer(stp, ctx, args.decode_layer, args, world, local))
         if rank == 0:
             print(json.dumps(out), flush=True)
         stp.staple_context_destroy(ctx)

@@ -163,7 +163,7 @@ staple_status launch(const char* name, const DeviceInfo& di, const CUtensorMap& 
   const CUtensorMap& o3 = (o && EPI == tc::EPI_DZ) ? o[3] : a;
   if (p.nsplit > 0) {
     STP_LAUNCH("gemm_split_zero", st,
-               tc::zero_split_tiles_kernel<<<p.nsplit, 256, 0, st>>>(p));
+               tc::zero_split_tiles_kernel<<<p.nsplit * (tc::BM / tc::kZeroRows), 256, 0, st>>>(p));
     if (cudaGetLastError() != cudaSuccess) return STAPLE_ECUDA;
   }
   STP_LAUNCH(name, st,

@@ -631,13 +631,16 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 // Zero the output of the split tiles (EPI_F32), which both halves then add
-// onto: block i takes split tile i, 128 rows x 256 columns of fp32.
+// onto: block i takes rows 16 (i % 8) .. +15 of split tile i / 8 (256 fp32
+// columns), four float4 stores per thread.
+constexpr int kZeroRows = 16;
 __global__ void __launch_bounds__(256) zero_split_tiles_kernel(const Params p) {
-  const int t = p.tiles_m * p.tiles_n - p.nsplit + int(blockIdx.x);
+  const int t = p.tiles_m * p.tiles_n - p.nsplit + int(blockIdx.x) / (BM / kZeroRows);
+  const int r0 = (int(blockIdx.x) % (BM / kZeroRows)) * kZeroRows;
   int mb, nb;
   tile_coords(t, p, mb, nb);
-  for (int i = threadIdx.x; i < BM * (BN / 4); i += 256) {
-    const int m = mb * BM + i / (BN / 4), n = nb * BN + (i % (BN / 4)) * 4;
+  for (int i = threadIdx.x; i < kZeroRows * (BN / 4); i += 256) {
+    const int m = mb * BM + r0 + i / (BN / 4), n = nb * BN + (i % (BN / 4)) * 4;
     if (m >= p.M || n >= p.N) continue;
     float* base = m < p.m_split ? static_cast<float*>(p.out) + int64_t(m) * p.ldo
                                 : static_cast<float*>(p.out2) + int64_t(m - p.m_split) * p.ldo;
