@@ -172,7 +172,7 @@ CAPTURED_TRAFFIC = {
         "sources": ["token_indexed_sparse_staple_b200/csrc/decode_fused.cuh",
                     "token_indexed_sparse_staple_b200/csrc/common.cuh",
                     "token_indexed_sparse_staple_b200/csrc/ffn_tc.cu"],   # ffn_tc.cu: grid
-        "sha256": "b1b6ba17135675dfabb65430f207951aafebc7d6f7ec3f50aff5152d862db984",
+        "sha256": "04826201685b1e8820649aa11eb1499cd19cadefc4c087ed5f73fb38ba1962fa",
         "profile": "profiles/decode_fused_olmo2_1b_T64.md",
     },
 }
