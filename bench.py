@@ -169,10 +169,13 @@ class Clocks:
 CAPTURED_TRAFFIC = {
     "k5k6_decode_fused": {
         "bytes": 103_393_280,   # mean of two launches: 104,610,304 and 102,176,256
-        "sources": ["token_indexed_sparse_staple_b200/csrc/decode_fused.cuh",
-                    "token_indexed_sparse_staple_b200/csrc/common.cuh",
-                    "token_indexed_sparse_staple_b200/csrc/ffn_tc.cu"],   # ffn_tc.cu: grid
-        "sha256": "04826201685b1e8820649aa11eb1499cd19cadefc4c087ed5f73fb38ba1962fa",
+        # (file, first marker, end marker): the decode launcher's part of ffn_tc.cu sets the grid
+        "sources": [("token_indexed_sparse_staple_b200/csrc/decode_fused.cuh", None, None),
+                    ("token_indexed_sparse_staple_b200/csrc/common.cuh", None, None),
+                    ("token_indexed_sparse_staple_b200/csrc/ffn_tc.cu",
+                     "// ---------------------------------------------------------------- decode",
+                     "staple_status tc_ffn_fwd(")],
+        "sha256": "264d06806942323181ec84b5977a4d8d235d15407759d4e45b45e8ad32a8bd84",
         "profile": "profiles/decode_fused_olmo2_1b_T64.md",
     },
 }
@@ -183,9 +186,16 @@ def captured_traffic(kernel):
     if c is None:
         return None, "no capture"
     h = hashlib.sha256()
-    for f in c["sources"]:
+    for f, first, end in c["sources"]:
         with open(os.path.join(ROOT, f), "rb") as fh:
-            h.update(fh.read())
+            text = fh.read()
+        if first is not None:
+            i = text.find(first.encode())
+            j = text.find(end.encode(), i)
+            if i < 0 or j < 0:
+                return None, "decode launcher not found for the capture in " + c["profile"]
+            text = text[i:j]
+        h.update(text)
     if h.hexdigest() != c["sha256"]:
         return None, "kernel changed since the capture in " + c["profile"]
     return c["bytes"], c["profile"]
