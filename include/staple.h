@@ -314,11 +314,15 @@ typedef struct staple_embed {
  * T >= 0.  fp32 needs F a multiple of 8.
  * bf16 with 1 <= T <= 256 (decode sizes; the pages serve at batch 64 on one
  * B200: thelatestinai listing, Table 4) runs one persistent kernel that
- * streams both projections' weights across all SMs and needs the workspace
+ * streams both projections' weights across the SMs and needs the workspace
  * (staple_workspace_bytes, zero-filled once); larger T runs the tiled GEMMs
- * and ignores it.  That kernel's blocks wait on one another, so its whole
- * grid must be resident at once: STAPLE_EUNSUPPORTED when the device cannot
- * hold it (the grid exceeds the SMs times the blocks per SM). */
+ * and ignores it.  The down projection's split-k pieces are summed either by
+ * a second, small kernel, or, when the layer has enough down tiles (128-row
+ * blocks of d_model; e.g. d_model 4096), inside the same launch by clusters
+ * of 4 blocks through distributed shared memory.  The persistent kernel's
+ * blocks wait on one another, so its whole grid must be resident at once:
+ * STAPLE_EUNSUPPORTED when the device cannot hold it (the grid exceeds what
+ * the device holds at once, in blocks or in clusters). */
 staple_status staple_ffn_fwd(staple_context* ctx, staple_dtype dtype, int32_t T, int32_t D,
                              int32_t F, const void* x, const staple_embed* embed,
                              const void* w_gate, const void* w_up, const void* w_down, void* z,
