@@ -277,6 +277,13 @@ __global__ void __launch_bounds__(1024)
 // ---------------------------------------------------------------------------
 enum GatherMode { G_HITS = 0, G_MISSES = 1, G_LIST = 2, G_REFRESH = 3, G_SCATTER = 4 };
 
+// The work items are 2 KB chunks of rows (a warp's four 16-byte loads per
+// lane), in row-major order: with a few long rows (a decode step's misses,
+// 88 KB each for four grouped 7B layers) every warp of the grid still has one
+// in flight, where one warp per row would leave most of them idle and walk
+// each row one round trip at a time.
+constexpr int kChunkVecs = 128;
+
 template <int MODE>
 __global__ void __launch_bounds__(256)
     gather_kernel(const uint8_t* __restrict__ src, int64_t src_pitch,
@@ -288,7 +295,11 @@ __global__ void __launch_bounds__(256)
   const int nw = (gridDim.x * blockDim.x) >> 5;
   const int n = *count_dev;
   const int64_t vecs = row_bytes / 16;
-  for (int i = gw; i < n; i += nw) {
+  const int64_t cpr = (vecs + kChunkVecs - 1) / kChunkVecs;   // chunks per row
+  const int64_t items = int64_t(n) * cpr;
+  for (int64_t it = gw; it < items; it += nw) {
+    const int i = int(it / cpr);
+    const int64_t c0 = (it - int64_t(i) * cpr) * kChunkVecs;
     int j;
     int64_t srow;
     if (MODE == G_HITS) {          // rows[j] = cache[slot[j]] for hits
@@ -311,15 +322,17 @@ __global__ void __launch_bounds__(256)
     }
     const uint4* sp = reinterpret_cast<const uint4*>(src + srow * src_pitch);
     uint4* dp = reinterpret_cast<uint4*>(rows + int64_t(j) * row_bytes);
-    int64_t v = lane;
-    for (; v + 96 < vecs; v += 128) {
+    const int64_t vend = c0 + kChunkVecs < vecs ? c0 + kChunkVecs : vecs;
+    int64_t v = c0 + lane;
+    if (v + 96 < vend) {
       const uint4 a0 = sp[v], a1 = sp[v + 32], a2 = sp[v + 64], a3 = sp[v + 96];
       dp[v] = a0;
       dp[v + 32] = a1;
       dp[v + 64] = a2;
       dp[v + 96] = a3;
+    } else {
+      for (; v < vend; v += 32) dp[v] = sp[v];
     }
-    for (; v < vecs; v += 32) dp[v] = sp[v];
   }
 }
 

@@ -100,13 +100,17 @@ class Retrieval:
         return stp.make_embed(stp.STAPLE_EMBED_ROWS, base, self.G * self.F, self.inverse, self.T)
 
 
-def issue_dedup(ctx, r: Retrieval, ids, V: int, stream):
+def issue_dedup(ctx, r: Retrieval, ids, V: int, stream, u_to_host: bool = True):
+    """The batch's dedup on `stream`; with u_to_host, U is also copied to pinned
+    host memory (the training stack reads it there; a decode step does not,
+    and the copy would sit between the dedup and the first gather)."""
     import torch
     stp.staple_dedup(ctx, ids, r.T, V, r.unique, r.inverse, r.seg, r.sorted_pos, r.U,
                      stream=stream)
-    with torch.cuda.stream(stream):
-        r.U_host.copy_(r.U, non_blocking=True)   # 4 bytes; read by the host much later
-    r.U_known.record(stream)
+    if u_to_host:
+        with torch.cuda.stream(stream):
+            r.U_host.copy_(r.U, non_blocking=True)   # 4 bytes; read by the host much later
+        r.U_known.record(stream)
 
 
 def issue_group(ctx, r: Retrieval, tables: GroupedTables, g: int, stream, side):
@@ -288,7 +292,7 @@ class DecodeStack:
         st = stream or torch.cuda.current_stream()
         r = self.r
         self.pf.wait_stream(st)
-        issue_dedup(self.ctx, r, self.ids_buf, self.V, self.pf)
+        issue_dedup(self.ctx, r, self.ids_buf, self.V, self.pf, u_to_host=False)
         for gi in range(self.tables.n_groups):
             issue_group(self.ctx, r, self.tables, gi, self.pf, self.pf_side)
         for l in range(self.L):
