@@ -821,12 +821,11 @@ def run_stack_decode(stp, ctx, w, steps, world, local):
             s.run(st)
         torch.cuda.synchronize()
         assert stp.staple_get_error(ctx, st) == 0
-        s.capture(st)
+        # one graph per recorded batch: each step's graph copies that batch's ids and x in
+        graphs = [s.capture(st, ids[k], xs[k]) for k in range(S)]
 
         def one(k):
-            s.ids_buf.copy_(ids[k % S])
-            s.xs[0].copy_(xs[k % S])
-            s.replay()
+            graphs[k % S].replay()
 
         with torch.cuda.stream(st):
             for k in range(8):
@@ -849,6 +848,7 @@ def run_stack_decode(stp, ctx, w, steps, world, local):
         misses = [int(m.item()) for m in s.r.mc]
         U = int(s.r.U.item())
         s.release()
+        del graphs
         # a few steps outside the graph with per-launch CUDA events
         stp.staple_trace_enable(ctx, True)
         with torch.cuda.stream(st):
@@ -870,7 +870,8 @@ def run_stack_decode(stp, ctx, w, steps, world, local):
             "weight_frac": wbytes / (step_ms * 1e-3) / 1e9 / peaks()["hbm_gbs"],
             "sm_mhz": clocks.get("sm_mhz"),
             "table_bytes_host": L * V * F * 2, "setup_s": setup_s,
-            "graph": "one CUDA graph per step: dedup, 4 group gathers on side streams, 16 layers",
+            "graph": ("one CUDA graph per step (one per recorded batch): the batch's ids and x "
+                      "copied in, dedup, 4 group gathers on side streams, 16 layers"),
             "clocks": clocks, "kernels_4_traced_steps": kern}
 
 

@@ -277,11 +277,14 @@ __global__ void __launch_bounds__(1024)
 // ---------------------------------------------------------------------------
 enum GatherMode { G_HITS = 0, G_MISSES = 1, G_LIST = 2, G_REFRESH = 3, G_SCATTER = 4 };
 
-// The work items are 2 KB chunks of rows (a warp's four 16-byte loads per
-// lane), in row-major order: with a few long rows (a decode step's misses,
-// 88 KB each for four grouped 7B layers) every warp of the grid still has one
-// in flight, where one warp per row would leave most of them idle and walk
-// each row one round trip at a time.
+// A warp copies a row, or, when there are fewer rows than warps, a 2 KB
+// chunk of one (its four 16-byte loads per lane), in row-major order: with a
+// few long rows (a decode step's misses, 88 KB each for four grouped 7B
+// layers) every warp of the grid then has one in flight, where one warp per
+// row would leave most of them idle and walk each row one round trip at a
+// time.  With many rows (a training batch's misses) each warp keeps its own
+// row: over the host link many rows in flight at once read faster than the
+// same bytes a few rows at a time.
 constexpr int kChunkVecs = 128;
 
 template <int MODE>
@@ -295,11 +298,12 @@ __global__ void __launch_bounds__(256)
   const int nw = (gridDim.x * blockDim.x) >> 5;
   const int n = *count_dev;
   const int64_t vecs = row_bytes / 16;
-  const int64_t cpr = (vecs + kChunkVecs - 1) / kChunkVecs;   // chunks per row
+  const int64_t cv = n < nw ? kChunkVecs : vecs;   // 16-byte vectors per work item
+  const int64_t cpr = (vecs + cv - 1) / cv;        // work items per row
   const int64_t items = int64_t(n) * cpr;
   for (int64_t it = gw; it < items; it += nw) {
     const int i = int(it / cpr);
-    const int64_t c0 = (it - int64_t(i) * cpr) * kChunkVecs;
+    const int64_t c0 = (it - int64_t(i) * cpr) * cv;
     int j;
     int64_t srow;
     if (MODE == G_HITS) {          // rows[j] = cache[slot[j]] for hits
@@ -322,17 +326,16 @@ __global__ void __launch_bounds__(256)
     }
     const uint4* sp = reinterpret_cast<const uint4*>(src + srow * src_pitch);
     uint4* dp = reinterpret_cast<uint4*>(rows + int64_t(j) * row_bytes);
-    const int64_t vend = c0 + kChunkVecs < vecs ? c0 + kChunkVecs : vecs;
+    const int64_t vend = c0 + cv < vecs ? c0 + cv : vecs;
     int64_t v = c0 + lane;
-    if (v + 96 < vend) {
+    for (; v + 96 < vend; v += 128) {
       const uint4 a0 = sp[v], a1 = sp[v + 32], a2 = sp[v + 64], a3 = sp[v + 96];
       dp[v] = a0;
       dp[v + 32] = a1;
       dp[v + 64] = a2;
       dp[v + 96] = a3;
-    } else {
-      for (; v < vend; v += 32) dp[v] = sp[v];
     }
+    for (; v < vend; v += 32) dp[v] = sp[v];
   }
 }
 

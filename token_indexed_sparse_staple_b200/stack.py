@@ -304,11 +304,21 @@ class DecodeStack:
                                None, None, self.ws, self.wsb, stream=st)
         st.wait_stream(self.pf)                    # join the prefetch streams (graph capture)
 
-    def capture(self, stream):
+    def capture(self, stream, ids_src=None, x_src=None):
+        """Record a step into a CUDA graph (kept for replay() and returned).
+        With ids_src / x_src the graph first copies them into ids_buf /
+        xs[0], so that a set of graphs feeds recorded inputs with no copy
+        outside the graphs."""
         import torch
-        self.graph = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(self.graph, stream=stream):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            if ids_src is not None:
+                self.ids_buf.copy_(ids_src)
+            if x_src is not None:
+                self.xs[0].copy_(x_src)
             self.run(stream)
+        self.graph = g
+        return g
 
     def replay(self):
         self.graph.replay()
