@@ -145,3 +145,41 @@ def test_decode_stack_graph_matches_oracle_per_layer(stp, ctx):
         s.release()
     finally:
         tables.close()
+
+
+def test_decode_stack_graphs_with_recorded_inputs(stp, ctx):
+    """One captured step graph per batch, each copying its own ids and x in
+    (capture with ids_src / x_src): replayed out of capture order, every
+    replay computes its own batch, checked per layer against the oracle."""
+    import torch
+
+    from token_indexed_sparse_staple_b200.stack import DecodeStack
+    L, G, T, D, F, V = 4, 4, 64, 128, 256, 1000
+    layers, groups = _stack_inputs(L, G, D, F, V)
+    freq = syn.calibration_freq(V, n_tokens=1 << 18)
+    W, tables = _build(stp, ctx, layers, groups, V, F, G, freq)
+    try:
+        s = DecodeStack(ctx, W, tables, T, D, F, V)
+        st = torch.cuda.Stream()
+        with torch.cuda.stream(st):
+            s.run(st)
+        torch.cuda.synchronize()
+        batches = [syn.zipf_ids(T, V, 1.1, seed=180 + k) for k in range(3)]
+        ids_src = [torch.from_numpy(b).cuda() for b in batches]
+        x_src = [dev(syn.bf16_normal((T, D), 1.0, 190 + k)[0], "bf16") for k in range(3)]
+        graphs = [s.capture(st, ids_src[k], x_src[k]) for k in range(3)]
+        for k in (2, 0, 1, 2):
+            with torch.cuda.stream(st):
+                graphs[k].replay()
+            torch.cuda.synchronize()
+            assert stp.staple_get_error(ctx) == 0
+            assert torch.equal(s.ids_buf, ids_src[k])
+            for l in range(L):
+                wg, wu, wd, E = (_f64b(a) for a in layers[l])
+                fw = oracle.ffn_forward(f64(s.xs[l]), batches[k], wg, wu, wd, E)
+                assert_close(f64(s.xs[l + 1]), fw["y"], TOL["bf16"], f"batch {k} y layer {l}")
+            np.testing.assert_array_equal(f64(s.xs[0]), f64(x_src[k]))
+        del graphs
+        s.release()
+    finally:
+        tables.close()
