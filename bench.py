@@ -609,10 +609,12 @@ def run_train(stp, ctx, w, steps, warmup, world, local):
 
     try:
         # The E-path and dense runs alternate in rounds of steps, so that both
-        # see the same clocks under the power cap; all of these steps run
+        # see the same clocks under the power cap, and the mode that goes
+        # first alternates from round to round (ABBA), so that a drift of the
+        # clock over the run does not favour either; all of these steps run
         # untraced.  (name, E path on, STEM, SMs the GEMMs leave to the
         # prefetch kernels)
-        rounds = 5 if steps >= 5 else 1
+        rounds = 10 if steps >= 10 else 1
         per = [steps // rounds + (1 if r < steps % rounds else 0) for r in range(rounds)]
         stp.staple_set_sm_reserve(ctx, 0)
         warm(True, False, 0)
@@ -624,7 +626,8 @@ def run_train(stp, ctx, w, steps, warmup, world, local):
             torch.cuda.synchronize()
             t0 = time.time()
             for r in range(rounds):
-                for mode, staple in (("staple_r0", True), ("dense", False)):
+                order = (("staple_r0", True), ("dense", False))
+                for mode, staple in (order if r % 2 == 0 else order[::-1]):
                     evs[mode].append(timed(staple, False, s_next, per[r]))
                     s_next += per[r] + 2
             torch.cuda.synchronize()
@@ -1204,7 +1207,8 @@ def main():
                 "ms_per_step": r3(st_ms), "dense_ms_per_step": r3(de_ms),
                 "e_path_overhead": r3((st_ms - de_ms) / de_ms), "steps": args.train_steps,
                 "sm_reserve": 0,
-                "timing": "E path and dense run alternated in rounds of steps, untraced",
+                "timing": ("E path and dense run alternated in 10 rounds of steps, the first mode "
+                           "alternating (ABBA), untraced"),
                 "ms_by_sm_reserve": {str(tr[m]["sm_reserve"]): r3(tr[m]["ms"] / args.train_steps)
                                      for m in ("staple_r0", "staple")},
                 "stem_ms_per_step": r3(tr["stem"]["ms"] / args.train_steps),
