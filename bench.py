@@ -354,49 +354,61 @@ def run_decode(stp, ctx, w, args, world, local):
     res["launches_per_step"] = sum(d["launches"] for d in kern.values()) / G
     # end to end through the public call with host buffers: every step copies
     # its x and ids in from pinned memory and its y out.  As a serving loop
-    # would, the copies run on two copy streams, double-buffered, so that a
-    # step's copies overlap its neighbours' layer calls, and the steps are
-    # captured in CUDA graphs of G steps like the kernel-only run.
+    # would, the copies run on two copy streams in chunks of C steps, with the
+    # device inputs and outputs double-buffered by chunk: chunk c's copies in
+    # overlap chunk c-1's layer calls and chunk c-1's copies out overlap
+    # chunk c's, and only the first call of a chunk waits on a copy, so the
+    # other calls follow one another as programmatic dependents.  The steps
+    # are captured in CUDA graphs of up to 512 steps (the first chunk's copies
+    # in and the last chunk's copies out of a graph are not overlapped).
     Ke = K
     h2d = st["x"][0].numel() * 2 + st["ids"][0].numel() * 4
     d2h = st["y"].numel() * 2
+    C = 16
     cin, cout = torch.cuda.Stream(), torch.cuda.Stream()
-    xd = [torch.empty_like(st["x"][0]) for _ in range(2)]
-    idd = [torch.empty_like(st["ids"][0]) for _ in range(2)]
-    yd = [torch.empty_like(st["y"]) for _ in range(2)]
-    embd = [stp.make_embed(stp.STAPLE_EMBED_TABLE, st["table"], w.F, idd[i], w.V) for i in range(2)]
+    xd = [torch.empty_like(st["x"][0]) for _ in range(2 * C)]
+    idd = [torch.empty_like(st["ids"][0]) for _ in range(2 * C)]
+    yd = [torch.empty_like(st["y"]) for _ in range(2 * C)]
+    embd = [stp.make_embed(stp.STAPLE_EMBED_TABLE, st["table"], w.F, idd[i], w.V)
+            for i in range(2 * C)]
     ev_in, ev_used, ev_out = ([torch.cuda.Event() for _ in range(2)] for _ in range(3))
 
-    def e2e_step(s):
-        i, r, b = s % 2, s % st["R"], s % st["S"]
-        cin.wait_event(ev_used[i])        # the call two steps back has read xd[i], idd[i]
+    def e2e_chunk(s0, n):
+        """Steps s0 .. s0+n-1 (n <= C), one chunk; buffers half (s0 // C) % 2."""
+        h = (s0 // C) % 2
+        cin.wait_event(ev_used[h])        # the chunk two back has read these inputs
         with torch.cuda.stream(cin):
-            xd[i].copy_(st["x_host"][b], non_blocking=True)
-            idd[i].copy_(st["ids_host"][b], non_blocking=True)
-        ev_in[i].record(cin)
-        stream.wait_event(ev_in[i])
-        stream.wait_event(ev_out[i])      # yd[i] of two steps back is on the host
-        stp.staple_ffn_fwd(ctx, stp.STAPLE_BF16, w.T, w.D, w.F, xd[i], embd[i], st["wg"][r],
-                           st["wu"][r], st["wd"][r], st["z"], yd[i], None, None, st["ws"],
-                           st["wsb"], stream=stream)
-        ev_used[i].record(stream)
-        cout.wait_event(ev_used[i])
+            for k in range(n):
+                b = (s0 + k) % st["S"]
+                xd[h * C + k].copy_(st["x_host"][b], non_blocking=True)
+                idd[h * C + k].copy_(st["ids_host"][b], non_blocking=True)
+        ev_in[h].record(cin)
+        stream.wait_event(ev_in[h])
+        stream.wait_event(ev_out[h])      # the chunk two back's outputs are on the host
+        for k in range(n):
+            r = (s0 + k) % st["R"]
+            stp.staple_ffn_fwd(ctx, stp.STAPLE_BF16, w.T, w.D, w.F, xd[h * C + k], embd[h * C + k],
+                               st["wg"][r], st["wu"][r], st["wd"][r], st["z"], yd[h * C + k],
+                               None, None, st["ws"], st["wsb"], stream=stream)
+        ev_used[h].record(stream)
+        cout.wait_event(ev_used[h])
         with torch.cuda.stream(cout):
-            st["y_host"][b].copy_(yd[i], non_blocking=True)
-        ev_out[i].record(cout)
+            for k in range(n):
+                st["y_host"][(s0 + k) % st["S"]].copy_(yd[h * C + k], non_blocking=True)
+        ev_out[h].record(cout)
 
     def e2e_graph(n):
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g, stream=stream):
             for e in ev_used + ev_out:     # fork the copy streams into the capture
                 e.record(stream)
-            for s in range(n):
-                e2e_step(s)
+            for s0 in range(0, n, C):
+                e2e_chunk(s0, min(C, n - s0))
             stream.wait_stream(cin)        # and join them before it ends
             stream.wait_stream(cout)
         return g
 
-    G = min(64, Ke)
+    G = min(512, Ke)
     full = e2e_graph(G)
     rem = e2e_graph(Ke % G) if Ke % G else None
     with torch.cuda.stream(stream):
@@ -1158,8 +1170,8 @@ def main():
                 "unit": "tokens/s", "h2d_bytes_per_step": dec["e2e"]["h2d"],
                 "d2h_bytes_per_step": dec["e2e"]["d2h"], "steps": dec["e2e"]["K"],
                 "how": ("per step: pinned H2D of x and ids on a copy stream, staple_ffn_fwd, "
-                        "D2H of y on another copy stream; double-buffered, steps in CUDA graphs "
-                        "of 64")},
+                        "D2H of y on another copy stream; copies in chunks of 16 steps, "
+                        "double-buffered by chunk, steps in CUDA graphs of 512")},
         "gpu_launches": int(round(dec["launches_per_step"] * K)),
         "clocks": dec["clocks"],
         "decode_dense": {"us_per_step": r3(dense_us), "us_per_step_staple": r3(step_us),
