@@ -1049,6 +1049,28 @@ def cpu_baseline_train(w, seconds=12.0, n=256):
                       f"{dt:.1f} s; extrapolated to the microbatch (cost linear in tokens)"}
 
 
+def cpu_baseline_stack_decode(w, seconds=8.0):
+    """The oracle's forward of one of the stack's layers on a whole decode
+    batch, repeated for ~seconds; a step runs w.layers such layers, so the
+    step's tokens/s is the layer's divided by the layer count (an
+    extrapolation: the cost is linear in layers)."""
+    one = syn.Workload(w.name + "-one-layer", T=w.T, D=w.D, F=w.F, V=w.V, layers=1,
+                       dtype="bf16", w_std=w.w_std, e_std=w.e_std, x_std=w.x_std,
+                       dy_std=w.dy_std, table="device", cache_frac=0.0, group=1, training=False)
+    batch = oracle_decode_batch(one)
+    reps = 0
+    t0 = time.time()
+    while time.time() - t0 < seconds or reps == 0:
+        oracle_decode_tokens(batch, w.T)
+        reps += 1
+    dt = time.time() - t0
+    return {"value": w.T * reps / (dt * w.layers), "unit": "tokens/s", "cores": blas_threads(),
+            "kind": "oracle",
+            "sample": f"{reps} forwards of one {w.D} x {w.F} layer on a {w.T}-token batch (fp64 "
+                      f"numpy oracle), {dt:.1f} s; extrapolated to {w.layers} layers (cost "
+                      f"linear in layers)"}
+
+
 def reference_arm(w, args, budget_s=60.0):
     """--impl reference: the oracle on the decode workload (same config, metric
     and step count as the CUDA arm).  A step is the oracle's forward of the
@@ -1257,6 +1279,18 @@ def main():
             except Exception as ex:  # the headline line must still print
                 line[key] = {"error": repr(ex)}
             release_pinned()
+        if world == 1 and rank == 0 and not args.no_cpu_baseline:
+            sd = line.get("stack_decode", {})
+            if "error" not in sd:
+                sd["cpu_baseline"] = cpu_baseline_stack_decode(syn.WORKLOADS["olmo2-7b-decode-16l"])
+            stt, tb = line.get("stack_train", {}), (train or {}).get("cpu_baseline")
+            if "error" not in stt and tb:
+                nl = syn.WORKLOADS["olmo2-1b-train-12l"].layers
+                stt["cpu_baseline"] = {
+                    "value": tb["value"] / nl, "unit": "tokens/s", "cores": tb["cores"],
+                    "kind": "oracle",
+                    "sample": f"the training layer's oracle sample ({tb['value']:.0f} tokens/s "
+                              f"fwd+bwd for one layer) over {nl} layers (cost linear in layers)"}
     if train is not None:
         line["train_layer"] = train   # last, so that a tail of the output holds it
     stp.staple_context_destroy(ctx)
