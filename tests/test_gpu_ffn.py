@@ -214,15 +214,17 @@ def test_bf16_decode_saves_g_and_h(stp, ctx):
 
 
 @pytest.mark.parametrize("D,F", [(2048, 1024), (1024, 8192), (4096, 11008), (4096, 1024),
-                                 (128, 192), (4352, 1024)])
+                                 (128, 192), (4352, 1024), (4032, 1024), (4416, 1024)])
 def test_bf16_decode_split_k_shapes(stp, ctx, D, F):
     """Both decode paths.  Two launches (the split-k sum in its own kernel):
     down tiles whose K is split over a few to many blocks (d_model 2048 and
     1024), d_ff 192 (fewer k units per down tile than a cluster has blocks),
-    d_model 4352 (more down tiles, 34, than clusters fit on the device at
-    once).  One launch in clusters (one cluster per down tile, the sum in
-    shared memory): d_model 4096 with d_ff 1024, and the 7B shape (d_ff
-    11008 = 172 gate/up tiles over 128 blocks, so some blocks make two)."""
+    d_model 4352 and 4416 (more down tiles, 34 and 35, than clusters fit on the
+    device at once; 4416 ends in a half tile of 64 rows).  One launch in
+    clusters (one cluster per down tile, the sum in shared memory): d_model
+    4096 and 4032 (32 tiles, the last of 64 rows) with d_ff 1024, and the 7B
+    shape (d_ff 11008 = 172 gate/up tiles over 128 blocks, so some blocks make
+    two)."""
     w = _bf16_workload(64, D, F, 2000)
     inp = syn.make_layer_inputs(w, with_dy=False)
     got = run_layer(stp, ctx, inp, w.D, w.F, w.V, embed="table", training=False)
