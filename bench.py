@@ -175,7 +175,7 @@ CAPTURED_TRAFFIC = {
                     ("token_indexed_sparse_staple_b200/csrc/ffn_tc.cu",
                      "// ---------------------------------------------------------------- decode",
                      "staple_status tc_ffn_fwd(")],
-        "sha256": "264d06806942323181ec84b5977a4d8d235d15407759d4e45b45e8ad32a8bd84",
+        "sha256": "cf520aacfa4d1fd5cff8432d22cd0ce2dd8c032b819af63ac5fdecb827823a73",
         "profile": "profiles/decode_fused_olmo2_1b_T64.md",
     },
 }

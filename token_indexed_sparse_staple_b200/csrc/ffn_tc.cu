@@ -314,7 +314,7 @@ staple_status tc_decode_fwd(const DeviceInfo& di, int T, int D, int F, const voi
                                  fused::decode_fused_kernel<false, true, true>},
                                 {fused::decode_fused_kernel<true, false, true>,
                                  fused::decode_fused_kernel<true, true, true>}}};
-  const int smem = fused::smem_bytes(pl.N, pl.sub, FT);
+  int smem = fused::smem_bytes(pl.N, pl.sub, FT);   // (the path's own rings: below)
   static std::atomic<uint64_t> attr_done{0};
   const uint64_t bit = uint64_t(1) << (di.device & 63);
   if (!(attr_done.load() & bit)) {
@@ -379,6 +379,14 @@ staple_status tc_decode_fwd(const DeviceInfo& di, int T, int D, int F, const voi
            pl.Dt * fused::kCluster >= pl.grid) ? 1 : 0;
   }
   const int grid = clu ? pl.Dt * fused::kCluster : pl.grid;
+  // the rings for the path taken: the most down units a block gets sets the
+  // activation ring's depth
+  {
+    const int upb = clu ? cdiv(pl.ud, fused::kCluster) : cdiv(pl.Ud, grid);
+    p.stages = fused::ring_stages(pl.N, pl.sub, FT, upb);
+    p.stages_b = fused::stages_b(pl.N, pl.sub, upb);
+    smem = fused::smem_bytes(pl.N, pl.sub, FT, upb);
+  }
   // down-step ordering only where some block makes two or more gate/up tiles
   const int order = pl.G > grid ? 1 : 0;
   const Kern kern = kerns[clu][order][stem ? 1 : 0];
