@@ -937,6 +937,7 @@ def run_stack_train(stp, ctx, w, steps, world, local):
                 ev0.record(st)
                 for _ in range(steps):
                     r = one()
+                st.wait_event(s.host_ready)   # the last step's dE rows are on the host
                 ev1.record(st)
             torch.cuda.synchronize()
             c1 = time.time()

@@ -78,6 +78,7 @@ def test_train_stack_matches_oracle_per_layer(stp, ctx, de_return):
             dyt = dev(syn.bf16_normal((T, D), 1.0, 70 + step)[0], "bf16")
             r = s.step(torch.from_numpy(ids).cuda(), x0, dyt,
                        next_ids=torch.from_numpy(nxt).cuda() if step == 0 else None)
+            s.host_ready.synchronize()   # this step's dE rows are in host memory
             torch.cuda.synchronize()
             assert stp.staple_get_error(ctx) == 0
             u_ref, _, _, _ = oracle.dedup(ids)

@@ -181,6 +181,7 @@ class TrainStack:
             ws=torch.zeros(max(wsb, 256), dtype=torch.uint8, device="cuda"), wsb=wsb)
         self.retr = [Retrieval(T, F, self.G, tables.n_groups) for _ in range(2)]
         self.pf, self.pf_side, self.copy = (torch.cuda.Stream() for _ in range(3))
+        self.host_ready = torch.cuda.Event()   # the last step's dE rows are in host memory
         self.step_no = 0
         self._primed = None   # (step, ids) whose dedup + group 0 are in flight
 
@@ -198,7 +199,10 @@ class TrainStack:
         during this step's backward; the next step then uses those ids (its
         own `ids` argument is not read again).  Returns the Retrieval used
         (its U_dev, unique ids and hit/miss maps stay valid until the step
-        after next)."""
+        after next).  The step's dE rows reach host memory when host_ready
+        completes (wait on it before reading host_dE): later work on `stream`,
+        such as the next step's forward, does not wait for the last layer's
+        copy-out, since no table optimizer runs between the steps here."""
         import torch
         st = stream or torch.cuda.current_stream()
         b, T, D, F = self.b, self.T, self.D, self.F
@@ -255,7 +259,7 @@ class TrainStack:
                                w.w_gate, w.w_up, dx, dwg, dwu, dwd, stream=st)
             dy = dx
         r.free.record(self.copy)                   # after the last reader (layer 0's copy-out)
-        st.wait_stream(self.copy)                  # the step ends when dE is on the host
+        self.host_ready.record(self.copy)
         self.step_no += 1
         return r
 
