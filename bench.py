@@ -1119,7 +1119,7 @@ def main():
     ap.add_argument("--no-train", action="store_true")
     ap.add_argument("--no-stacks", action="store_true")
     ap.add_argument("--stack-decode-steps", type=int, default=256)
-    ap.add_argument("--stack-train-steps", type=int, default=4)
+    ap.add_argument("--stack-train-steps", type=int, default=8)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--dw-down", action="store_true",
                     help="only time the training layer's dW_down GEMM (profiling case)")
